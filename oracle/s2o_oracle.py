@@ -1,0 +1,371 @@
+"""Plain fp64 CPU oracle for S2O's prefill hot path.
+
+TEST INFRASTRUCTURE ONLY. This module is the checker: only the test suite, the
+smoke check and the CPU-baseline leg of the benchmark import it. The product
+library never calls it and shares no code with it.
+
+Source: "S2O: Early Stopping for Sparse Attention via Online Permutation"
+(arXiv 2602.22575), as described on
+
+  * the pith.science page, "read the original abstract": keys are loaded in
+    a non-contiguous, importance-guided order given by an index list, blocks
+    are processed from high to low importance and processing stops once the
+    current block's score falls below a threshold;
+  * the gist.science technical summary (in French), section 1 "Permutation en
+    ligne via Chargement Guide par Index" (segment ranking: historical keys
+    are scored against a representative query of the segment, under a causal
+    mask; the physical K/V layout is kept and an index array drives the
+    loads), section 2 "Regle d'Arret Anticipe" (blocks in decreasing estimated
+    importance, stop once the block's marginal attention mass falls below
+    tau) and section 3 "Implementation du Noyau" (pass 1: dense causal window
+    of the segment; pass 2: historical keys in permuted order with the early
+    stop).
+
+The pages give no formulas.  Where they leave a step open, this oracle takes
+the following readings (the GPU library takes the same ones):
+
+  * representative query: the unweighted mean of the segment's query rows over
+    all query heads of the GQA group (query head h uses KV head h // G);
+  * score of key j: s_j = qbar . k_j / sqrt(d), natural exponent;
+  * admissible keys of segment s: A(s) = [0, e(s)), e(s) = min(N, Lq*(s+1));
+  * always kept: sinks [0, n_sink) and the window [max(0, Lq*s - W), e(s));
+  * candidates: the rest of A(s), i.e. [n_sink, Lq*s - W) when non-empty;
+  * order: candidates by s_j descending, ties to the lower index;
+  * blocks: Bk consecutive entries of that order (the last may be partial);
+  * block mass: m_b = sum_{j in b} exp(s_j - M) / Z, with M and Z the max and
+    the sum of exp(s_j - M) over all of A(s);
+  * stop: C = index of the first block with m_b < tau (that block is not
+    kept), or the number of blocks if none is below tau;
+  * attention: every row i of the segment, for every head of the group, gets
+    exact softmax attention over Keep(s) intersected with [0, i].
+
+All arithmetic is IEEE fp64 on inputs widened exactly from bf16.  Loops are
+plain; numpy's matmul, sort and sum are used as library steps only.  The
+oracle is single-threaded when its caller limits BLAS to one thread.
+"""
+from __future__ import annotations
+
+import math
+from dataclasses import dataclass, field
+
+import numpy as np
+
+NEAR_TIE_REL = 1e-6  # relative width of the near-tie bands for scores and masses
+
+
+@dataclass(frozen=True)
+class Params:
+    """Method constants.  Defaults are the library's compiled specialisation."""
+
+    Lq: int = 128          # query-segment length
+    Bk: int = 64           # stopping granularity (keys per block)
+    n_sink: int = 64       # sink tokens [0, n_sink) are always kept
+    window_prev: int = 128  # keys before the segment that are always kept
+    tau: float = 1e-3      # stopping threshold on block mass
+
+
+# ---------------------------------------------------------------------------
+# bf16 handling (the oracle's own; inputs arrive as raw bf16 bit patterns)
+# ---------------------------------------------------------------------------
+
+def widen_bf16(bits: np.ndarray) -> np.ndarray:
+    """Exact bf16 -> fp64: a bf16 value is the top half of an fp32 word."""
+    if bits.dtype != np.uint16:
+        raise TypeError("expected raw bf16 bits as uint16")
+    f32 = (bits.astype(np.uint32) << np.uint32(16)).view(np.float32)
+    return f32.astype(np.float64)
+
+
+def _f64(x: np.ndarray) -> np.ndarray:
+    if x.dtype == np.uint16:
+        return widen_bf16(x)
+    return np.asarray(x, dtype=np.float64)
+
+
+# ---------------------------------------------------------------------------
+# Segment geometry
+# ---------------------------------------------------------------------------
+
+def num_segments(N: int, p: Params) -> int:
+    return (N + p.Lq - 1) // p.Lq
+
+
+def segment_rows(N: int, s: int, p: Params) -> tuple[int, int]:
+    return p.Lq * s, min(N, p.Lq * (s + 1))
+
+
+def admissible_end(N: int, s: int, p: Params) -> int:
+    """e(s): keys [0, e(s)) are causally admissible for segment s."""
+    return min(N, p.Lq * (s + 1))
+
+
+def window_start(s: int, p: Params) -> int:
+    return max(0, p.Lq * s - p.window_prev)
+
+
+def candidate_range(N: int, s: int, p: Params) -> tuple[int, int]:
+    """[lo, hi) of the candidate keys: A(s) minus sinks and window."""
+    lo, hi = p.n_sink, window_start(s, p)
+    if hi <= lo:
+        return lo, lo
+    return lo, hi
+
+
+def num_candidates(N: int, s: int, p: Params) -> int:
+    lo, hi = candidate_range(N, s, p)
+    return hi - lo
+
+
+def candidate_offsets(N: int, p: Params) -> np.ndarray:
+    """off[s] = sum of |Cand(t)| for t < s; off[S] = total per (b, kvh)."""
+    S = num_segments(N, p)
+    off = np.zeros(S + 1, dtype=np.int64)
+    for s in range(S):
+        off[s + 1] = off[s] + num_candidates(N, s, p)
+    return off
+
+
+def num_blocks(n_cand: int, p: Params) -> int:
+    return (n_cand + p.Bk - 1) // p.Bk
+
+
+def always_kept(N: int, s: int, p: Params) -> np.ndarray:
+    """Sinks union window, ascending."""
+    e = admissible_end(N, s, p)
+    sinks = set(range(0, min(p.n_sink, e)))
+    window = set(range(window_start(s, p), e))
+    return np.array(sorted(sinks | window), dtype=np.int64)
+
+
+# ---------------------------------------------------------------------------
+# Plan: pooled query, scores, (M, Z), order, block masses, stop
+# ---------------------------------------------------------------------------
+
+@dataclass
+class SegmentPlan:
+    s: int
+    qbar: np.ndarray            # [d]
+    scores: np.ndarray          # [e(s)] s_j for every admissible key
+    M: float
+    Z: float
+    order: np.ndarray           # candidate indices, importance order
+    masses: np.ndarray          # [n_blocks]
+    C: int                      # kept candidate blocks
+    score_ties: np.ndarray      # positions p with |sigma_p - sigma_{p+1}| <= tol
+    mass_ties: np.ndarray       # blocks b with |m_b - tau| <= 1e-6 tau
+    tie_tol: float = 0.0
+    keep: np.ndarray = field(default=None)  # Keep(s), ascending
+
+
+def pooled_query(Qf: np.ndarray, b: int, kvh: int, s: int, G: int, p: Params) -> np.ndarray:
+    """qbar = mean over the group's G query heads and the segment's rows."""
+    N = Qf.shape[2]
+    r0, r1 = segment_rows(N, s, p)
+    acc = np.zeros(Qf.shape[3], dtype=np.float64)
+    count = 0
+    for g in range(G):
+        h = kvh * G + g
+        for i in range(r0, r1):
+            acc += _f64(Qf[b, h, i])
+            count += 1
+    return acc / count
+
+
+def key_scores(qbar: np.ndarray, Kf: np.ndarray, b: int, kvh: int, e: int) -> np.ndarray:
+    """s_j = qbar . k_j / sqrt(d) for j in [0, e)."""
+    d = Kf.shape[3]
+    K = _f64(Kf[b, kvh, :e])
+    return (K @ qbar) / math.sqrt(d)
+
+
+def plan_segment(Qf, Kf, b: int, kvh: int, s: int, G: int, p: Params) -> SegmentPlan:
+    N = Kf.shape[2]
+    e = admissible_end(N, s, p)
+    qbar = pooled_query(Qf, b, kvh, s, G, p)
+    sc = key_scores(qbar, Kf, b, kvh, e)
+    if not np.all(np.isfinite(sc)):
+        raise ValueError("non-finite score")
+    M = float(np.max(sc))
+    Z = float(np.sum(np.exp(sc - M)))
+
+    lo, hi = candidate_range(N, s, p)
+    cand = np.arange(lo, hi, dtype=np.int64)
+    cs = sc[lo:hi]
+    # order by (-s_j, j): lexsort's last key is the primary one
+    order = cand[np.lexsort((cand, -cs))] if hi > lo else cand
+
+    w = np.exp(sc[order] - M) / Z
+    nb = num_blocks(hi - lo, p)
+    masses = np.array([w[k * p.Bk:(k + 1) * p.Bk].sum() for k in range(nb)], dtype=np.float64)
+    C = nb
+    for k in range(nb):
+        if masses[k] < p.tau:
+            C = k
+            break
+
+    tol = NEAR_TIE_REL * float(np.max(np.abs(sc)))
+    srt = sc[order]
+    score_ties = np.nonzero(np.abs(srt[:-1] - srt[1:]) <= tol)[0] if len(srt) > 1 else np.zeros(0, np.int64)
+    mass_ties = np.nonzero(np.abs(masses - p.tau) <= NEAR_TIE_REL * p.tau)[0]
+
+    keep = keep_set(N, s, order, C, p)
+    return SegmentPlan(s=s, qbar=qbar, scores=sc, M=M, Z=Z, order=order, masses=masses, C=C,
+                       score_ties=score_ties, mass_ties=mass_ties, tie_tol=tol, keep=keep)
+
+
+def plan(Qf, Kf, p: Params, segments=None):
+    """Plan of every (b, kvh, s), in the library's packed layout.
+
+    Returns dict with
+      scores   [B, Hkv, T]  candidate scores, candidate-position order
+      perm     [B, Hkv, T]  candidate indices in importance order (absolute)
+      nblocks  [B, Hkv, S]  kept candidate blocks C(s)
+      seg_stats[B, Hkv, S, 2]  (M, Z)
+      plans    {(b, kvh, s): SegmentPlan}
+    where T = sum_s |Cand(s)| and segment s occupies [off[s], off[s+1]).
+    With `segments` given, only those segments are planned (other entries of
+    the packed arrays are left at -1 / nan).
+    """
+    B, Hq, N, d = Qf.shape
+    Hkv = Kf.shape[1]
+    G = Hq // Hkv
+    S = num_segments(N, p)
+    off = candidate_offsets(N, p)
+    T = int(off[-1])
+    scores = np.full((B, Hkv, T), np.nan)
+    perm = np.full((B, Hkv, T), -1, dtype=np.int64)
+    nblocks = np.full((B, Hkv, S), -1, dtype=np.int64)
+    stats = np.full((B, Hkv, S, 2), np.nan)
+    plans = {}
+    segs = range(S) if segments is None else segments
+    for b in range(B):
+        for kvh in range(Hkv):
+            for s in segs:
+                sp = plan_segment(Qf, Kf, b, kvh, s, G, p)
+                lo, hi = candidate_range(N, s, p)
+                scores[b, kvh, off[s]:off[s + 1]] = sp.scores[lo:hi]
+                perm[b, kvh, off[s]:off[s + 1]] = sp.order
+                nblocks[b, kvh, s] = sp.C
+                stats[b, kvh, s] = (sp.M, sp.Z)
+                plans[(b, kvh, s)] = sp
+    return dict(scores=scores, perm=perm, nblocks=nblocks, seg_stats=stats, plans=plans, offsets=off)
+
+
+def keep_set(N: int, s: int, perm_seg: np.ndarray, C: int, p: Params) -> np.ndarray:
+    """Keep(s) = sinks U window U first C*Bk entries of the segment's order."""
+    n = len(perm_seg)
+    return np.union1d(always_kept(N, s, p), np.asarray(perm_seg[:min(C * p.Bk, n)], dtype=np.int64))
+
+
+# ---------------------------------------------------------------------------
+# Attention over a kept set
+# ---------------------------------------------------------------------------
+
+def attention_segment(Qf, Kf, Vf, b: int, kvh: int, s: int, G: int, keep: np.ndarray,
+                      p: Params, phys_of_logical: np.ndarray | None = None) -> np.ndarray:
+    """Exact softmax attention of the segment's rows over keep intersected with [0, i].
+
+    Returns [G, rows, d].  Keys are addressed through an index list: logical key
+    j is read from physical row phys_of_logical[j] (identity when None).  This is
+    the "virtual to physical" loading of the pages; the causal mask and the kept
+    set use logical positions.
+    Softmax is two-pass per row: the maximum first, then the normalised sum.
+    """
+    N, d = Qf.shape[2], Qf.shape[3]
+    r0, r1 = segment_rows(N, s, p)
+    keep = np.asarray(keep, dtype=np.int64)
+    phys = keep if phys_of_logical is None else np.asarray(phys_of_logical)[keep]
+    Kk = _f64(Kf[b, kvh][phys])
+    Vk = _f64(Vf[b, kvh][phys])
+    out = np.zeros((G, r1 - r0, d))
+    rows = np.arange(r0, r1)
+    visible = keep[None, :] <= rows[:, None]
+    for g in range(G):
+        Qs = _f64(Qf[b, kvh * G + g, r0:r1])
+        S = (Qs @ Kk.T) / math.sqrt(d)
+        S = np.where(visible, S, -np.inf)
+        m = S.max(axis=1, keepdims=True)
+        P = np.exp(S - m)
+        ell = P.sum(axis=1, keepdims=True)
+        out[g] = (P @ Vk) / ell
+    return out
+
+
+def dense_segment(Qf, Kf, Vf, b: int, kvh: int, s: int, G: int, p: Params) -> np.ndarray:
+    """Causal attention of the segment's rows over every admissible key."""
+    N = Qf.shape[2]
+    keep = np.arange(0, admissible_end(N, s, p), dtype=np.int64)
+    return attention_segment(Qf, Kf, Vf, b, kvh, s, G, keep, p)
+
+
+def attention(Qf, Kf, Vf, perm, nblocks, p: Params, segments=None, offsets=None):
+    """Sparse prefill output O[B, Hq, N, d] (fp64) for the given plan.
+
+    perm / nblocks in the packed layout of `plan`.  Rows of segments not listed
+    in `segments` are left at nan.
+    """
+    B, Hq, N, d = Qf.shape
+    Hkv = Kf.shape[1]
+    G = Hq // Hkv
+    S = num_segments(N, p)
+    off = candidate_offsets(N, p) if offsets is None else offsets
+    O = np.full((B, Hq, N, d), np.nan)
+    segs = range(S) if segments is None else segments
+    for b in range(B):
+        for kvh in range(Hkv):
+            for s in segs:
+                keep = keep_set(N, s, perm[b, kvh, off[s]:off[s + 1]], int(nblocks[b, kvh, s]), p)
+                r0, r1 = segment_rows(N, s, p)
+                O[b, kvh * G:(kvh + 1) * G, r0:r1] = attention_segment(Qf, Kf, Vf, b, kvh, s, G, keep, p)
+    return O
+
+
+def dense_attention(Qf, Kf, Vf, p: Params, segments=None):
+    B, Hq, N, d = Qf.shape
+    Hkv = Kf.shape[1]
+    G = Hq // Hkv
+    S = num_segments(N, p)
+    O = np.full((B, Hq, N, d), np.nan)
+    segs = range(S) if segments is None else segments
+    for b in range(B):
+        for kvh in range(Hkv):
+            for s in segs:
+                r0, r1 = segment_rows(N, s, p)
+                O[b, kvh * G:(kvh + 1) * G, r0:r1] = dense_segment(Qf, Kf, Vf, b, kvh, s, G, p)
+    return O
+
+
+# ---------------------------------------------------------------------------
+# Contiguous top-k comparator (block-sparse baseline at matched block count)
+# ---------------------------------------------------------------------------
+
+def contiguous_plan_segment(sp: SegmentPlan, N: int, C_match: int, p: Params) -> np.ndarray:
+    """Kept tokens of the block-granular comparator for one segment.
+
+    The candidates are cut into blocks of Bk keys in their original order; each
+    block is ranked by its pooled-softmax mass sum exp(s_j - M) / Z (ties to
+    the lower block); the top C_match blocks are kept.  Returns the kept blocks'
+    token indices, block by block in rank order, each block ascending, followed
+    by the remaining candidate blocks in rank order.
+    """
+    lo, hi = candidate_range(N, sp.s, p)
+    nb = num_blocks(hi - lo, p)
+    w = np.exp(sp.scores[lo:hi] - sp.M) / sp.Z
+    bm = np.array([w[k * p.Bk:(k + 1) * p.Bk].sum() for k in range(nb)])
+    rank = np.lexsort((np.arange(nb), -bm))
+    out = [np.arange(lo + k * p.Bk, min(hi, lo + (k + 1) * p.Bk)) for k in rank]
+    return np.concatenate(out).astype(np.int64) if out else np.zeros(0, np.int64)
+
+
+# ---------------------------------------------------------------------------
+# Measurement definitions
+# ---------------------------------------------------------------------------
+
+def kept_pairs_segment(N: int, s: int, keep: np.ndarray, p: Params) -> int:
+    """Number of (row, key) pairs computed for one head: sum_i |Keep(s) cap [0, i]|."""
+    r0, r1 = segment_rows(N, s, p)
+    keep = np.sort(np.asarray(keep))
+    total = 0
+    for i in range(r0, r1):
+        total += int(np.searchsorted(keep, i, side="right"))
+    return total

@@ -1,0 +1,370 @@
+"""Pins of the fp64 oracle against facts that do not come from the oracle itself.
+
+Each test checks one part of the method (pooling, scores, order, masses, stop,
+attention) against a closed form, an invariant, a library routine or a
+brute-force evaluation on a tiny input.
+"""
+import json
+import math
+import os
+
+import numpy as np
+import pytest
+import torch
+
+from oracle import s2o_oracle as O
+from score_keys_pooled_b200 import synth
+
+GOLDEN = os.path.join(os.path.dirname(__file__), "golden")
+E = math.e
+
+
+def _ev(expr: str) -> float:
+    return float(eval(expr, {"__builtins__": {}}, {"e": E}))
+
+
+def _bits(x):
+    return synth.to_bf16_bits(np.asarray(x, dtype=np.float32))
+
+
+# ---------------------------------------------------------------------------
+# bf16 widening
+# ---------------------------------------------------------------------------
+
+def test_widen_bf16_known_patterns():
+    bits = np.array([0x3F80, 0xC000, 0x0001, 0x7F7F, 0x0000, 0x8000, 0x3EAB], dtype=np.uint16)
+    got = O.widen_bf16(bits)
+    want = [1.0, -2.0, 2.0 ** -133, (2 - 2 ** -7) * 2.0 ** 127, 0.0, -0.0, 0.333984375]
+    assert list(got) == want
+
+
+# ---------------------------------------------------------------------------
+# geometry
+# ---------------------------------------------------------------------------
+
+def test_candidate_offsets_closed_form_default_params():
+    # with Lq=128, W=128, n_sink=64 and N a multiple of 128:
+    # |Cand(s)| = max(0, 128 s - 192) and off(s) = 64 (s-2)^2 for s >= 2
+    p = O.Params()
+    N = 128 * 40
+    off = O.candidate_offsets(N, p)
+    for s in range(41):
+        want = 64 * (s - 2) ** 2 if s >= 2 else 0
+        assert off[s] == want
+    for s in range(40):
+        assert O.num_candidates(N, s, p) == max(0, 128 * s - 192)
+
+
+def test_sets_partition_admissible_keys():
+    p = O.Params(Lq=4, Bk=2, n_sink=1, window_prev=4)
+    for N in (1, 3, 8, 13, 16):
+        for s in range(O.num_segments(N, p)):
+            e = O.admissible_end(N, s, p)
+            lo, hi = O.candidate_range(N, s, p)
+            kept = set(O.always_kept(N, s, p).tolist())
+            cand = set(range(lo, hi))
+            assert kept.isdisjoint(cand)
+            assert kept | cand == set(range(e))
+
+
+# ---------------------------------------------------------------------------
+# pooling and scores
+# ---------------------------------------------------------------------------
+
+def test_pooled_query_closed_form_and_group_mapping():
+    # head g of group 1 has row i = (g+1) * ((i - r0) mod 16) in dim 0 (bf16-exact);
+    # the mean over G=4 heads and 128 rows is (1+2+3+4) * 8 * (0+...+15) / 512
+    p = O.Params()
+    B, Hkv, G, N, d = 1, 2, 4, 256, 8
+    Q = np.zeros((B, Hkv * G, N, d), dtype=np.float32)
+    Q[:, 0:4] = 1000.0  # group 0 must not leak into group 1
+    for g in range(G):
+        for i in range(128, 256):
+            Q[0, 4 + g, i, 0] = (g + 1) * ((i - 128) % 16)
+            Q[0, 4 + g, i, 3] = -1.0
+    qb = O.pooled_query(_bits(Q), 0, 1, 1, G, p)
+    want0 = (1 + 2 + 3 + 4) * 8 * 120 / 512
+    assert qb[0] == want0
+    assert qb[3] == -1.0
+    assert np.all(qb[[1, 2, 4, 5, 6, 7]] == 0.0)
+
+
+def test_scores_one_hot_keys_are_exact():
+    p = O.Params(Lq=4, Bk=2, n_sink=1, window_prev=0)
+    d = 16
+    N = 8
+    a = np.array([0, 1, -3, 2, 0.5, 7, -1, 4], dtype=np.float32)
+    K = np.zeros((1, 1, N, d), dtype=np.float32)
+    K[0, 0, :, 5] = a
+    Q = np.zeros((1, 1, N, d), dtype=np.float32)
+    Q[0, 0, 4:8, 5] = 3.0
+    sp = O.plan_segment(_bits(Q), _bits(K), 0, 0, 1, 1, p)
+    assert np.array_equal(sp.scores, 3.0 * a.astype(np.float64) / 4.0)
+
+
+# ---------------------------------------------------------------------------
+# hand-worked two-segment examples (tests/golden/hand_two_segment.json)
+# ---------------------------------------------------------------------------
+
+def _golden_case(case):
+    sh = case["shape"]
+    Q = np.zeros((sh["B"], sh["Hq"], sh["N"], sh["d"]), dtype=np.float32)
+    if "Q_rows_dim0" in case:
+        for i, v in case["Q_rows_dim0"].items():
+            Q[0, :, int(i), 0] = v
+    for h, rows in case.get("Q_rows_dim0_by_head", {}).items():
+        for i, v in rows.items():
+            Q[0, int(h), int(i), 0] = v
+    K = np.zeros((sh["B"], sh["Hkv"], sh["N"], sh["d"]), dtype=np.float32)
+    K[0, 0, :, 0] = case["K_dim0"]
+    V = np.zeros_like(K)
+    V[0, 0, :, 0] = case["V_dim0"]
+    V[0, 0, :, 1] = case["V_dim1_all"]
+    return _bits(Q), _bits(K), _bits(V)
+
+
+def _load_golden():
+    with open(os.path.join(GOLDEN, "hand_two_segment.json")) as f:
+        return json.load(f)
+
+
+@pytest.mark.parametrize("ci", [0, 1])
+def test_hand_worked_plans(ci):
+    g = _load_golden()
+    case = g["cases"][ci]
+    Q, K, V = _golden_case(case)
+    for stop in case["stops"]:
+        p = O.Params(tau=stop["tau"], **case["params"])
+        res = O.plan(Q, K, p)
+        for seg in case["segments"]:
+            sp = res["plans"][(0, 0, seg["s"])]
+            assert sp.order.tolist() == seg["order"]
+            assert sp.M == pytest.approx(_ev(seg["M"]), rel=0, abs=1e-14)
+            assert sp.Z == pytest.approx(_ev(seg["Z"]), rel=1e-14)
+            want_m = [_ev(x) for x in seg["masses"]]
+            assert np.allclose(sp.masses, want_m, rtol=1e-13, atol=0)
+        assert res["nblocks"][0, 0].tolist() == stop["C"]
+
+
+def test_hand_worked_outputs():
+    g = _load_golden()
+    case = g["cases"][0]
+    Q, K, V = _golden_case(case)
+    p = O.Params(tau=0.2, **case["params"])
+    res = O.plan(Q, K, p)
+    out = O.attention(Q, K, V, res["perm"], res["nblocks"], p)
+    for i, (x0, x1) in case["outputs_tau_0.2"]["rows"].items():
+        row = out[0, 0, int(i)]
+        assert row[0] == pytest.approx(_ev(x0), rel=1e-14, abs=1e-15)
+        assert row[1] == pytest.approx(_ev(x1), rel=1e-14)
+        assert np.all(row[2:] == 0)
+
+
+def test_hand_worked_contiguous_comparator():
+    g = _load_golden()
+    spec = g["contiguous"]
+    case = [c for c in g["cases"] if c["name"] == spec["case"]][0]
+    Q, K, V = _golden_case(case)
+    p = O.Params(tau=0.2, **case["params"])
+    sp = O.plan_segment(Q, K, 0, 0, spec["s"], 1, p)
+    full = O.contiguous_plan_segment(sp, case["shape"]["N"], spec["C_match"], p)
+    assert full.tolist() == spec["expected_full"]
+    assert full[:spec["C_match"] * p.Bk].tolist() == spec["expected_prefix"]
+
+
+# ---------------------------------------------------------------------------
+# all-ties closed form: Q = 0 makes every score exactly 0
+# ---------------------------------------------------------------------------
+
+# tau = 0.0625 = 64/1024 hits the mass of the e(s)=1024 segment exactly (a power
+# of two, so the fp64 sum is exact): a block whose mass equals tau is kept.
+@pytest.mark.parametrize("tau", [0.0, 1e-3, 0.05, 0.0625, 0.07, 2.0])
+def test_all_ties_closed_form(tau):
+    p = O.Params(tau=tau)
+    B, Hq, Hkv, N, d = 1, 2, 1, 1024, 128
+    rng = np.random.default_rng(5)
+    Q = np.zeros((B, Hq, N, d), dtype=np.uint16)
+    K = _bits(rng.standard_normal((B, Hkv, N, d)))
+    res = O.plan(Q, K, p)
+    for s in range(O.num_segments(N, p)):
+        sp = res["plans"][(0, 0, s)]
+        e = O.admissible_end(N, s, p)
+        lo, hi = O.candidate_range(N, s, p)
+        assert sp.M == 0.0 and sp.Z == float(e)
+        assert sp.order.tolist() == list(range(lo, hi))
+        nb = O.num_blocks(hi - lo, p)
+        assert np.allclose(sp.masses, 64.0 / e, rtol=1e-14, atol=0)
+        want_C = nb if 64.0 / e >= tau else 0
+        assert sp.C == want_C
+        if e == 1024 and tau == 0.0625:
+            assert nb > 0 and sp.C == nb and np.all(sp.masses == tau)
+        # every adjacent pair is an exact tie
+        assert len(sp.score_ties) == max(0, hi - lo - 1)
+
+
+# ---------------------------------------------------------------------------
+# invariants on random inputs
+# ---------------------------------------------------------------------------
+
+def _random_case(seed, B=1, Hq=4, Hkv=1, N=768, d=64, planted=True):
+    Q, K, V = synth.generate(B, Hq, Hkv, N, d, planted=planted, band=d >= 32, n_stripe=6, seed=seed)
+    return Q, K, V
+
+
+def test_masses_sum_to_one_and_are_nonincreasing():
+    p = O.Params(tau=1e-3)
+    Q, K, V = _random_case(1)
+    N = Q.shape[2]
+    res = O.plan(Q, K, p)
+    for s in range(O.num_segments(N, p)):
+        sp = res["plans"][(0, 0, s)]
+        always = O.always_kept(N, s, p)
+        rest = np.exp(sp.scores[always] - sp.M).sum() / sp.Z
+        assert sp.masses.sum() + rest == pytest.approx(1.0, abs=1e-12)
+        assert np.all(np.diff(sp.masses) <= 0)
+        # the stop rule: every kept block is >= tau, the first dropped one < tau
+        assert np.all(sp.masses[:sp.C] >= p.tau)
+        if sp.C < len(sp.masses):
+            assert sp.masses[sp.C] < p.tau
+
+
+def test_order_is_sorted_with_index_tiebreak():
+    p = O.Params()
+    Q, K, V = _random_case(2)
+    res = O.plan(Q, K, p)
+    N = Q.shape[2]
+    for s in range(O.num_segments(N, p)):
+        sp = res["plans"][(0, 0, s)]
+        sc = sp.scores[sp.order]
+        for a in range(len(sc) - 1):
+            assert sc[a] > sc[a + 1] or (sc[a] == sc[a + 1] and sp.order[a] < sp.order[a + 1])
+
+
+def test_tau_zero_equals_library_causal_attention():
+    # tau = 0 keeps every block, so the output must be plain causal attention;
+    # torch's scaled_dot_product_attention in fp64 is the independent reference.
+    p = O.Params(tau=0.0)
+    Q, K, V = _random_case(3, Hq=4, Hkv=2, N=640, d=64)
+    res = O.plan(Q, K, p)
+    N = Q.shape[2]
+    for s in range(O.num_segments(N, p)):
+        lo, hi = O.candidate_range(N, s, p)
+        assert res["nblocks"][0, 0, s] == O.num_blocks(hi - lo, p)
+    out = O.attention(Q, K, V, res["perm"], res["nblocks"], p)
+    G = 2
+    q = torch.from_numpy(O.widen_bf16(Q))
+    k = torch.from_numpy(O.widen_bf16(K)).repeat_interleave(G, dim=1)
+    v = torch.from_numpy(O.widen_bf16(V)).repeat_interleave(G, dim=1)
+    ref = torch.nn.functional.scaled_dot_product_attention(q, k, v, is_causal=True).numpy()
+    assert np.max(np.abs(out - ref)) < 1e-12
+
+
+def test_output_invariant_under_physical_permutation():
+    # Keys are addressed through an index list; storing K/V rows in another
+    # physical order and remapping the indices must not change the output.
+    p = O.Params(tau=3e-3)
+    Q, K, V = _random_case(4, Hq=2, Hkv=1, N=896, d=64)
+    N = Q.shape[2]
+    res = O.plan(Q, K, p)
+    rng = np.random.default_rng(11)
+    pi = rng.permutation(N)            # logical j lives at physical row pi[j]
+    Kp = np.empty_like(K)
+    Vp = np.empty_like(V)
+    Kp[:, :, pi] = K
+    Vp[:, :, pi] = V
+    off = res["offsets"]
+    for s in (0, 1, 3, 6):
+        keep = O.keep_set(N, s, res["perm"][0, 0, off[s]:off[s + 1]], int(res["nblocks"][0, 0, s]), p)
+        a = O.attention_segment(Q, K, V, 0, 0, s, 2, keep, p)
+        b = O.attention_segment(Q, Kp, Vp, 0, 0, s, 2, keep, p, phys_of_logical=pi)
+        assert np.max(np.abs(a - b)) <= 1e-12
+
+
+def test_near_tie_reporting():
+    p = O.Params(Lq=4, Bk=2, n_sink=1, window_prev=0, tau=0.3)
+    N, d = 8, 4
+    K = np.zeros((1, 1, N, d), dtype=np.float32)
+    K[0, 0, :, 0] = [0, 1, 1, 2, 0, 0, 0, 0]  # keys 1 and 2 tie exactly
+    Q = np.zeros((1, 1, N, d), dtype=np.float32)
+    Q[0, 0, 4:, 0] = 2.0
+    sp = O.plan_segment(_bits(Q), _bits(K), 0, 0, 1, 1, p)
+    assert sp.order.tolist() == [3, 1, 2]
+    assert sp.score_ties.tolist() == [1]
+
+
+# ---------------------------------------------------------------------------
+# brute force on N = 16
+# ---------------------------------------------------------------------------
+
+def _brute_force(Qv, Kv, Vv, G, Lq, Bk, n_sink, W, tau):
+    """Plain-Python evaluation of the method on a tiny input (lists and math)."""
+    B, Hq, N, d = len(Qv), len(Qv[0]), len(Qv[0][0]), len(Qv[0][0][0])
+    Hkv = Hq // G
+    out = [[[[0.0] * d for _ in range(N)] for _ in range(Hq)] for _ in range(B)]
+    Cs = {}
+    S = -(-N // Lq)
+    for b in range(B):
+        for kv in range(Hkv):
+            for s in range(S):
+                rows = list(range(Lq * s, min(N, Lq * s + Lq)))
+                e = rows[-1] + 1
+                qbar = [sum(Qv[b][kv * G + g][i][c] for g in range(G) for i in rows) / (G * len(rows))
+                        for c in range(d)]
+                sc = [sum(qbar[c] * Kv[b][kv][j][c] for c in range(d)) / math.sqrt(d) for j in range(e)]
+                Mx = max(sc)
+                Zs = sum(math.exp(x - Mx) for x in sc)
+                w0 = max(0, Lq * s - W)
+                always = set(range(min(n_sink, e))) | set(range(w0, e))
+                cand = [j for j in range(e) if j not in always]
+                order = sorted(cand, key=lambda j: (-sc[j], j))
+                blocks = [order[k:k + Bk] for k in range(0, len(order), Bk)]
+                mass = [sum(math.exp(sc[j] - Mx) for j in blk) / Zs for blk in blocks]
+                # C = the largest c such that each of the first c blocks has mass >= tau
+                C = 0
+                while C < len(blocks) and all(mass[t] >= tau for t in range(C + 1)):
+                    C += 1
+                Cs[(b, kv, s)] = C
+                keep = always | {j for blk in blocks[:C] for j in blk}
+                for g in range(G):
+                    h = kv * G + g
+                    for i in rows:
+                        vis = [j for j in range(i + 1) if j in keep]
+                        logits = [sum(Qv[b][h][i][c] * Kv[b][kv][j][c] for c in range(d)) / math.sqrt(d)
+                                  for j in vis]
+                        mx = max(logits)
+                        ws = [math.exp(x - mx) for x in logits]
+                        tot = sum(ws)
+                        for c in range(d):
+                            out[b][h][i][c] = sum(wj * Vv[b][kv][j][c] for wj, j in zip(ws, vis)) / tot
+    return out, Cs
+
+
+@pytest.mark.parametrize("tau", [0.0, 0.05, 0.2])
+def test_brute_force_n16(tau):
+    p = O.Params(Lq=4, Bk=2, n_sink=1, window_prev=4, tau=tau)
+    rng = np.random.default_rng(7)
+    B, Hq, Hkv, N, d = 1, 2, 1, 16, 8
+    Q = _bits(rng.standard_normal((B, Hq, N, d)) * 1.5)
+    K = _bits(rng.standard_normal((B, Hkv, N, d)) * 1.5)
+    V = _bits(rng.standard_normal((B, Hkv, N, d)))
+    res = O.plan(Q, K, p)
+    out = O.attention(Q, K, V, res["perm"], res["nblocks"], p)
+    bf, Cs = _brute_force(O.widen_bf16(Q).tolist(), O.widen_bf16(K).tolist(), O.widen_bf16(V).tolist(),
+                          2, 4, 2, 1, 4, tau)
+    for (b, kv, s), C in Cs.items():
+        assert res["nblocks"][b, kv, s] == C
+    assert np.max(np.abs(out - np.array(bf))) < 1e-12
+    if tau > 0:
+        # the threshold must actually bind somewhere for the test to mean something
+        full = [O.num_blocks(O.num_candidates(N, s, p), p) for s in range(4)]
+        assert any(res["nblocks"][0, 0, s] < full[s] for s in range(4))
+
+
+def test_kept_pairs_dense_closed_form():
+    p = O.Params(tau=0.0)
+    N = 512
+    total = 0
+    for s in range(O.num_segments(N, p)):
+        keep = np.arange(O.admissible_end(N, s, p))
+        total += O.kept_pairs_segment(N, s, keep, p)
+    assert total == N * (N + 1) // 2
