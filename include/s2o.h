@@ -1,0 +1,205 @@
+/*
+ * s2o.h -- C ABI of the S2O sparse-prefill library for NVIDIA B200 (sm_100a).
+ *
+ * S2O ("S2O: Early Stopping for Sparse Attention via Online Permutation",
+ * arXiv 2602.22575) splits causal prefill attention into
+ *
+ *   plan       for every (batch b, KV head kvh, query segment s of Lq rows):
+ *              pool the segment's queries into one vector, score every
+ *              causally admissible key against it, sort the non-local keys
+ *              by score into an index list (the "online permutation": no
+ *              K/V data moves), cut the list into blocks of Bk keys and stop
+ *              at the first block whose estimated softmax mass is below tau;
+ *   attention  exact online-softmax attention of every row of the segment
+ *              over the kept keys: sinks, the local window and the kept
+ *              blocks, gathered by index.
+ *
+ * Sources on the pages (no formulas are given there):
+ *   - pith.science page, "read the original abstract": index-guided loading
+ *     of non-contiguous tokens, blocks from high to low importance, stop once
+ *     the current block score falls below a threshold;
+ *   - gist.science technical summary, section 1 "Permutation en ligne via
+ *     Chargement Guide par Index" (segment ranking, representative query,
+ *     causal mask, index arrays over an unchanged HBM layout), section 2
+ *     "Regle d'Arret Anticipe" (stop on marginal mass below tau) and section 3
+ *     "Implementation du Noyau" (pass 1: dense causal window; pass 2: keys in
+ *     permuted order with the early stop).
+ *
+ * The rule this library fixes where the pages are silent:
+ *   qbar(b,kvh,s) = mean of Q[b, kvh*G + g, i, :] over the G = Hq/Hkv heads of
+ *                   the group and the rows i of segment s;
+ *   s_j           = qbar . k_j / sqrt(d) for j in A(s) = [0, e(s)),
+ *                   e(s) = min(N, Lq*(s+1));
+ *   always kept   sinks [0, n_sink) and window [max(0, Lq*s - W), e(s));
+ *   candidates    Cand(s) = [n_sink, Lq*s - W) (empty when Lq*s - W <= n_sink);
+ *   order         candidates by s_j descending, ties to the lower index;
+ *   block mass    m_b = sum_{j in block b} exp(s_j - M) / Z, M = max_{A(s)} s_j,
+ *                 Z = sum_{A(s)} exp(s_j - M);
+ *   stop          C(s) = first b with m_b < tau, else the number of blocks;
+ *   attention     O[b,h,i,:] = softmax_j(q_i . k_j / sqrt(d)) V over
+ *                 j in Keep(s) intersected with [0, i],
+ *                 Keep(s) = sinks U window U perm[0 : Bk*C(s)].
+ *
+ * Compiled specialisation: Lq = 128, Bk = 64, n_sink = 64, W = 128, d = 128.
+ * Other values return S2O_ERR_UNSUPPORTED_SHAPE.  N may be any positive size
+ * (the last segment may be partial); with these constants every candidate
+ * block is full, |Cand(s)| = max(0, 128 s - 192).
+ *
+ * Layouts (all row-major, contiguous, device memory unless stated):
+ *   Q  [B, Hq,  N, d]  bf16 (raw 16-bit patterns)
+ *   K  [B, Hkv, N, d]  bf16
+ *   V  [B, Hkv, N, d]  bf16
+ *   O  [B, Hq,  N, d]  bf16 or fp32 (out_dtype)
+ *   scores [B, Hkv, T] fp32  candidate scores in candidate order: segment s
+ *                            occupies [off(s), off(s+1)), entry k is key
+ *                            n_sink + k; T = s2o_num_candidates(), off(s) =
+ *                            s2o_candidate_offset()
+ *   perm   [B, Hkv, T] int32 absolute key indices, same packing; within a
+ *                            segment the importance order (full list)
+ *   nblocks   [B, Hkv, S] int32  C(s)
+ *   seg_stats [B, Hkv, S, 2] fp32  (M, Z), may be NULL
+ * Pointers must be 16-byte aligned.  Query head h reads KV head h / (Hq/Hkv).
+ *
+ * Ownership: the caller allocates every buffer, including the plan workspace
+ * (size from s2o_plan_workspace_size).  The library never allocates device
+ * memory and keeps only one piece of global state per device: a 32-bit
+ * device error word (see s2o_last_device_error).
+ *
+ * Execution: every call except s2o_prefill_host and s2o_last_device_error is
+ * asynchronous on the given stream (NULL = the legacy default stream) and
+ * returns after argument checks and kernel launches.  Argument errors are
+ * reported before anything is launched; launch failures map to S2O_ERR_CUDA.
+ * Errors found on the device (non-finite input, an out-of-range index in a
+ * caller-supplied plan, a bounded wait that ran out) set the device error
+ * word; outputs of that call are then unspecified.
+ */
+#ifndef S2O_H
+#define S2O_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef struct CUstream_st* s2o_stream_t; /* a cudaStream_t */
+
+typedef struct s2o_config {
+  int32_t B, Hq, Hkv, N, d;
+  int32_t Lq;          /* query segment length (128) */
+  int32_t Bk;          /* keys per block, the stopping granularity (64) */
+  int32_t n_sink;      /* always-kept sink tokens [0, n_sink) (64) */
+  int32_t window_prev; /* always-kept keys before the segment (128) */
+  double tau;          /* stop threshold on block mass, >= 0 */
+} s2o_config;
+
+typedef enum s2o_status {
+  S2O_OK = 0,
+  S2O_ERR_INVALID_ARG = 1,         /* null pointer, bad size, misalignment */
+  S2O_ERR_UNSUPPORTED_SHAPE = 2,   /* constants other than the compiled ones */
+  S2O_ERR_WORKSPACE_TOO_SMALL = 3,
+  S2O_ERR_CUDA = 4,                /* a CUDA runtime call or launch failed */
+  S2O_ERR_DEVICE_TIMEOUT = 5,      /* a bounded device wait ran out */
+  S2O_ERR_NONFINITE = 6,           /* Inf/NaN in Q or K, or a non-finite score */
+  S2O_ERR_BAD_PLAN = 7             /* perm/nblocks out of range in s2o_attention */
+} s2o_status;
+
+enum { S2O_OUT_BF16 = 0, S2O_OUT_F32 = 1 };
+
+/* Number of query segments S = ceil(N / Lq).  Returns -1 on a bad config. */
+int32_t s2o_num_segments(const s2o_config* cfg);
+
+/* T = sum over segments of |Cand(s)| (per (b, kvh)).  -1 on a bad config. */
+int64_t s2o_num_candidates(const s2o_config* cfg);
+
+/* off(s) = sum_{t < s} |Cand(t)|, 0 <= s <= S.  -1 on a bad config or s. */
+int64_t s2o_candidate_offset(const s2o_config* cfg, int32_t s);
+
+/* Bytes of device workspace s2o_plan needs for this config. */
+s2o_status s2o_plan_workspace_size(const s2o_config* cfg, size_t* bytes);
+
+/*
+ * s2o_plan -- pooled scores, importance order and stop point of every
+ * segment (the pages' preprocessing / index generation: pith.science
+ * abstract; gist.science technical summary, sections 1 and 2).
+ *   Q, K       device bf16 inputs (layouts above)
+ *   scores     out, device fp32 [B,Hkv,T]
+ *   perm       out, device int32 [B,Hkv,T]
+ *   nblocks    out, device int32 [B,Hkv,S]
+ *   seg_stats  out, device fp32 [B,Hkv,S,2] or NULL
+ *   workspace  device scratch of at least s2o_plan_workspace_size() bytes,
+ *              256-byte aligned; its contents need no initialisation
+ */
+s2o_status s2o_plan(const s2o_config* cfg, const uint16_t* Q, const uint16_t* K,
+                    float* scores, int32_t* perm, int32_t* nblocks, float* seg_stats,
+                    void* workspace, size_t workspace_bytes, s2o_stream_t stream);
+
+/*
+ * s2o_plan_contiguous -- block-granular comparator at a matched block count:
+ * the candidates of each segment are cut into Bk-key blocks in their
+ * original order, ranked by pooled mass sum exp(s_j - M) / Z (ties to the
+ * lower block) and the first nblocks_match[b,kvh,s] blocks of that ranking
+ * are the kept set.  This is the block-sparse baseline whose intra-block
+ * redundancy the pages describe (gist.science technical summary, "Enonce du
+ * Probleme"); it feeds s2o_attention unchanged, with nblocks_match as its
+ * nblocks.
+ *   scores, seg_stats  device inputs from s2o_plan (seg_stats required)
+ *   nblocks_match      device int32 [B,Hkv,S]
+ *   perm_out           out, device int32 [B,Hkv,T]: ranked blocks, each
+ *                      block's keys ascending
+ */
+s2o_status s2o_plan_contiguous(const s2o_config* cfg, const float* scores, const float* seg_stats,
+                               const int32_t* nblocks_match, int32_t* perm_out, s2o_stream_t stream);
+
+/*
+ * s2o_attention -- sparse prefill output over Keep(s) (gist.science technical
+ * summary, section 3 "Implementation du Noyau": pass 1 = the segment's dense
+ * causal window, pass 2 = keys in permuted order up to the stop point).
+ *   Q, K, V    device bf16 inputs
+ *   perm       device int32 [B,Hkv,T] (s2o_plan or s2o_plan_contiguous)
+ *   nblocks    device int32 [B,Hkv,S], 0 <= nblocks <= |Cand(s)| / Bk
+ *   O          out, device [B,Hq,N,d], bf16 (S2O_OUT_BF16) or fp32 (S2O_OUT_F32)
+ * Every perm entry read must lie in Cand(s); violations are clamped, set the
+ * device error word (S2O_ERR_BAD_PLAN) and leave O unspecified.
+ */
+s2o_status s2o_attention(const s2o_config* cfg, const uint16_t* Q, const uint16_t* K,
+                         const uint16_t* V, const int32_t* perm, const int32_t* nblocks,
+                         void* O, int32_t out_dtype, s2o_stream_t stream);
+
+/* Device bytes s2o_prefill_host needs in its arena. */
+s2o_status s2o_prefill_arena_size(const s2o_config* cfg, int32_t out_dtype, size_t* bytes);
+
+/*
+ * s2o_prefill_host -- the whole path from HOST buffers: copies Q, K, V to
+ * the device arena, plans, runs the attention and copies O back to host O.
+ * Host buffers should be page-locked for full copy speed.  The arena is
+ * caller-allocated device memory of s2o_prefill_arena_size() bytes, 256-byte
+ * aligned.  Synchronises the stream before returning and reports device
+ * errors of this call (like s2o_last_device_error).
+ *   nblocks_host  optional host int32 [B,Hkv,S] copy of C(s), or NULL
+ */
+s2o_status s2o_prefill_host(const s2o_config* cfg, const uint16_t* Q_host, const uint16_t* K_host,
+                            const uint16_t* V_host, void* O_host, int32_t out_dtype,
+                            int32_t* nblocks_host, void* arena, size_t arena_bytes,
+                            s2o_stream_t stream);
+
+/* Static description of a status code. */
+const char* s2o_status_string(s2o_status st);
+
+/*
+ * Synchronises `stream`, reads and clears the current device's error word and
+ * maps it to a status (S2O_OK when no device error was recorded).  The word
+ * is shared by every stream of the device.
+ */
+s2o_status s2o_last_device_error(s2o_stream_t stream);
+
+/* Number of kernels the last s2o_plan / s2o_attention / s2o_plan_contiguous
+ * call on this thread launched (the library's own kernels only). */
+int32_t s2o_last_launch_count(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* S2O_H */

@@ -1,0 +1,187 @@
+"""S2O sparse prefill attention for B200: thin Python binding of libs2o.so.
+
+The functions below only marshal arguments (torch tensors -> device pointers,
+the current CUDA stream) into the C ABI declared in include/s2o.h; every step
+of the method runs in the library's CUDA kernels.  There is no CPU fallback:
+if the compiled library is missing, importing the binding's entry points
+raises.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import re
+
+PKG = os.path.dirname(os.path.abspath(__file__))
+ROOT = os.path.dirname(PKG)
+LIB_PATH = os.path.join(PKG, "libs2o.so")
+HEADER = os.path.join(ROOT, "include", "s2o.h")
+
+OUT_BF16, OUT_F32 = 0, 1
+
+STATUS = {
+    0: "S2O_OK", 1: "S2O_ERR_INVALID_ARG", 2: "S2O_ERR_UNSUPPORTED_SHAPE",
+    3: "S2O_ERR_WORKSPACE_TOO_SMALL", 4: "S2O_ERR_CUDA", 5: "S2O_ERR_DEVICE_TIMEOUT",
+    6: "S2O_ERR_NONFINITE", 7: "S2O_ERR_BAD_PLAN",
+}
+
+
+class S2OError(RuntimeError):
+    def __init__(self, code: int, what: str):
+        super().__init__(f"{what}: {STATUS.get(code, code)}")
+        self.code = code
+
+
+class Config(ctypes.Structure):
+    _fields_ = [("B", ctypes.c_int32), ("Hq", ctypes.c_int32), ("Hkv", ctypes.c_int32),
+                ("N", ctypes.c_int32), ("d", ctypes.c_int32), ("Lq", ctypes.c_int32),
+                ("Bk", ctypes.c_int32), ("n_sink", ctypes.c_int32), ("window_prev", ctypes.c_int32),
+                ("tau", ctypes.c_double)]
+
+
+def make_config(B, Hq, Hkv, N, d=128, tau=1e-3, Lq=128, Bk=64, n_sink=64, window_prev=128) -> Config:
+    return Config(B, Hq, Hkv, N, d, Lq, Bk, n_sink, window_prev, float(tau))
+
+
+_lib = None
+_P = ctypes.c_void_p
+_CFG = ctypes.POINTER(Config)
+
+
+def lib() -> ctypes.CDLL:
+    """The loaded CUDA library (built in-tree by score_keys_pooled_b200.build)."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(LIB_PATH):
+            raise ImportError(f"{LIB_PATH} is not built; run `python -m score_keys_pooled_b200.build`")
+        L = ctypes.CDLL(LIB_PATH)
+        L.s2o_num_segments.argtypes = [_CFG]
+        L.s2o_num_segments.restype = ctypes.c_int32
+        L.s2o_num_candidates.argtypes = [_CFG]
+        L.s2o_num_candidates.restype = ctypes.c_int64
+        L.s2o_candidate_offset.argtypes = [_CFG, ctypes.c_int32]
+        L.s2o_candidate_offset.restype = ctypes.c_int64
+        L.s2o_plan_workspace_size.argtypes = [_CFG, ctypes.POINTER(ctypes.c_size_t)]
+        L.s2o_plan.argtypes = [_CFG, _P, _P, _P, _P, _P, _P, _P, ctypes.c_size_t, _P]
+        L.s2o_plan_contiguous.argtypes = [_CFG, _P, _P, _P, _P, _P]
+        L.s2o_attention.argtypes = [_CFG, _P, _P, _P, _P, _P, _P, ctypes.c_int32, _P]
+        L.s2o_prefill_arena_size.argtypes = [_CFG, ctypes.c_int32, ctypes.POINTER(ctypes.c_size_t)]
+        L.s2o_prefill_host.argtypes = [_CFG, _P, _P, _P, _P, ctypes.c_int32, _P, _P, ctypes.c_size_t, _P]
+        L.s2o_status_string.argtypes = [ctypes.c_int]
+        L.s2o_status_string.restype = ctypes.c_char_p
+        L.s2o_last_device_error.argtypes = [_P]
+        L.s2o_last_launch_count.restype = ctypes.c_int32
+        for name in ("s2o_plan_workspace_size", "s2o_plan", "s2o_plan_contiguous", "s2o_attention",
+                     "s2o_prefill_arena_size", "s2o_prefill_host", "s2o_last_device_error"):
+            getattr(L, name).restype = ctypes.c_int
+        _lib = L
+    return _lib
+
+
+def header_functions() -> list[str]:
+    """Names of the functions include/s2o.h declares."""
+    text = open(HEADER).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(s2o_[a-z_0-9]+)\s*\(", text)))
+
+
+def _check(code: int, what: str):
+    if code != 0:
+        raise S2OError(code, what)
+
+
+def _stream(stream=None):
+    import torch
+    s = torch.cuda.current_stream() if stream is None else stream
+    return ctypes.c_void_p(s.cuda_stream)
+
+
+def _ptr(t):
+    return ctypes.c_void_p(t.data_ptr()) if t is not None else None
+
+
+def num_segments(cfg: Config) -> int:
+    return lib().s2o_num_segments(ctypes.byref(cfg))
+
+
+def num_candidates(cfg: Config) -> int:
+    return lib().s2o_num_candidates(ctypes.byref(cfg))
+
+
+def candidate_offset(cfg: Config, s: int) -> int:
+    return lib().s2o_candidate_offset(ctypes.byref(cfg), s)
+
+
+def plan_workspace_size(cfg: Config) -> int:
+    n = ctypes.c_size_t(0)
+    _check(lib().s2o_plan_workspace_size(ctypes.byref(cfg), ctypes.byref(n)), "s2o_plan_workspace_size")
+    return n.value
+
+
+def prefill_arena_size(cfg: Config, out_dtype: int = OUT_BF16) -> int:
+    n = ctypes.c_size_t(0)
+    _check(lib().s2o_prefill_arena_size(ctypes.byref(cfg), out_dtype, ctypes.byref(n)), "s2o_prefill_arena_size")
+    return n.value
+
+
+def alloc_plan(cfg: Config, device="cuda", workspace=True):
+    """Device buffers for one s2o_plan call (allocated by torch)."""
+    import torch
+    BH = cfg.B * cfg.Hkv
+    S, T = num_segments(cfg), num_candidates(cfg)
+    out = dict(
+        scores=torch.empty(BH * T + 4, dtype=torch.float32, device=device),
+        perm=torch.empty(BH * T + 4, dtype=torch.int32, device=device),
+        nblocks=torch.empty(BH * S, dtype=torch.int32, device=device),
+        seg_stats=torch.empty(BH * S * 2, dtype=torch.float32, device=device),
+    )
+    if workspace:
+        out["workspace"] = torch.empty(plan_workspace_size(cfg), dtype=torch.uint8, device=device)
+    return out
+
+
+def plan(cfg: Config, Q, K, bufs=None, stream=None):
+    """Run s2o_plan; returns the buffer dict (scores, perm, nblocks, seg_stats)."""
+    bufs = alloc_plan(cfg, Q.device) if bufs is None else bufs
+    ws = bufs["workspace"]
+    _check(lib().s2o_plan(ctypes.byref(cfg), _ptr(Q), _ptr(K), _ptr(bufs["scores"]), _ptr(bufs["perm"]),
+                          _ptr(bufs["nblocks"]), _ptr(bufs.get("seg_stats")), _ptr(ws), ws.numel(),
+                          _stream(stream)), "s2o_plan")
+    return bufs
+
+
+def plan_contiguous(cfg: Config, scores, seg_stats, nblocks_match, perm_out, stream=None):
+    _check(lib().s2o_plan_contiguous(ctypes.byref(cfg), _ptr(scores), _ptr(seg_stats), _ptr(nblocks_match),
+                                     _ptr(perm_out), _stream(stream)), "s2o_plan_contiguous")
+    return perm_out
+
+
+def attention(cfg: Config, Q, K, V, perm, nblocks, O=None, out_dtype: int = OUT_BF16, stream=None):
+    import torch
+    if O is None:
+        O = torch.empty(Q.shape, dtype=torch.bfloat16 if out_dtype == OUT_BF16 else torch.float32,
+                        device=Q.device)
+    _check(lib().s2o_attention(ctypes.byref(cfg), _ptr(Q), _ptr(K), _ptr(V), _ptr(perm), _ptr(nblocks),
+                               _ptr(O), out_dtype, _stream(stream)), "s2o_attention")
+    return O
+
+
+def prefill_host(cfg: Config, Q_host, K_host, V_host, O_host, arena, nblocks_host=None,
+                 out_dtype: int = OUT_BF16, stream=None):
+    """Whole path from host tensors (pinned for speed) through the C ABI."""
+    _check(lib().s2o_prefill_host(ctypes.byref(cfg), _ptr(Q_host), _ptr(K_host), _ptr(V_host), _ptr(O_host),
+                                  out_dtype, _ptr(nblocks_host), _ptr(arena), arena.numel(), _stream(stream)),
+           "s2o_prefill_host")
+    return O_host
+
+
+def last_device_error(stream=None) -> int:
+    return lib().s2o_last_device_error(_stream(stream))
+
+
+def last_launch_count() -> int:
+    return lib().s2o_last_launch_count()
+
+
+def status_string(code: int) -> str:
+    return lib().s2o_status_string(code).decode()

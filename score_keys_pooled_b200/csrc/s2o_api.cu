@@ -1,0 +1,276 @@
+// C ABI of the S2O library: argument checks, workspace layout and launches.
+// Everything that computes runs in the kernels of pool_score.cuh,
+// seg_sort.cuh and sparse_attn.cuh.
+#include <cmath>
+#include <cstring>
+#include <mutex>
+
+#include "s2o.h"
+#include "s2o_common.cuh"
+#include "pool_score.cuh"
+#include "seg_sort.cuh"
+#include "sparse_attn.cuh"
+
+using namespace s2o;
+
+namespace {
+
+thread_local int32_t t_launches = 0;
+
+constexpr int kMaxN = 1 << 19;  // bounds the S x S partial-statistics table
+
+inline bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+inline size_t round256(size_t x) { return (x + 255) & ~size_t(255); }
+
+s2o_status check_cfg(const s2o_config* c) {
+  if (!c) return S2O_ERR_INVALID_ARG;
+  if (c->B <= 0 || c->Hq <= 0 || c->Hkv <= 0 || c->N <= 0 || c->d <= 0) return S2O_ERR_INVALID_ARG;
+  if (c->Hq % c->Hkv) return S2O_ERR_INVALID_ARG;
+  if (!std::isfinite(c->tau) || c->tau < 0) return S2O_ERR_INVALID_ARG;
+  if (c->d != kD || c->Lq != kLq || c->Bk != kBk || c->n_sink != kSink || c->window_prev != kWin)
+    return S2O_ERR_UNSUPPORTED_SHAPE;
+  if (c->N > kMaxN) return S2O_ERR_UNSUPPORTED_SHAPE;
+  if ((int64_t)c->B * c->Hkv > 65535 || (int64_t)c->B * c->Hq > 65535) return S2O_ERR_UNSUPPORTED_SHAPE;
+  return S2O_OK;
+}
+
+int32_t nseg(const s2o_config* c) { return (c->N + kLq - 1) / kLq; }
+int64_t ncand_total(const s2o_config* c) { return cand_offset(nseg(c)); }
+
+struct PlanWs {
+  float* qbar;
+  float2* part;
+  float* segM;
+  double* segZ;
+  uint32_t *keyA, *keyB, *valA, *valB;
+  size_t bytes;
+};
+
+PlanWs plan_layout(const s2o_config* c, void* base) {
+  const size_t BH = (size_t)c->B * c->Hkv, S = (size_t)nseg(c), T = (size_t)ncand_total(c);
+  PlanWs w{};
+  size_t off = 0;
+  auto take = [&](size_t bytes) {
+    uint8_t* p = static_cast<uint8_t*>(base) + off;
+    off += round256(bytes);
+    return static_cast<void*>(p);
+  };
+  w.qbar = static_cast<float*>(take(BH * S * kD * sizeof(float)));
+  w.part = static_cast<float2*>(take(BH * S * S * sizeof(float2)));
+  w.segM = static_cast<float*>(take(BH * S * sizeof(float)));
+  w.segZ = static_cast<double*>(take(BH * S * sizeof(double)));
+  w.keyA = static_cast<uint32_t*>(take(BH * T * 4 + 16));
+  w.keyB = static_cast<uint32_t*>(take(BH * T * 4 + 16));
+  w.valA = static_cast<uint32_t*>(take(BH * T * 4 + 16));
+  w.valB = static_cast<uint32_t*>(take(BH * T * 4 + 16));
+  w.bytes = off;
+  return w;
+}
+
+std::once_flag g_attr_once;
+cudaError_t g_attr_err = cudaSuccess;
+
+cudaError_t set_kernel_attributes() {
+  std::call_once(g_attr_once, [] {
+    cudaError_t e = cudaFuncSetAttribute(k_score, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kScoreSmem);
+    if (e == cudaSuccess)
+      e = cudaFuncSetAttribute(k_sparse_attn, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kAttnSmem);
+    if (e == cudaSuccess)
+      e = cudaFuncSetAttribute(k_contig_plan, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                               (int)(kContigMaxBlocks * sizeof(unsigned long long)));
+    g_attr_err = e;
+  });
+  return g_attr_err;
+}
+
+s2o_status launch_status() {
+  return cudaGetLastError() == cudaSuccess ? S2O_OK : S2O_ERR_CUDA;
+}
+
+}  // namespace
+
+extern "C" {
+
+int32_t s2o_num_segments(const s2o_config* cfg) {
+  if (check_cfg(cfg) != S2O_OK) return -1;
+  return nseg(cfg);
+}
+
+int64_t s2o_num_candidates(const s2o_config* cfg) {
+  if (check_cfg(cfg) != S2O_OK) return -1;
+  return ncand_total(cfg);
+}
+
+int64_t s2o_candidate_offset(const s2o_config* cfg, int32_t s) {
+  if (check_cfg(cfg) != S2O_OK || s < 0 || s > nseg(cfg)) return -1;
+  return cand_offset(s);
+}
+
+s2o_status s2o_plan_workspace_size(const s2o_config* cfg, size_t* bytes) {
+  s2o_status st = check_cfg(cfg);
+  if (st != S2O_OK) return st;
+  if (!bytes) return S2O_ERR_INVALID_ARG;
+  *bytes = plan_layout(cfg, nullptr).bytes;
+  return S2O_OK;
+}
+
+s2o_status s2o_plan(const s2o_config* cfg, const uint16_t* Q, const uint16_t* K, float* scores, int32_t* perm,
+                    int32_t* nblocks, float* seg_stats, void* workspace, size_t workspace_bytes,
+                    s2o_stream_t stream) {
+  t_launches = 0;
+  s2o_status st = check_cfg(cfg);
+  if (st != S2O_OK) return st;
+  if (!Q || !K || !scores || !perm || !nblocks || !workspace) return S2O_ERR_INVALID_ARG;
+  if (!aligned16(Q) || !aligned16(K) || !aligned16(scores) || !aligned16(perm) || !aligned16(nblocks) ||
+      (seg_stats && !aligned16(seg_stats)) || (reinterpret_cast<uintptr_t>(workspace) & 255u))
+    return S2O_ERR_INVALID_ARG;
+  const PlanWs w = plan_layout(cfg, workspace);
+  if (workspace_bytes < w.bytes) return S2O_ERR_WORKSPACE_TOO_SMALL;
+  if (set_kernel_attributes() != cudaSuccess) return S2O_ERR_CUDA;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  const int S = nseg(cfg);
+  const int BH = cfg->B * cfg->Hkv;
+  const int64_t T = ncand_total(cfg);
+
+  k_pool<<<dim3(S, BH), 256, 0, s>>>(Q, w.qbar, cfg->Hq, cfg->Hkv, cfg->N, S);
+  ++t_launches;
+  const int ntiles = (cfg->N + kScoreKeys - 1) / kScoreKeys;
+  const int nchunks = (S + kScoreSegs - 1) / kScoreSegs;
+  k_score<<<dim3(ntiles, nchunks, BH), 256, kScoreSmem, s>>>(K, w.qbar, scores, w.part, cfg->Hkv, cfg->N, S, T);
+  ++t_launches;
+  const int nwarps = BH * S;
+  k_seg_stats<<<(nwarps * 32 + 255) / 256, 256, 0, s>>>(w.part, w.segM, w.segZ, seg_stats, BH, S);
+  ++t_launches;
+  k_sort<<<BH * S, kSortThreads, 0, s>>>(scores, w.segM, w.segZ, w.keyA, w.keyB, w.valA, w.valB, perm, nblocks,
+                                         BH, S, T, cfg->tau);
+  ++t_launches;
+  return launch_status();
+}
+
+s2o_status s2o_plan_contiguous(const s2o_config* cfg, const float* scores, const float* seg_stats,
+                               const int32_t* nblocks_match, int32_t* perm_out, s2o_stream_t stream) {
+  t_launches = 0;
+  s2o_status st = check_cfg(cfg);
+  if (st != S2O_OK) return st;
+  if (!scores || !seg_stats || !nblocks_match || !perm_out) return S2O_ERR_INVALID_ARG;
+  if (!aligned16(scores) || !aligned16(seg_stats) || !aligned16(perm_out)) return S2O_ERR_INVALID_ARG;
+  if (set_kernel_attributes() != cudaSuccess) return S2O_ERR_CUDA;
+  const int S = nseg(cfg);
+  const int BH = cfg->B * cfg->Hkv;
+  int P = 1;
+  while (P < (int)(num_cand(S - 1) / kBk)) P <<= 1;
+  if (P > kContigMaxBlocks) return S2O_ERR_UNSUPPORTED_SHAPE;
+  (void)nblocks_match;  // the ranking covers every block; attention reads the first nblocks_match
+  k_contig_plan<<<BH * S, 1024, P * sizeof(unsigned long long), reinterpret_cast<cudaStream_t>(stream)>>>(
+      scores, seg_stats, perm_out, BH, S, ncand_total(cfg));
+  ++t_launches;
+  return launch_status();
+}
+
+s2o_status s2o_attention(const s2o_config* cfg, const uint16_t* Q, const uint16_t* K, const uint16_t* V,
+                         const int32_t* perm, const int32_t* nblocks, void* O, int32_t out_dtype,
+                         s2o_stream_t stream) {
+  t_launches = 0;
+  s2o_status st = check_cfg(cfg);
+  if (st != S2O_OK) return st;
+  if (!Q || !K || !V || !perm || !nblocks || !O) return S2O_ERR_INVALID_ARG;
+  if (out_dtype != S2O_OUT_BF16 && out_dtype != S2O_OUT_F32) return S2O_ERR_INVALID_ARG;
+  if (!aligned16(Q) || !aligned16(K) || !aligned16(V) || !aligned16(O) || !aligned16(perm))
+    return S2O_ERR_INVALID_ARG;
+  if (set_kernel_attributes() != cudaSuccess) return S2O_ERR_CUDA;
+  AttnArgs a;
+  a.Q = Q; a.K = K; a.V = V; a.perm = perm; a.nblocks = nblocks; a.O = O;
+  a.B = cfg->B; a.Hq = cfg->Hq; a.Hkv = cfg->Hkv; a.N = cfg->N; a.S = nseg(cfg);
+  a.T = ncand_total(cfg);
+  a.out_f32 = out_dtype == S2O_OUT_F32;
+  const int64_t ncta = (int64_t)cfg->B * cfg->Hq * a.S;
+  k_sparse_attn<<<(unsigned)ncta, kAttnThreads, kAttnSmem, reinterpret_cast<cudaStream_t>(stream)>>>(a);
+  ++t_launches;
+  return launch_status();
+}
+
+s2o_status s2o_prefill_arena_size(const s2o_config* cfg, int32_t out_dtype, size_t* bytes) {
+  s2o_status st = check_cfg(cfg);
+  if (st != S2O_OK) return st;
+  if (!bytes || (out_dtype != S2O_OUT_BF16 && out_dtype != S2O_OUT_F32)) return S2O_ERR_INVALID_ARG;
+  const size_t q = (size_t)cfg->B * cfg->Hq * cfg->N * kD, kv = (size_t)cfg->B * cfg->Hkv * cfg->N * kD;
+  const size_t T = (size_t)cfg->B * cfg->Hkv * ncand_total(cfg), S = (size_t)cfg->B * cfg->Hkv * nseg(cfg);
+  size_t ws = 0;
+  s2o_plan_workspace_size(cfg, &ws);
+  *bytes = round256(q * 2) + 2 * round256(kv * 2) + round256(q * (out_dtype == S2O_OUT_F32 ? 4 : 2)) +
+           round256(T * 4 + 16) * 2 + round256(S * 4) + ws;
+  return S2O_OK;
+}
+
+s2o_status s2o_prefill_host(const s2o_config* cfg, const uint16_t* Q_host, const uint16_t* K_host,
+                            const uint16_t* V_host, void* O_host, int32_t out_dtype, int32_t* nblocks_host,
+                            void* arena, size_t arena_bytes, s2o_stream_t stream) {
+  s2o_status st = check_cfg(cfg);
+  if (st != S2O_OK) return st;
+  if (!Q_host || !K_host || !V_host || !O_host || !arena) return S2O_ERR_INVALID_ARG;
+  size_t need = 0;
+  st = s2o_prefill_arena_size(cfg, out_dtype, &need);
+  if (st != S2O_OK) return st;
+  if (arena_bytes < need) return S2O_ERR_WORKSPACE_TOO_SMALL;
+  if (reinterpret_cast<uintptr_t>(arena) & 255u) return S2O_ERR_INVALID_ARG;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  const size_t q = (size_t)cfg->B * cfg->Hq * cfg->N * kD, kv = (size_t)cfg->B * cfg->Hkv * cfg->N * kD;
+  const size_t T = (size_t)cfg->B * cfg->Hkv * ncand_total(cfg), S = (size_t)cfg->B * cfg->Hkv * nseg(cfg);
+  const size_t obytes = q * (out_dtype == S2O_OUT_F32 ? 4 : 2);
+  uint8_t* p = static_cast<uint8_t*>(arena);
+  uint16_t* dQ = reinterpret_cast<uint16_t*>(p); p += round256(q * 2);
+  uint16_t* dK = reinterpret_cast<uint16_t*>(p); p += round256(kv * 2);
+  uint16_t* dV = reinterpret_cast<uint16_t*>(p); p += round256(kv * 2);
+  void* dO = p; p += round256(obytes);
+  float* dscores = reinterpret_cast<float*>(p); p += round256(T * 4 + 16);
+  int32_t* dperm = reinterpret_cast<int32_t*>(p); p += round256(T * 4 + 16);
+  int32_t* dnb = reinterpret_cast<int32_t*>(p); p += round256(S * 4);
+  void* ws = p;
+  size_t wsb = 0;
+  s2o_plan_workspace_size(cfg, &wsb);
+
+  if (cudaMemcpyAsync(dQ, Q_host, q * 2, cudaMemcpyHostToDevice, s) != cudaSuccess ||
+      cudaMemcpyAsync(dK, K_host, kv * 2, cudaMemcpyHostToDevice, s) != cudaSuccess ||
+      cudaMemcpyAsync(dV, V_host, kv * 2, cudaMemcpyHostToDevice, s) != cudaSuccess)
+    return S2O_ERR_CUDA;
+  st = s2o_plan(cfg, dQ, dK, dscores, dperm, dnb, nullptr, ws, wsb, stream);
+  if (st != S2O_OK) return st;
+  const int32_t n_plan = t_launches;
+  st = s2o_attention(cfg, dQ, dK, dV, dperm, dnb, dO, out_dtype, stream);
+  if (st != S2O_OK) return st;
+  t_launches += n_plan;
+  if (cudaMemcpyAsync(O_host, dO, obytes, cudaMemcpyDeviceToHost, s) != cudaSuccess) return S2O_ERR_CUDA;
+  if (nblocks_host && cudaMemcpyAsync(nblocks_host, dnb, S * 4, cudaMemcpyDeviceToHost, s) != cudaSuccess)
+    return S2O_ERR_CUDA;
+  return s2o_last_device_error(stream);
+}
+
+const char* s2o_status_string(s2o_status st) {
+  switch (st) {
+    case S2O_OK: return "ok";
+    case S2O_ERR_INVALID_ARG: return "invalid argument";
+    case S2O_ERR_UNSUPPORTED_SHAPE: return "unsupported shape or constants";
+    case S2O_ERR_WORKSPACE_TOO_SMALL: return "workspace too small";
+    case S2O_ERR_CUDA: return "CUDA runtime error";
+    case S2O_ERR_DEVICE_TIMEOUT: return "bounded device wait ran out";
+    case S2O_ERR_NONFINITE: return "non-finite input or score";
+    case S2O_ERR_BAD_PLAN: return "plan index out of range";
+  }
+  return "unknown status";
+}
+
+s2o_status s2o_last_device_error(s2o_stream_t stream) {
+  if (cudaStreamSynchronize(reinterpret_cast<cudaStream_t>(stream)) != cudaSuccess) return S2O_ERR_CUDA;
+  unsigned word = 0;
+  if (cudaMemcpyFromSymbol(&word, g_s2o_error, sizeof(word)) != cudaSuccess) return S2O_ERR_CUDA;
+  const unsigned zero = 0;
+  if (word && cudaMemcpyToSymbol(g_s2o_error, &zero, sizeof(zero)) != cudaSuccess) return S2O_ERR_CUDA;
+  if (word & kErrTimeout) return S2O_ERR_DEVICE_TIMEOUT;
+  if (word & kErrNonFinite) return S2O_ERR_NONFINITE;
+  if (word & kErrBadPlan) return S2O_ERR_BAD_PLAN;
+  return S2O_OK;
+}
+
+int32_t s2o_last_launch_count(void) { return t_launches; }
+
+}  // extern "C"

@@ -1,0 +1,262 @@
+"""GPU parity: the CUDA plan and attention, called through the C ABI, against
+the fp64 oracle on the same seeded bf16 inputs."""
+import numpy as np
+import pytest
+import torch
+
+import score_keys_pooled_b200 as s2o
+from score_keys_pooled_b200 import synth
+from oracle import s2o_oracle as O
+from tests import parity
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _gpu():
+    if not torch.cuda.is_available():
+        pytest.skip("needs a CUDA device")
+    s2o.lib()
+
+
+def dev(a: np.ndarray) -> torch.Tensor:
+    return torch.from_numpy(np.ascontiguousarray(a).view(np.int16)).cuda()
+
+
+def run_path(Q, K, V, tau, out_dtype=s2o.OUT_BF16):
+    B, Hq, N, d = Q.shape
+    cfg = s2o.make_config(B, Hq, K.shape[1], N, tau=tau)
+    q, k, v = dev(Q), dev(K), dev(V)
+    bufs = s2o.plan(cfg, q, k)
+    assert s2o.last_launch_count() == 4
+    out = s2o.attention(cfg, q, k, v, bufs["perm"], bufs["nblocks"], out_dtype=out_dtype)
+    assert s2o.last_launch_count() == 1
+    assert s2o.last_device_error() == 0
+    return cfg, bufs, out
+
+
+def host_plan(cfg, bufs):
+    BH = cfg.B * cfg.Hkv
+    S, T = s2o.num_segments(cfg), s2o.num_candidates(cfg)
+    perm = bufs["perm"][:BH * T].cpu().numpy().reshape(cfg.B, cfg.Hkv, T)
+    nb = bufs["nblocks"].cpu().numpy().reshape(cfg.B, cfg.Hkv, S)
+    scores = bufs["scores"][:BH * T].cpu().numpy().reshape(cfg.B, cfg.Hkv, T)
+    stats = bufs["seg_stats"].cpu().numpy().reshape(cfg.B, cfg.Hkv, S, 2)
+    return perm, nb, scores, stats
+
+
+def check_plan(Q, K, cfg, bufs, p, segments=None, kvheads=None, what=""):
+    perm, nb, scores, stats = host_plan(cfg, bufs)
+    G = cfg.Hq // cfg.Hkv
+    off = O.candidate_offsets(cfg.N, p)
+    S = O.num_segments(cfg.N, p)
+    segs = range(S) if segments is None else segments
+    heads = [(b, h) for b in range(cfg.B) for h in (range(cfg.Hkv) if kvheads is None else kvheads)]
+    swaps = flips = 0
+    plans = {}
+    for b, kvh in heads:
+        for s in segs:
+            sp = O.plan_segment(Q, K, b, kvh, s, G, p)
+            plans[(b, kvh, s)] = sp
+            lo, hi = O.candidate_range(cfg.N, s, p)
+            # scores agree with the fp64 ones to fp32 accuracy
+            gs = scores[b, kvh, off[s]:off[s + 1]]
+            tol = 1e-6 * max(1.0, float(np.max(np.abs(sp.scores))))
+            assert np.max(np.abs(gs - sp.scores[lo:hi]), initial=0.0) <= tol
+            assert abs(stats[b, kvh, s, 0] - sp.M) <= tol
+            assert abs(stats[b, kvh, s, 1] / sp.Z - 1.0) <= 1e-5
+            sw, fl = parity.compare_segment_plan(perm[b, kvh, off[s]:off[s + 1]], int(nb[b, kvh, s]), sp, p)
+            swaps += sw
+            flips += fl
+    parity.log_near_ties({"case": what, "tau": p.tau, "segments": len(segs) * len(heads),
+                          "swapped_positions": swaps, "C_flips": flips})
+    return perm, nb, plans
+
+
+def check_output(Q, K, V, cfg, perm, nb, out, p, segments=None, kvheads=None, what=""):
+    G = cfg.Hq // cfg.Hkv
+    off = O.candidate_offsets(cfg.N, p)
+    S = O.num_segments(cfg.N, p)
+    segs = range(S) if segments is None else segments
+    got = out.float().cpu().numpy()
+    worst = (0.0, 0.0)
+    for b in range(cfg.B):
+        for kvh in (range(cfg.Hkv) if kvheads is None else kvheads):
+            for s in segs:
+                keep = O.keep_set(cfg.N, s, perm[b, kvh, off[s]:off[s + 1]], int(nb[b, kvh, s]), p)
+                ref = O.attention_segment(Q, K, V, b, kvh, s, G, keep, p)
+                r0, r1 = O.segment_rows(cfg.N, s, p)
+                g = got[b, kvh * G:(kvh + 1) * G, r0:r1]
+                e = parity.assert_output_close(g, ref, f"{what} b={b} kvh={kvh} s={s}")
+                worst = (max(worst[0], e[0]), max(worst[1], e[1]))
+    return worst
+
+
+SMALL = [
+    # (B, Hq, Hkv, N, tau, planted, band)
+    (1, 1, 1, 1024, 1e-3, True, False),
+    (1, 8, 2, 1280, 3e-3, True, True),
+    (1, 8, 2, 1280, 0.0, True, True),
+    (1, 8, 2, 1280, 2.0, True, True),
+    (2, 4, 2, 768, 1e-2, True, False),
+    (1, 4, 1, 1000, 1e-2, True, True),
+    (1, 4, 1, 1111, 5e-3, False, False),
+    (1, 4, 4, 640, 1e-3, True, True),
+]
+
+
+@pytest.mark.parametrize("B,Hq,Hkv,N,tau,planted,band", SMALL)
+@pytest.mark.parametrize("out_dtype", [s2o.OUT_BF16, s2o.OUT_F32])
+def test_small_cases_full_parity(B, Hq, Hkv, N, tau, planted, band, out_dtype):
+    Q, K, V = synth.generate(B, Hq, Hkv, N, 128, planted=planted, band=band, n_stripe=8, seed=N + Hq)
+    p = O.Params(tau=tau)
+    cfg, bufs, out = run_path(Q, K, V, tau, out_dtype)
+    perm, nb, plans = check_plan(Q, K, cfg, bufs, p, what=f"small N={N}")
+    if tau == 0.0:
+        for (b, kvh, s), sp in plans.items():
+            assert nb[b, kvh, s] == O.num_blocks(O.num_candidates(N, s, p), p)
+    check_output(Q, K, V, cfg, perm, nb, out, p, what=f"small N={N}")
+
+
+@pytest.mark.parametrize("N", [1, 63, 64, 127, 128, 129, 255, 256, 300, 385])
+def test_ragged_and_tiny_lengths(N):
+    Q, K, V = synth.generate(1, 2, 1, N, 128, planted=N > 4, band=True, n_stripe=2, seed=N)
+    p = O.Params(tau=1e-3)
+    cfg, bufs, out = run_path(Q, K, V, 1e-3)
+    perm, nb, _ = check_plan(Q, K, cfg, bufs, p, what=f"ragged N={N}")
+    check_output(Q, K, V, cfg, perm, nb, out, p, what=f"ragged N={N}")
+
+
+@pytest.mark.parametrize("tau", [1e-3, 0.0625, 0.07])
+def test_all_ties_bit_exact(tau):
+    # Q = 0: every score is exactly 0, so the order is ascending and
+    # m_b = 64 / e(s) exactly; no tolerance applies.
+    N = 1024
+    Q = np.zeros((1, 4, N, 128), dtype=np.uint16)
+    _, K, V = synth.generate(1, 4, 1, N, 128, planted=True, band=False, n_stripe=8, seed=3)
+    cfg, bufs, out = run_path(Q, K, V, tau)
+    perm, nb, scores, stats = host_plan(cfg, bufs)
+    p = O.Params(tau=tau)
+    off = O.candidate_offsets(N, p)
+    assert np.all(scores == 0.0)
+    for s in range(O.num_segments(N, p)):
+        lo, hi = O.candidate_range(N, s, p)
+        assert np.array_equal(perm[0, 0, off[s]:off[s + 1]], np.arange(lo, hi))
+        e = O.admissible_end(N, s, p)
+        nbk = O.num_blocks(hi - lo, p)
+        assert nb[0, 0, s] == (nbk if 64.0 / e >= tau else 0)
+        assert stats[0, 0, s, 0] == 0.0 and stats[0, 0, s, 1] == float(e)
+
+
+def test_nonfinite_input_is_reported():
+    Q, K, V = synth.generate(1, 4, 1, 512, 128, planted=True, band=False, n_stripe=4, seed=9)
+    K = K.copy()
+    K[0, 0, 300, 5] = 0x7FC0  # bf16 NaN
+    cfg = s2o.make_config(1, 4, 1, 512, tau=1e-3)
+    s2o.plan(cfg, dev(Q), dev(K))
+    assert s2o.last_device_error() == 6
+    assert s2o.last_device_error() == 0  # the word is cleared by the read
+
+
+def test_out_of_range_plan_is_clamped_and_reported():
+    Q, K, V = synth.generate(1, 4, 1, 768, 128, planted=True, band=False, n_stripe=4, seed=10)
+    cfg = s2o.make_config(1, 4, 1, 768, tau=0.0)
+    q, k, v = dev(Q), dev(K), dev(V)
+    bufs = s2o.plan(cfg, q, k)
+    perm = bufs["perm"].clone()
+    perm[3] = 10 ** 6
+    s2o.attention(cfg, q, k, v, perm, bufs["nblocks"])
+    assert s2o.last_device_error() == 7
+    nbad = bufs["nblocks"].clone()
+    nbad[4] = 999
+    s2o.attention(cfg, q, k, v, bufs["perm"], nbad)
+    assert s2o.last_device_error() == 7
+    assert s2o.last_device_error() == 0
+
+
+def test_host_buffer_entry_matches_device_path():
+    Q, K, V = synth.generate(1, 8, 2, 1536, 128, planted=True, band=True, n_stripe=8, seed=12)
+    cfg, bufs, out = run_path(Q, K, V, 1e-3)
+    arena = torch.empty(s2o.prefill_arena_size(cfg), dtype=torch.uint8, device="cuda")
+    pin = lambda a: torch.from_numpy(a.view(np.int16)).pin_memory()
+    O_host = torch.empty(Q.shape, dtype=torch.int16).pin_memory()
+    nb_host = torch.empty(cfg.B * cfg.Hkv * s2o.num_segments(cfg), dtype=torch.int32)
+    s2o.prefill_host(cfg, pin(Q), pin(K), pin(V), O_host, arena, nblocks_host=nb_host)
+    assert torch.equal(O_host.view(torch.bfloat16), out.cpu())
+    assert torch.equal(nb_host, bufs["nblocks"].cpu())
+
+
+def sampled_segments(S):
+    base = {0, 1, 2, 3, S // 4, S // 2, 3 * S // 4, S - 1}
+    rng = np.random.default_rng(1)
+    extra = [int(x) for x in rng.choice(np.arange(4, S - 1), 8, replace=False)]
+    return sorted(base | set(extra))
+
+
+@pytest.mark.parametrize("name", ["tiny_1k", "llama_16k"])
+def test_workload_full_plan_sampled_output(name):
+    w = synth.WORKLOADS[name]
+    Q, K, V = synth.generate_workload(w)
+    p = O.Params(tau=w.tau)
+    cfg, bufs, out = run_path(Q, K, V, w.tau)
+    perm, nb, _ = check_plan(Q, K, cfg, bufs, p, what=name)
+    S = O.num_segments(w.N, p)
+    segs = None if S <= 8 else sampled_segments(S)
+    check_output(Q, K, V, cfg, perm, nb, out, p, segments=segs, what=name)
+
+
+@pytest.mark.parametrize("name", ["llama_128k", "flat_128k"])
+def test_workload_128k_sampled(name):
+    # full-size launch (the benchmark's configuration); the oracle checks
+    # sampled segments of every KV head for the plan and of two KV heads for
+    # the output
+    w = synth.WORKLOADS[name]
+    Q, K, V = synth.generate_workload(w)
+    p = O.Params(tau=w.tau)
+    cfg, bufs, out = run_path(Q, K, V, w.tau)
+    S = O.num_segments(w.N, p)
+    segs = sampled_segments(S)
+    perm, nb, _ = check_plan(Q, K, cfg, bufs, p, segments=segs, what=name)
+    check_output(Q, K, V, cfg, perm, nb, out, p, segments=segs[::2], kvheads=[0, w.Hkv - 1], what=name)
+
+
+def test_sweep_64k_tau_and_contiguous():
+    w = synth.WORKLOADS["sweep_64k"]
+    Q, K, V = synth.generate_workload(w)
+    S = O.num_segments(w.N, O.Params())
+    segs = [2, 5, S // 3, S - 1]
+    q, k, v = dev(Q), dev(K), dev(V)
+    for tau in synth.TAU_SWEEP:
+        p = O.Params(tau=tau)
+        cfg = s2o.make_config(w.B, w.Hq, w.Hkv, w.N, tau=tau)
+        bufs = s2o.plan(cfg, q, k)
+        assert s2o.last_device_error() == 0
+        perm, nb, plans = check_plan(Q, K, cfg, bufs, p, segments=segs, kvheads=[0, 5], what=f"sweep tau={tau}")
+        if tau in (1e-3, 1e-2):
+            out = s2o.attention(cfg, q, k, v, bufs["perm"], bufs["nblocks"])
+            check_output(Q, K, V, cfg, perm, nb, out, p, segments=segs, kvheads=[5], what=f"sweep tau={tau}")
+            # contiguous comparator at the same per-segment block count
+            pc = torch.empty_like(bufs["perm"])
+            s2o.plan_contiguous(cfg, bufs["scores"], bufs["seg_stats"], bufs["nblocks"], pc)
+            assert s2o.last_device_error() == 0
+            T = s2o.num_candidates(cfg)
+            pch = pc[:cfg.B * cfg.Hkv * T].cpu().numpy().reshape(cfg.B, cfg.Hkv, T)
+            off = O.candidate_offsets(w.N, p)
+            for s in segs:
+                sp = plans[(0, 5, s)]
+                want = O.contiguous_plan_segment(sp, w.N, int(nb[0, 5, s]), p)
+                got = pch[0, 5, off[s]:off[s + 1]]
+                # block ranks may only differ between blocks of near-equal mass
+                gb = got.reshape(-1, p.Bk)[:, 0]
+                wb = want.reshape(-1, p.Bk)[:, 0]
+                if not np.array_equal(gb, wb):
+                    lo, hi = O.candidate_range(w.N, s, p)
+                    wts = np.exp(sp.scores[lo:hi] - sp.M) / sp.Z
+                    bm = wts.reshape(-1, p.Bk).sum(1)
+                    diff = np.nonzero(gb != wb)[0]
+                    tolm = 1e-6 * bm.max()
+                    assert np.all(np.abs(bm[(gb[diff] - lo) // p.Bk] - bm[(wb[diff] - lo) // p.Bk]) <= tolm)
+                assert np.array_equal(np.sort(got), np.arange(O.candidate_range(w.N, s, p)[0],
+                                                               O.candidate_range(w.N, s, p)[1]))
+            outc = s2o.attention(cfg, q, k, v, pc, bufs["nblocks"])
+            check_output(Q, K, V, cfg, pch, nb, outc, p, segments=segs, kvheads=[5], what=f"contig tau={tau}")
