@@ -15,10 +15,10 @@ namespace s2o {
 
 // ---------------------------------------------------------------------------
 // pool: one CTA per (s, b*Hkv); 256 threads; thread = (16-byte chunk, row group)
-// Q is read once with 16-byte loads; sums are fp64 (exact for bf16 inputs up
-// to 2^36 terms of similar magnitude), rounded once to fp32 at the end.
+// Q is read once with 16-byte loads; sums and the mean are fp64 (exact for
+// bf16 inputs whose magnitudes span less than ~2^36).
 // ---------------------------------------------------------------------------
-__global__ void __launch_bounds__(256) k_pool(const uint16_t* __restrict__ Q, float* __restrict__ qbar,
+__global__ void __launch_bounds__(256) k_pool(const uint16_t* __restrict__ Q, double* __restrict__ qbar,
                                              int Hq, int Hkv, int N, int S) {
   const int s = blockIdx.x;
   const int bk = blockIdx.y;  // b * Hkv + kvh
@@ -54,16 +54,22 @@ __global__ void __launch_bounds__(256) k_pool(const uint16_t* __restrict__ Q, fl
 #pragma unroll
     for (int r = 0; r < 16; ++r) t += red[r][threadIdx.x];
     const double cnt = (double)G * (double)(r1 - r0);
-    qbar[((size_t)bk * S + s) * kD + threadIdx.x] = (float)(t / cnt);
+    qbar[((size_t)bk * S + s) * kD + threadIdx.x] = t / cnt;
   }
 }
 
 // ---------------------------------------------------------------------------
 // score: CTA = (key tile t of 128 keys, chunk of 64 segments, b*Hkv).
 // Only segments s >= t see tile t (e(s) = 128 s + 128 > 128 t), so CTAs whose
-// chunk ends before t exit at once.  The tile's keys (transposed, fp32) and
-// the chunk's pooled queries (transposed) sit in shared memory; each thread
-// accumulates an 8 key x 4 segment block of dot products in fp32 FMA.
+// chunk ends before t exit at once.  Dot products are accumulated in fp64:
+// qbar is the exact fp64 mean of bf16 values and k_j is bf16, so every
+// product is exact and the sum carries ~1e-15 relative error; each score is
+// rounded once to fp32.  (fp32 accumulation of these 128-term dots errs by
+// ~1e-6 relative when the terms share a sign, the width of the near-tie band
+// the importance order is checked against.)
+// The d = 128 reduction runs in two halves of 64 so that the transposed key
+// tile (fp64) and pooled queries (fp64) fit twice per SM.  Thread (tk, ts)
+// accumulates keys tk + 16 a (a < 8) x segments ts + 16 b (b < 4).
 // Outputs:
 //   scores[bk][off(s) + j - 64] for candidate keys j of segment s
 //   part[bk][s][t] = (max over the tile's admissible keys,
@@ -71,13 +77,12 @@ __global__ void __launch_bounds__(256) k_pool(const uint16_t* __restrict__ Q, fl
 // ---------------------------------------------------------------------------
 constexpr int kScoreKeys = 128;
 constexpr int kScoreSegs = 64;
-constexpr int kKtStride = kScoreKeys + 4;   // padded row of the transposed key tile
-constexpr int kQtStride = kScoreSegs + 4;
-constexpr size_t kScoreSmem = sizeof(float) * (kD * kKtStride + kD * kQtStride);
+constexpr int kScoreHalf = 64;  // d per pass
+constexpr size_t kScoreSmem = sizeof(double) * (kScoreHalf * kScoreKeys + kScoreHalf * kScoreSegs);
 
-__global__ void __launch_bounds__(256) k_score(const uint16_t* __restrict__ K, const float* __restrict__ qbar,
-                                              float* __restrict__ scores, float2* __restrict__ part,
-                                              int Hkv, int N, int S, int64_t T) {
+__global__ void __launch_bounds__(256, 2) k_score(const uint16_t* __restrict__ K, const double* __restrict__ qbar,
+                                                 float* __restrict__ scores, float2* __restrict__ part,
+                                                 int Hkv, int N, int S, int64_t T) {
   const int t = blockIdx.x;           // key tile
   const int chunk = blockIdx.y;       // segment chunk
   const int bk = blockIdx.z;          // b * Hkv + kvh
@@ -85,70 +90,71 @@ __global__ void __launch_bounds__(256) k_score(const uint16_t* __restrict__ K, c
   const int s_hi = min(S, s_lo + kScoreSegs);
   if (s_hi - 1 < t) return;
 
-  extern __shared__ float sm[];
-  float* Kt = sm;                       // [d][kKtStride]
-  float* Qt = sm + kD * kKtStride;      // [d][kQtStride]
+  extern __shared__ double smd[];
+  double* Kt = smd;                               // [64 d][128 keys]
+  double* Qt = smd + kScoreHalf * kScoreKeys;     // [64 d][64 segs]
   const int tid = threadIdx.x;
-
-  // key tile -> fp32, transposed; keys >= N are zero (and never admissible)
+  const int tk = tid & 15;
+  const int ts = tid >> 4;
   const uint16_t* Kb = K + (size_t)bk * N * kD;
-  for (int q = tid; q < kScoreKeys * 16; q += 256) {
-    const int key = q & (kScoreKeys - 1), c = q >> 7;
-    const int j = t * kScoreKeys + key;
-    uint4 w = make_uint4(0, 0, 0, 0);
-    if (j < N) w = *reinterpret_cast<const uint4*>(Kb + (size_t)j * kD + 8 * c);
-    if (bf16x2_nonfinite(w.x) | bf16x2_nonfinite(w.y) | bf16x2_nonfinite(w.z) | bf16x2_nonfinite(w.w))
-      set_error(kErrNonFinite);
-    float* col = Kt + (8 * c) * kKtStride + key;
-    col[0 * kKtStride] = bf16_lo(w.x); col[1 * kKtStride] = bf16_hi(w.x);
-    col[2 * kKtStride] = bf16_lo(w.y); col[3 * kKtStride] = bf16_hi(w.y);
-    col[4 * kKtStride] = bf16_lo(w.z); col[5 * kKtStride] = bf16_hi(w.z);
-    col[6 * kKtStride] = bf16_lo(w.w); col[7 * kKtStride] = bf16_hi(w.w);
-  }
-  // pooled queries of the chunk, transposed
-  const float* qb = qbar + (size_t)bk * S * kD;
-  for (int q = tid; q < kScoreSegs * kD; q += 256) {
-    const int seg = q / kD, dd = q % kD;
-    const int s = s_lo + seg;
-    Qt[dd * kQtStride + seg] = (s < S) ? qb[(size_t)s * kD + dd] : 0.f;
-  }
-  __syncthreads();
+  const double* qb = qbar + (size_t)bk * S * kD;
 
-  const int tk = tid & 15;   // keys tk*8 .. tk*8+7
-  const int ts = tid >> 4;   // segments ts*4 .. ts*4+3
-  float acc[8][4];
+  double acc[8][4];
 #pragma unroll
   for (int a = 0; a < 8; ++a)
 #pragma unroll
-    for (int q = 0; q < 4; ++q) acc[a][q] = 0.f;
+    for (int q = 0; q < 4; ++q) acc[a][q] = 0.0;
 
-#pragma unroll 4
-  for (int dd = 0; dd < kD; ++dd) {
-    const float4 k0 = *reinterpret_cast<const float4*>(Kt + dd * kKtStride + tk * 8);
-    const float4 k1 = *reinterpret_cast<const float4*>(Kt + dd * kKtStride + tk * 8 + 4);
-    const float4 qv = *reinterpret_cast<const float4*>(Qt + dd * kQtStride + ts * 4);
-    const float kk[8] = {k0.x, k0.y, k0.z, k0.w, k1.x, k1.y, k1.z, k1.w};
-    const float qq[4] = {qv.x, qv.y, qv.z, qv.w};
+  for (int half = 0; half < 2; ++half) {
+    if (half) __syncthreads();
+    // key tile half -> fp64, transposed; keys >= N are zero (never admissible)
+    for (int q = tid; q < kScoreKeys * 8; q += 256) {
+      const int key = q & (kScoreKeys - 1), c = q >> 7;  // c: 16-byte chunk 0..7 of this half
+      const int j = t * kScoreKeys + key;
+      uint4 w = make_uint4(0, 0, 0, 0);
+      if (j < N) w = *reinterpret_cast<const uint4*>(Kb + (size_t)j * kD + half * kScoreHalf + 8 * c);
+      if (bf16x2_nonfinite(w.x) | bf16x2_nonfinite(w.y) | bf16x2_nonfinite(w.z) | bf16x2_nonfinite(w.w))
+        set_error(kErrNonFinite);
+      double* col = Kt + (8 * c) * kScoreKeys + key;
+      col[0 * kScoreKeys] = bf16_lo(w.x); col[1 * kScoreKeys] = bf16_hi(w.x);
+      col[2 * kScoreKeys] = bf16_lo(w.y); col[3 * kScoreKeys] = bf16_hi(w.y);
+      col[4 * kScoreKeys] = bf16_lo(w.z); col[5 * kScoreKeys] = bf16_hi(w.z);
+      col[6 * kScoreKeys] = bf16_lo(w.w); col[7 * kScoreKeys] = bf16_hi(w.w);
+    }
+    for (int q = tid; q < kScoreSegs * kScoreHalf; q += 256) {
+      const int seg = q / kScoreHalf, dd = q % kScoreHalf;
+      const int s = s_lo + seg;
+      Qt[dd * kScoreSegs + seg] = (s < S) ? qb[(size_t)s * kD + half * kScoreHalf + dd] : 0.0;
+    }
+    __syncthreads();
+#pragma unroll 2
+    for (int dd = 0; dd < kScoreHalf; ++dd) {
+      double kk[8], qq[4];
 #pragma unroll
-    for (int a = 0; a < 8; ++a)
+      for (int a = 0; a < 8; ++a) kk[a] = Kt[dd * kScoreKeys + tk + 16 * a];
 #pragma unroll
-      for (int q = 0; q < 4; ++q) acc[a][q] = fmaf(kk[a], qq[q], acc[a][q]);
+      for (int q = 0; q < 4; ++q) qq[q] = Qt[dd * kScoreSegs + ts + 16 * q];
+#pragma unroll
+      for (int a = 0; a < 8; ++a)
+#pragma unroll
+        for (int q = 0; q < 4; ++q) acc[a][q] = fma(kk[a], qq[q], acc[a][q]);
+    }
   }
 
-  const float inv_sqrt_d = 0.08838834764831845f;  // 1/sqrt(128), correctly rounded
   float* sc_bk = scores + (size_t)bk * T;
   float2* part_bk = part + (size_t)bk * S * S;
+  const double sqrt_d = 11.313708498984761;  // sqrt(128)
 #pragma unroll
   for (int q = 0; q < 4; ++q) {
-    const int s = s_lo + ts * 4 + q;
+    const int s = s_lo + ts + 16 * q;
     const bool seg_ok = (s < s_hi) && (s >= t);
     const int cand_hi = s * kLq - kWin;  // candidates are [64, cand_hi)
     float v[8];
     float mloc = -INFINITY;
 #pragma unroll
     for (int a = 0; a < 8; ++a) {
-      const int j = t * kScoreKeys + tk * 8 + a;
-      v[a] = acc[a][q] * inv_sqrt_d;
+      const int j = t * kScoreKeys + tk + 16 * a;
+      v[a] = (float)(acc[a][q] / sqrt_d);
       const bool adm = seg_ok && (j < N);
       if (adm) {
         if (!isfinite(v[a])) set_error(kErrNonFinite);

@@ -38,7 +38,7 @@ int32_t nseg(const s2o_config* c) { return (c->N + kLq - 1) / kLq; }
 int64_t ncand_total(const s2o_config* c) { return cand_offset(nseg(c)); }
 
 struct PlanWs {
-  float* qbar;
+  double* qbar;
   float2* part;
   float* segM;
   double* segZ;
@@ -55,7 +55,7 @@ PlanWs plan_layout(const s2o_config* c, void* base) {
     off += round256(bytes);
     return static_cast<void*>(p);
   };
-  w.qbar = static_cast<float*>(take(BH * S * kD * sizeof(float)));
+  w.qbar = static_cast<double*>(take(BH * S * kD * sizeof(double)));
   w.part = static_cast<float2*>(take(BH * S * S * sizeof(float2)));
   w.segM = static_cast<float*>(take(BH * S * sizeof(float)));
   w.segZ = static_cast<double*>(take(BH * S * sizeof(double)));

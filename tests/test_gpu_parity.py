@@ -59,11 +59,12 @@ def check_plan(Q, K, cfg, bufs, p, segments=None, kvheads=None, what=""):
             sp = O.plan_segment(Q, K, b, kvh, s, G, p)
             plans[(b, kvh, s)] = sp
             lo, hi = O.candidate_range(cfg.N, s, p)
-            # scores agree with the fp64 ones to fp32 accuracy
-            gs = scores[b, kvh, off[s]:off[s + 1]]
-            tol = 1e-6 * max(1.0, float(np.max(np.abs(sp.scores))))
-            assert np.max(np.abs(gs - sp.scores[lo:hi]), initial=0.0) <= tol
-            assert abs(stats[b, kvh, s, 0] - sp.M) <= tol
+            # scores are the fp64 values rounded once to fp32 (half an ulp)
+            gs = scores[b, kvh, off[s]:off[s + 1]].astype(np.float64)
+            ref = sp.scores[lo:hi]
+            half_ulp = 0.5 * np.spacing(np.abs(ref).astype(np.float32)).astype(np.float64)
+            assert np.all(np.abs(gs - ref) <= half_ulp + 1e-13 * np.abs(ref) + 1e-300)
+            assert abs(stats[b, kvh, s, 0] - sp.M) <= 0.5 * float(np.spacing(np.float32(abs(sp.M)))) + 1e-13 * abs(sp.M)
             assert abs(stats[b, kvh, s, 1] / sp.Z - 1.0) <= 1e-5
             sw, fl = parity.compare_segment_plan(perm[b, kvh, off[s]:off[s + 1]], int(nb[b, kvh, s]), sp, p)
             swaps += sw
