@@ -61,6 +61,22 @@ def kept_pairs(nblocks: np.ndarray, N: int, G: int) -> int:
     return total
 
 
+def reduce_max_ms(ms: float, dist=None, device="cpu") -> float:
+    """Max over ranks of a per-rank time (the slowest rank bounds the job)."""
+    if dist is None or not dist.is_initialized() or dist.get_world_size() == 1:
+        return float(ms)
+    import torch
+    t = torch.tensor([float(ms)], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def whole_job_tflops(world: int, flops_per_rank: float, ms: float) -> float:
+    """Every rank solves its own problem: the job's throughput is all ranks'
+    work over the slowest rank's time."""
+    return world * flops_per_rank / (ms * 1e-3) / 1e12
+
+
 def load_peaks():
     path = os.path.join(ROOT, "MEASURED_PEAKS.json")
     if os.path.exists(path):
@@ -119,8 +135,9 @@ class ClockSampler:
 
 
 def cpu_oracle_sample(Q, K, V, tau, seconds=15.0):
-    """Oracle (fp64, one thread) on sampled segments of KV head 0: plan +
-    attention of every head of the group.  Returns (TFLOP/s dense-equiv, sample text)."""
+    """Oracle (fp64, one thread) on sampled segments, KV head by KV head: plan +
+    attention of every query head of the group, until `seconds` have passed.
+    Returns (dense-equivalent TFLOP/s of the rows done, sample text, seconds)."""
     from threadpoolctl import threadpool_limits
     from oracle import s2o_oracle as O
 
@@ -128,21 +145,26 @@ def cpu_oracle_sample(Q, K, V, tau, seconds=15.0):
     N, d = Q.shape[2], Q.shape[3]
     G = Q.shape[1] // K.shape[1]
     S = O.num_segments(N, p)
-    order = [S - 1, S // 2, S // 4, 3 * S // 4, 3, 2, 1, 0] + list(range(S - 2, 3, -97))
+    order = sorted({S - 1, S // 2, S // 4, 3 * S // 4, 3, 2, 1, 0} | set(range(S - 2, 3, -97)))
     done, flops, t0 = [], 0.0, time.perf_counter()
     with threadpool_limits(1):
-        for s in order:
-            sp = O.plan_segment(Q, K, 0, 0, s, G, p)
-            O.attention_segment(Q, K, V, 0, 0, s, G, sp.keep, p)
-            r0, r1 = O.segment_rows(N, s, p)
-            rows = np.arange(r0, r1, dtype=np.float64)
-            flops += G * 4.0 * d * float(np.sum(rows + 1))  # dense-equivalent work of these rows
-            done.append(s)
+        for kvh in range(K.shape[1]):
+            for s in order:
+                sp = O.plan_segment(Q, K, 0, kvh, s, G, p)
+                O.attention_segment(Q, K, V, 0, kvh, s, G, sp.keep, p)
+                r0, r1 = O.segment_rows(N, s, p)
+                rows = np.arange(r0, r1, dtype=np.float64)
+                flops += G * 4.0 * d * float(np.sum(rows + 1))  # dense-equivalent work of these rows
+                done.append((kvh, s))
+                if time.perf_counter() - t0 > seconds:
+                    break
             if time.perf_counter() - t0 > seconds:
                 break
     dt = time.perf_counter() - t0
-    sample = (f"oracle plan+attention of segments {done} (KV head 0, all {G} query heads of its group) "
-              f"of the {N}-token workload; fp64, 1 thread; {dt:.1f} s")
+    heads = sorted({h for h, _ in done})
+    sample = (f"oracle plan+attention of {len(done)} (KV head, segment) items, KV heads {heads}, segments "
+              f"{order} (all {G} query heads of each group) of the {N}-token workload; fp64, 1 thread; "
+              f"{dt:.1f} s")
     return flops / dt / 1e12, sample, dt
 
 
@@ -152,9 +174,9 @@ def reference_arm(args, w, world, rank):
         return
     from score_keys_pooled_b200 import synth
     Q, K, V = synth.generate_workload(w, seed=0)
-    budget = max(10.0, 120.0 / max(1, args.steps + args.warmup))
+    budget = max(2.0, 150.0 / max(1, args.steps + args.warmup))
     for _ in range(args.warmup):
-        cpu_oracle_sample(Q, K, V, w.tau, seconds=2.0)
+        cpu_oracle_sample(Q, K, V, w.tau, seconds=min(2.0, budget))
     vals, total = [], 0.0
     for _ in range(args.steps):
         v, sample, dt = cpu_oracle_sample(Q, K, V, w.tau, seconds=budget)
@@ -249,10 +271,7 @@ def main():
     total_ms = t_start.elapsed_time(t_end)
     plan_ms = [e[0].elapsed_time(e[1]) for e in ev]
     attn_ms = [e[1].elapsed_time(e[2]) for e in ev]
-    if dist:
-        t = torch.tensor([total_ms], device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        total_ms = float(t.item())
+    total_ms = reduce_max_ms(total_ms, dist, dev)
     st = s2o.last_device_error()
     if st != 0:
         raise RuntimeError(f"device error in the timed region: {s2o.status_string(st)}")
@@ -263,7 +282,7 @@ def main():
     dense = dense_flops(w.B, w.Hq, w.N, w.d)
     density = pairs / (w.B * w.Hq * w.N * (w.N + 1) / 2.0)
     ms_step = total_ms / args.steps
-    value = world * dense / (ms_step * 1e-3) / 1e12
+    value = whole_job_tflops(world, dense, ms_step)
 
     # roofline of the dominant kernel (sparse attention): algorithmic flops
     # = 4 d x kept (row, key) pairs, per launch, over its CUDA-event time
@@ -297,13 +316,10 @@ def main():
         e1.record(stream)
         torch.cuda.synchronize()
         e2e_ms = e0.elapsed_time(e1) / args.e2e_steps
-        if dist:
-            t = torch.tensor([e2e_ms], device=dev)
-            dist.all_reduce(t, op=dist.ReduceOp.MAX)
-            e2e_ms = float(t.item())
+        e2e_ms = reduce_max_ms(e2e_ms, dist, dev)
         h2d = (Qn.nbytes + Kn.nbytes + Vn.nbytes)
         d2h = Qn.nbytes + nb.size * 4
-        e2e = {"value": world * dense / (e2e_ms * 1e-3) / 1e12, "unit": "TFLOP/s", "ms_per_step": e2e_ms,
+        e2e = {"value": whole_job_tflops(world, dense, e2e_ms), "unit": "TFLOP/s", "ms_per_step": e2e_ms,
                "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h)}
         del arena
 
@@ -321,7 +337,7 @@ def main():
                        "global_batch": w.B * world, "seq_len": w.N, "parallelism": f"independent x{world}",
                        "l2": "inputs larger than L2 (Q alone is 1 GiB)"},
             "plan_ms": float(np.mean(plan_ms)), "attention_ms": attn_mean,
-            "attention_only_tflops": world * dense / (attn_mean * 1e-3) / 1e12,
+            "attention_only_tflops": whole_job_tflops(world, dense, attn_mean),
             "kept_pair_fraction": density,
             "roofline": roofline, "cpu_baseline": cpu, "e2e": e2e, "gpu_launches": launches,
             "clocks": clk.summary(),
