@@ -62,8 +62,8 @@
  *
  * Ownership: the caller allocates every buffer, including the plan workspace
  * (size from s2o_plan_workspace_size).  The library never allocates device
- * memory and keeps only one piece of global state per device: a 32-bit
- * device error word (see s2o_last_device_error).
+ * memory.  Its only global state per device is a 32-bit device error word
+ * (see s2o_last_device_error) and the fixed scratch of s2o_plan_noalloc.
  *
  * Execution: every call except s2o_prefill_host and s2o_last_device_error is
  * asynchronous on the given stream (NULL = the legacy default stream) and
@@ -134,6 +134,32 @@ s2o_status s2o_plan_workspace_size(const s2o_config* cfg, size_t* bytes);
 s2o_status s2o_plan(const s2o_config* cfg, const uint16_t* Q, const uint16_t* K,
                     float* scores, int32_t* perm, int32_t* nblocks, float* seg_stats,
                     void* workspace, size_t workspace_bytes, s2o_stream_t stream);
+
+/*
+ * s2o_plan_noalloc -- s2o_plan without a caller-supplied workspace, for
+ * callers that may not allocate device memory: plugins inside an engine or
+ * framework that owns all device memory through its own pool (a cudaMalloc of
+ * theirs would fail or break the pool's accounting), and code on a latency-
+ * critical path where cudaMalloc/cudaFree would synchronise the device.  The
+ * pages have no counterpart to this entry point; it is a deployment aid.
+ *   Outputs, layouts and results are those of s2o_plan (the caller still
+ *   passes Q, K and the output buffers).
+ *   Scratch: a 32 MiB array in the library's device memory (a file-scope
+ *   __device__ buffer that every GPU loading the library holds until the
+ *   process exits).  Configs whose plan workspace (s2o_plan_workspace_size)
+ *   exceeds 32 MiB -- e.g. B=1, 8 KV heads, N above ~8K -- are rejected with
+ *   S2O_ERR_WORKSPACE_TOO_SMALL before anything is launched.
+ *   The first call on a device looks up the buffer's device address for that
+ *   device (make that first call before any stream capture).  Nothing in the
+ *   buffer has to start at zero: every word the kernels read is written
+ *   earlier in the same call.  All calls share the one buffer, so calls whose
+ *   work overlaps on the GPU (other streams, other host threads) race and
+ *   corrupt each other's results; serialise them.
+ *   Allocates nothing: no cudaMalloc, cudaFree or allocating library call.
+ */
+s2o_status s2o_plan_noalloc(const s2o_config* cfg, const uint16_t* Q, const uint16_t* K,
+                            float* scores, int32_t* perm, int32_t* nblocks, float* seg_stats,
+                            s2o_stream_t stream);
 
 /*
  * s2o_plan_contiguous -- block-granular comparator at a matched block count:

@@ -13,6 +13,12 @@
 
 using namespace s2o;
 
+// Scratch of s2o_plan_noalloc: the plan's whole workspace lives here, so that
+// entry point never allocates.  Every GPU that loads the library holds these
+// 32 MiB until the process exits.
+constexpr size_t kNoAllocScratchBytes = size_t(32) << 20;
+static __device__ __align__(256) unsigned char g_s2o_plan_scratch[kNoAllocScratchBytes];
+
 namespace {
 
 thread_local int32_t t_launches = 0;
@@ -82,6 +88,11 @@ cudaError_t set_kernel_attributes() {
   });
   return g_attr_err;
 }
+
+// Device address of g_s2o_plan_scratch, looked up once per device.
+std::mutex g_scratch_mu;
+constexpr int kMaxDevices = 64;
+void* g_scratch_addr[kMaxDevices] = {};
 
 s2o_status launch_status() {
   return cudaGetLastError() == cudaSuccess ? S2O_OK : S2O_ERR_CUDA;
@@ -243,6 +254,30 @@ s2o_status s2o_prefill_host(const s2o_config* cfg, const uint16_t* Q_host, const
   if (nblocks_host && cudaMemcpyAsync(nblocks_host, dnb, S * 4, cudaMemcpyDeviceToHost, s) != cudaSuccess)
     return S2O_ERR_CUDA;
   return s2o_last_device_error(stream);
+}
+
+s2o_status s2o_plan_noalloc(const s2o_config* cfg, const uint16_t* Q, const uint16_t* K, float* scores,
+                            int32_t* perm, int32_t* nblocks, float* seg_stats, s2o_stream_t stream) {
+  t_launches = 0;
+  s2o_status st = check_cfg(cfg);
+  if (st != S2O_OK) return st;
+  if (plan_layout(cfg, nullptr).bytes > kNoAllocScratchBytes) return S2O_ERR_WORKSPACE_TOO_SMALL;
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return S2O_ERR_CUDA;
+  if (dev < 0 || dev >= kMaxDevices) return S2O_ERR_UNSUPPORTED_SHAPE;
+  void* scratch = nullptr;
+  {
+    std::lock_guard<std::mutex> lock(g_scratch_mu);
+    if (!g_scratch_addr[dev]) {
+      // In host code the array's name is only a host-side handle; the device
+      // address comes from the runtime, with this device current.
+      void* p = nullptr;
+      if (cudaGetSymbolAddress(&p, g_s2o_plan_scratch) != cudaSuccess || !p) return S2O_ERR_CUDA;
+      g_scratch_addr[dev] = p;
+    }
+    scratch = g_scratch_addr[dev];
+  }
+  return s2o_plan(cfg, Q, K, scores, perm, nblocks, seg_stats, scratch, kNoAllocScratchBytes, stream);
 }
 
 const char* s2o_status_string(s2o_status st) {
