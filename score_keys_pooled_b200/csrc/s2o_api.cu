@@ -10,6 +10,7 @@
 #include "pool_score.cuh"
 #include "seg_sort.cuh"
 #include "sparse_attn.cuh"
+#include "sparse_attn2.cuh"
 
 using namespace s2o;
 
@@ -81,6 +82,8 @@ cudaError_t set_kernel_attributes() {
     cudaError_t e = cudaFuncSetAttribute(k_score, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kScoreSmem);
     if (e == cudaSuccess)
       e = cudaFuncSetAttribute(k_sparse_attn, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kAttnSmem);
+    if (e == cudaSuccess)
+      e = cudaFuncSetAttribute(k_sparse_attn2, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kAttn2Smem);
     if (e == cudaSuccess)
       e = cudaFuncSetAttribute(k_contig_plan, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                (int)(kContigMaxBlocks * sizeof(unsigned long long)));
@@ -189,13 +192,26 @@ s2o_status s2o_attention(const s2o_config* cfg, const uint16_t* Q, const uint16_
   if (!aligned16(Q) || !aligned16(K) || !aligned16(V) || !aligned16(O) || !aligned16(perm))
     return S2O_ERR_INVALID_ARG;
   if (set_kernel_attributes() != cudaSuccess) return S2O_ERR_CUDA;
-  AttnArgs a;
-  a.Q = Q; a.K = K; a.V = V; a.perm = perm; a.nblocks = nblocks; a.O = O;
-  a.B = cfg->B; a.Hq = cfg->Hq; a.Hkv = cfg->Hkv; a.N = cfg->N; a.S = nseg(cfg);
-  a.T = ncand_total(cfg);
-  a.out_f32 = out_dtype == S2O_OUT_F32;
-  const int64_t ncta = (int64_t)cfg->B * cfg->Hq * a.S;
-  k_sparse_attn<<<(unsigned)ncta, kAttnThreads, kAttnSmem, reinterpret_cast<cudaStream_t>(stream)>>>(a);
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  const int G = cfg->Hq / cfg->Hkv;
+  if (G % 2 == 0) {
+    // two query heads of a KV group per CTA share every gathered K/V tile
+    Attn2Args a;
+    a.Q = Q; a.K = K; a.V = V; a.perm = perm; a.nblocks = nblocks; a.O = O;
+    a.B = cfg->B; a.Hq = cfg->Hq; a.Hkv = cfg->Hkv; a.N = cfg->N; a.S = nseg(cfg);
+    a.T = ncand_total(cfg);
+    a.out_f32 = out_dtype == S2O_OUT_F32;
+    const int64_t ncta = (int64_t)cfg->B * cfg->Hkv * a.S * (G / 2);
+    k_sparse_attn2<<<(unsigned)ncta, kAttn2Threads, kAttn2Smem, s>>>(a);
+  } else {
+    AttnArgs a;
+    a.Q = Q; a.K = K; a.V = V; a.perm = perm; a.nblocks = nblocks; a.O = O;
+    a.B = cfg->B; a.Hq = cfg->Hq; a.Hkv = cfg->Hkv; a.N = cfg->N; a.S = nseg(cfg);
+    a.T = ncand_total(cfg);
+    a.out_f32 = out_dtype == S2O_OUT_F32;
+    const int64_t ncta = (int64_t)cfg->B * cfg->Hq * a.S;
+    k_sparse_attn<<<(unsigned)ncta, kAttnThreads, kAttnSmem, s>>>(a);
+  }
   ++t_launches;
   return launch_status();
 }

@@ -1,0 +1,391 @@
+// Kernel (3), GQA form: two query heads of a KV group per CTA, warp-specialised.
+//
+// Same method as k_sparse_attn (gist.science technical summary, section 3:
+// pass 1 = the segment's dense causal window, pass 2 = keys in permuted order
+// up to the stop; section 1, "Chargement Planifie par Coordonnees": K/V rows
+// gathered by index), laid out for the B200 tensor core:
+//
+//   * one CTA = (b, kvh, s, pair): query heads h0 = kvh*G + 2*pair and h0+1
+//     share every gathered K/V tile (each tile is fetched once for 256 rows);
+//   * 128-key tiles: 64-key blocks of the key walk taken two at a time
+//     (diagonal, previous window, sinks, then the kept candidate blocks; an
+//     odd last block leaves an empty, zero-filled and masked half);
+//   * warp roles (352 threads): warps 0-3 and 4-7 run the online softmax of
+//     head 0 and head 1 (thread = row = TMEM lane), warp 8 issues tcgen05.mma
+//     from one thread, warps 9-10 gather K/V rows with 16-byte cp.async into a
+//     2-stage ring of 128B-swizzled tiles and signal an mbarrier on completion;
+//   * tensor memory (512 columns): S_i = Q_i K^T in columns [128 i, 128 i+128),
+//     O_i in [256 + 128 i, ...); P_i (bf16, two per column) overwrites the
+//     first 64 columns of S_i and is the A operand of O_i += P_i V straight
+//     from tensor memory, so P never touches shared memory;
+//   * while one head's softmax runs, the tensor core works on the other
+//     head's products (ping-pong through the mbarriers below).
+// Online softmax: exp2 domain, lazy rescale (the row's reference max moves
+// only when it grows by more than 2^8, which leaves the result exact).
+// Every mbarrier wait is bounded; a wait that runs out sets the device error
+// word and the CTA winds down without hanging.
+#pragma once
+#include "s2o_common.cuh"
+
+namespace s2o {
+
+constexpr int kKT2 = 128;                 // keys per tile
+constexpr int kAttn2Threads = 352;
+constexpr int kMmaWarp = 8;
+constexpr int kLoadWarp0 = 9;
+constexpr int kLoadThreads = 64;  // the row mapping below assumes 2 loader warps
+constexpr int kStages2 = 2;
+constexpr uint32_t kTile2Bytes = 2 * 128 * 128;      // one 128-row operand tile: 2 atoms x 128 rows x 128 B
+constexpr uint32_t kOff2Q = 0;                       // Q0, Q1
+constexpr uint32_t kOff2KV = 2 * kTile2Bytes;        // stage st: K at +2*st*tile, V at +(2*st+1)*tile
+constexpr uint32_t kOff2Bar = kOff2KV + 2 * kStages2 * kTile2Bytes;
+constexpr uint32_t kAttn2SmemData = kOff2Bar + 256;
+constexpr size_t kAttn2Smem = kAttn2SmemData + 1024;  // + alignment slack
+constexpr uint32_t kTmem2Cols = 512;
+
+// barrier slots (8 bytes each) from kOff2Bar
+constexpr int kBarKvFull = 0;   // [2]  loader -> MMA (count 64, cp.async arrive)
+constexpr int kBarKvEmpty = 2;  // [2]  MMA commit -> loader
+constexpr int kBarQFull = 4;    //      loader -> MMA (count 64)
+constexpr int kBarSFull = 5;    // [2]  MMA commit -> softmax i
+constexpr int kBarPFull = 7;    // [2]  softmax i (count 128) -> MMA
+constexpr int kBarODone = 9;    // [2]  MMA commit -> softmax i
+constexpr int kSlotTmem = 11;
+
+__device__ __forceinline__ void tc_mma_ts(uint32_t d_tmem, uint32_t a_tmem, uint64_t bdesc, uint32_t idesc,
+                                          uint32_t accumulate) {
+  asm volatile(
+      "{\n .reg .pred p;\n"
+      " setp.ne.b32 p, %4, 0;\n"
+      " tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n}\n" ::"r"(d_tmem),
+      "r"(a_tmem), "l"(bdesc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+__device__ __forceinline__ void mbar_arrive(uint32_t bar) {
+  asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];\n" ::"r"(bar) : "memory");
+}
+// arrive on `bar` once all cp.async of this thread issued so far have landed
+__device__ __forceinline__ void cp_async_arrive(uint32_t bar) {
+  asm volatile("cp.async.mbarrier.arrive.noinc.shared::cta.b64 [%0];\n" ::"r"(bar) : "memory");
+}
+// warp-uniform bounded wait: every lane polls, all agree on the outcome
+__device__ __forceinline__ bool warp_wait(uint32_t bar, uint32_t parity) {
+  const bool ok = mbar_wait_bounded(bar, parity);
+  return __all_sync(0xffffffffu, ok);
+}
+
+// 64-key block b of a work item: kind 0 = diagonal (causal, keys j0..j0+63),
+// 1 = contiguous, 2 = gathered candidate block j0 of perm, 3 = empty.
+struct Walk2 {
+  int n_diag, n_prev, n_sink, nb;
+};
+__device__ __forceinline__ Walk2 make_walk2(int s, int N, int C) {
+  Walk2 w;
+  const int rows = min(N, kLq * s + kLq) - kLq * s;
+  w.n_diag = (rows + kBk - 1) / kBk;
+  w.n_prev = (s >= 1) ? 2 : 0;
+  w.n_sink = (s >= 2) ? 1 : 0;
+  w.nb = w.n_diag + w.n_prev + w.n_sink + C;
+  return w;
+}
+__device__ __forceinline__ int walk2_block(const Walk2& w, int s, int b, int& j0) {
+  if (b >= w.nb) { j0 = 0; return 3; }
+  if (b < w.n_diag) { j0 = kLq * s + kBk * b; return 0; }
+  b -= w.n_diag;
+  if (b < w.n_prev) { j0 = kLq * s - kLq + kBk * b; return 1; }
+  b -= w.n_prev;
+  if (b < w.n_sink) { j0 = 0; return 1; }
+  j0 = b - w.n_sink;
+  return 2;
+}
+
+struct Attn2Args {
+  const uint16_t* Q;
+  const uint16_t* K;
+  const uint16_t* V;
+  const int32_t* perm;
+  const int32_t* nblocks;
+  void* O;
+  int B, Hq, Hkv, N, S;
+  int64_t T;
+  int out_f32;
+};
+
+__global__ void __launch_bounds__(kAttn2Threads, 1) k_sparse_attn2(Attn2Args a) {
+  extern __shared__ uint8_t smem_raw[];
+  const uint32_t sbase = (smem_u32(smem_raw) + 1023u) & ~1023u;
+  uint8_t* sgen = smem_raw + (sbase - smem_u32(smem_raw));
+  auto bar = [&](int k) { return sbase + kOff2Bar + 8u * (uint32_t)k; };
+  volatile uint32_t* tmem_slot = reinterpret_cast<volatile uint32_t*>(sgen + kOff2Bar + 8 * kSlotTmem);
+
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int G = a.Hq / a.Hkv;
+  const int pairs = G / 2;
+  const int w = blockIdx.x;
+  const int per_s = a.B * a.Hkv * pairs;
+  const int s = a.S - 1 - w / per_s;
+  const int rest = w % per_s;
+  const int bk = rest / pairs, pair = rest % pairs;
+  const int b = bk / a.Hkv, kvh = bk % a.Hkv;
+  const int h0 = kvh * G + 2 * pair;
+
+  int C = a.nblocks[(size_t)bk * a.S + s];
+  const int cmax = (int)(num_cand(s) / kBk);
+  if (C < 0 || C > cmax) {
+    if (tid == 0) set_error(kErrBadPlan);
+    C = C < 0 ? 0 : cmax;
+  }
+  const Walk2 wk = make_walk2(s, a.N, C);
+  const int ntiles = (wk.nb + 1) / 2;
+  const int row0 = kLq * s;
+
+  if (tid == 0) {
+    for (int k = 0; k < kSlotTmem; ++k) {
+      uint32_t count = 1;
+      if (k == kBarKvFull || k == kBarKvFull + 1 || k == kBarQFull) count = kLoadThreads;
+      if (k == kBarPFull || k == kBarPFull + 1) count = 128;
+      mbar_init(bar(k), count);
+    }
+    fence_mbar_init();
+  }
+  if (warp == kMmaWarp) {
+    tmem_alloc(smem_u32((const void*)tmem_slot), kTmem2Cols);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+
+  if (warp >= kLoadWarp0) {
+    // ------------------------------------------------------------------ loader
+    const int lw = warp - kLoadWarp0;
+    const int c16 = lane & 15, rsub = lane >> 4;
+    const uint32_t atom_off = (uint32_t)(c16 >> 3) * (128 * 128);
+    const uint32_t chunk = (uint32_t)(c16 & 7);
+    // Q tiles of the two heads: 2 x 64 row pairs
+    for (int p = lw; p < 128; p += kLoadThreads / 32) {
+      const int qi = p >> 6;
+      const int r = 2 * (p & 63) + rsub;
+      const bool ok = row0 + r < a.N;
+      const uint16_t* src = a.Q + ((size_t)(b * a.Hq + h0 + qi) * a.N + (size_t)(ok ? row0 + r : 0)) * kD + 8 * c16;
+      cp_async16(sbase + kOff2Q + qi * kTile2Bytes + atom_off + swz128((uint32_t)r, chunk), src, ok ? 16u : 0u);
+    }
+    cp_async_arrive(bar(kBarQFull));
+    const uint16_t* Kh = a.K + (size_t)bk * a.N * kD;
+    const uint16_t* Vh = a.V + (size_t)bk * a.N * kD;
+    const int32_t* pseg = a.perm + (size_t)bk * a.T + cand_offset(s);
+    const int cand_hi = kLq * s - kWin;
+    for (int t = 0; t < ntiles; ++t) {
+      const int st = t & 1;
+      if (!warp_wait(bar(kBarKvEmpty + st), (uint32_t)(((t >> 1) & 1) ^ 1))) {
+        if (lane == 0) set_error(kErrTimeout);
+        break;
+      }
+      const uint32_t sK = sbase + kOff2KV + (2 * st) * kTile2Bytes;
+      // this thread copies chunk c16 of rows r_i = 4 i + 2 lw + rsub (i < 32) of
+      // both K and V; the row indices are fetched first, as independent loads
+      int ja, jb;
+      const int kind_a = walk2_block(wk, s, 2 * t, ja);
+      const int kind_b = walk2_block(wk, s, 2 * t + 1, jb);
+      int jrow[32];
+#pragma unroll
+      for (int i = 0; i < 32; ++i) {
+        const int r = 4 * i + 2 * lw + rsub;
+        const int kind = i < 16 ? kind_a : kind_b;
+        const int j0 = i < 16 ? ja : jb;
+        int j = -1;  // -1: zero-fill
+        if (kind == 2) {
+          j = pseg[kBk * j0 + (r & 63)];
+          if (j < kSink || j >= cand_hi) {  // caller-supplied plan out of Cand(s)
+            set_error(kErrBadPlan);
+            j = kSink;
+          }
+        } else if (kind != 3) {
+          j = j0 + (r & 63);
+          if (j >= a.N) j = -1;
+        }
+        jrow[i] = j;
+      }
+#pragma unroll
+      for (int m = 0; m < 2; ++m) {
+        const uint16_t* base = m ? Vh : Kh;
+#pragma unroll
+        for (int i = 0; i < 32; ++i) {
+          const int r = 4 * i + 2 * lw + rsub;
+          const int j = jrow[i];
+          const uint16_t* src = base + (size_t)(j >= 0 ? j : 0) * kD + 8 * c16;
+          cp_async16(sK + m * kTile2Bytes + atom_off + swz128((uint32_t)r, chunk), src, j >= 0 ? 16u : 0u);
+        }
+      }
+      cp_async_arrive(bar(kBarKvFull + st));
+    }
+    cp_async_wait_all();
+  } else if (warp == kMmaWarp) {
+    // ------------------------------------------------------------------ MMA issuer
+    if (lane == 0) {
+      const uint32_t idesc_qk = idesc_bf16_f32(128, kKT2, false);
+      const uint32_t idesc_pv = idesc_bf16_f32(128, 128, true);
+      bool ok = mbar_wait_bounded(bar(kBarQFull), 0);
+      for (int t = 0; ok && t <= ntiles; ++t) {
+        for (int i = 0; ok && i < 2; ++i) {
+          if (t > 0) {
+            const int tp = t - 1;
+            ok = mbar_wait_bounded(bar(kBarPFull + i), (uint32_t)(tp & 1));
+            if (!ok) break;
+            tc_fence_after();
+            const uint32_t sV = sbase + kOff2KV + (2 * (tp & 1) + 1) * kTile2Bytes;
+#pragma unroll
+            for (int kk = 0; kk < kKT2 / 16; ++kk) {
+              const uint64_t bd = sdesc_sw128(sV + kk * (16 * 128), 128 * 128, 1024);
+              tc_mma_ts(tmem + 256 + 128 * i, tmem + 128 * i + 8 * kk, bd, idesc_pv, (tp > 0 || kk > 0) ? 1u : 0u);
+            }
+            tc_commit(bar(kBarODone + i));
+          }
+          if (t < ntiles) {
+            if (i == 0) {
+              ok = mbar_wait_bounded(bar(kBarKvFull + (t & 1)), (uint32_t)((t >> 1) & 1));
+              if (!ok) break;
+              fence_proxy_async_smem();
+            }
+            const uint32_t sQ = sbase + kOff2Q + i * kTile2Bytes;
+            const uint32_t sK = sbase + kOff2KV + (2 * (t & 1)) * kTile2Bytes;
+#pragma unroll
+            for (int kk = 0; kk < 8; ++kk) {
+              const uint64_t ad = sdesc_sw128(sQ + (kk >> 2) * (128 * 128) + (kk & 3) * 32, 16, 1024);
+              const uint64_t bd = sdesc_sw128(sK + (kk >> 2) * (128 * 128) + (kk & 3) * 32, 16, 1024);
+              tc_mma_ss(tmem + 128 * i, ad, bd, idesc_qk, kk > 0 ? 1u : 0u);
+            }
+            tc_commit(bar(kBarSFull + i));
+          }
+        }
+        if (ok && t > 0) tc_commit(bar(kBarKvEmpty + ((t - 1) & 1)));
+      }
+      if (!ok) set_error(kErrTimeout);
+    }
+  } else {
+    // ------------------------------------------------------------------ softmax
+    const int qi = warp >> 2;               // head of the pair
+    const int r = tid & 127;                // row in the segment
+    const int row = row0 + r;
+    const uint32_t lane_base = (uint32_t)((warp & 3) * 32) << 16;
+    const uint32_t tS = tmem + 128 * qi + lane_base;
+    const uint32_t tO = tmem + 256 + 128 * qi + lane_base;
+    const float sl2 = 1.4426950408889634f * 0.08838834764831845f;  // log2(e) / sqrt(d)
+    float m_run = -INFINITY, ell = 0.f;
+    bool ok = true;
+    for (int t = 0; t < ntiles; ++t) {
+      if (!warp_wait(bar(kBarSFull + qi), (uint32_t)(t & 1))) { ok = false; break; }
+      tc_fence_after();
+      // key c of a half is visible iff (c mod 64) <= lim of that half
+      int lim_a, lim_b;
+      {
+        int j0;
+        const int ka = walk2_block(wk, s, 2 * t, j0);
+        lim_a = ka == 3 ? -1 : (ka == 0 ? row - j0 : kBk);
+        const int kb = walk2_block(wk, s, 2 * t + 1, j0);
+        lim_b = kb == 3 ? -1 : (kb == 0 ? row - j0 : kBk);
+      }
+      // pass 1: row max of the tile, streaming S from tensor memory
+      float mt = -INFINITY;
+#pragma unroll
+      for (int cc = 0; cc < kKT2; cc += 32) {
+        float v[32];
+        tmem_ld32(tS + cc, v);
+        tc_wait_ld();
+        const int lim = cc < 64 ? lim_a : lim_b;
+#pragma unroll
+        for (int k = 0; k < 32; ++k)
+          if (((cc + k) & 63) <= lim) mt = fmaxf(mt, v[k]);
+      }
+      mt *= sl2;
+      const bool move = mt > m_run + 8.f;
+      float alpha = 1.f;
+      if (move) {
+        alpha = (m_run == -INFINITY) ? 0.f : ex2_approx(m_run - mt);
+        m_run = mt;
+        ell *= alpha;
+      }
+      // the previous P V must be done before P_i and O_i are rewritten (it was
+      // issued before this tile's S, so this wait normally returns at once)
+      if (t > 0) {
+        if (!warp_wait(bar(kBarODone + qi), (uint32_t)((t - 1) & 1))) { ok = false; break; }
+        tc_fence_after();
+        if (__any_sync(0xffffffffu, move)) {
+#pragma unroll
+          for (int cc = 0; cc < 128; cc += 32) {
+            float o[32];
+            tmem_ld32(tO + cc, o);
+            tc_wait_ld();
+#pragma unroll
+            for (int k = 0; k < 32; ++k) o[k] *= alpha;
+            tmem_st32(tO + cc, o);
+          }
+        }
+      }
+      // pass 2: P = exp2(S - m), packed bf16 pairs written over the S columns
+      // already read (P chunk k lands in columns [16k, 16k+16) < 32(k+1))
+      float rs = 0.f;
+#pragma unroll
+      for (int cc = 0; cc < kKT2; cc += 32) {
+        float v[32];
+        tmem_ld32(tS + cc, v);
+        tc_wait_ld();
+        const int lim = cc < 64 ? lim_a : lim_b;
+        uint32_t pk[16];
+#pragma unroll
+        for (int k = 0; k < 32; k += 2) {
+          const float p0 = (((cc + k) & 63) <= lim) ? ex2_approx(v[k] * sl2 - m_run) : 0.f;
+          const float p1 = (((cc + k + 1) & 63) <= lim) ? ex2_approx(v[k + 1] * sl2 - m_run) : 0.f;
+          rs += p0 + p1;
+          pk[k / 2] = pack_bf16x2(p0, p1);
+        }
+        tmem_st16(tS + cc / 2, pk);
+      }
+      ell += rs;
+      tc_wait_st();
+      tc_fence_before();
+      mbar_arrive(bar(kBarPFull + qi));
+    }
+    if (ok) ok = warp_wait(bar(kBarODone + qi), (uint32_t)((ntiles - 1) & 1));
+    if (!ok) {
+      if (lane == 0) set_error(kErrTimeout);
+    } else {
+      tc_fence_after();
+      const float inv = ell > 0.f ? 1.f / ell : 0.f;
+      const bool store = row < a.N;
+      const size_t orow = ((size_t)(b * a.Hq + h0 + qi) * a.N + (size_t)(store ? row : 0)) * kD;
+#pragma unroll
+      for (int cc = 0; cc < 128; cc += 32) {
+        float o[32];
+        tmem_ld32(tO + cc, o);
+        tc_wait_ld();
+        if (store) {
+          if (a.out_f32) {
+            float4* dst = reinterpret_cast<float4*>(static_cast<float*>(a.O) + orow + cc);
+#pragma unroll
+            for (int k = 0; k < 8; ++k)
+              dst[k] = make_float4(o[4 * k] * inv, o[4 * k + 1] * inv, o[4 * k + 2] * inv, o[4 * k + 3] * inv);
+          } else {
+            uint4* dst = reinterpret_cast<uint4*>(static_cast<uint16_t*>(a.O) + orow + cc);
+#pragma unroll
+            for (int k = 0; k < 4; ++k)
+              dst[k] = make_uint4(pack_bf16x2(o[8 * k] * inv, o[8 * k + 1] * inv),
+                                  pack_bf16x2(o[8 * k + 2] * inv, o[8 * k + 3] * inv),
+                                  pack_bf16x2(o[8 * k + 4] * inv, o[8 * k + 5] * inv),
+                                  pack_bf16x2(o[8 * k + 6] * inv, o[8 * k + 7] * inv));
+          }
+        }
+      }
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == kMmaWarp) {
+    tc_fence_after();
+    tmem_dealloc(tmem, kTmem2Cols);
+  }
+}
+
+}  // namespace s2o

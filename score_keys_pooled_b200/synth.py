@@ -51,6 +51,8 @@ WORKLOADS = {
     "tiny_1k": Workload("tiny_1k", 1, 1, 1, 1024, 128, 1e-3, True, False, 8),
     # Llama-3.1-8B-shaped layer at 16K with sinks, 0.5% stripes and a band
     "llama_16k": Workload("llama_16k", 1, 32, 8, 16384, 128, 1e-3, True, True, stripe_count_fraction(16384)),
+    # same generator at 32K: large enough to exceed L2, small enough to profile
+    "llama_32k": Workload("llama_32k", 1, 32, 8, 32768, 128, 1e-3, True, True, stripe_count_fraction(32768)),
     # same generator at 128K: the headline prefill workload
     "llama_128k": Workload("llama_128k", 1, 32, 8, 131072, 128, 1e-3, True, True, stripe_count_fraction(131072)),
     # sinks + 8 stripes, no band, GQA 32/8 at 64K: the tau sweep workload
