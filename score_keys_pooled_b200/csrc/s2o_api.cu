@@ -92,6 +92,38 @@ cudaError_t set_kernel_attributes() {
   return g_attr_err;
 }
 
+// Tensor-map encoder of the driver, fetched through the runtime once.
+using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                   const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                   CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+std::once_flag g_encode_once;
+EncodeTiledFn g_encode = nullptr;
+
+EncodeTiledFn tensor_map_encoder() {
+  std::call_once(g_encode_once, [] {
+    void* fn = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &fn, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      g_encode = reinterpret_cast<EncodeTiledFn>(fn);
+  });
+  return g_encode;
+}
+
+// [rows, 128] bf16 rows of 256 bytes, boxes of 64 columns x box_rows rows,
+// 128-byte swizzle (the layout the tensor-core descriptors expect).
+bool encode_rows_map(CUtensorMap* map, const void* base, uint64_t rows, uint32_t box_rows) {
+  EncodeTiledFn enc = tensor_map_encoder();
+  if (!enc) return false;
+  const cuuint64_t dims[2] = {(cuuint64_t)kD, (cuuint64_t)rows};
+  const cuuint64_t strides[1] = {(cuuint64_t)kD * 2};
+  const cuuint32_t box[2] = {64, box_rows};
+  const cuuint32_t estr[2] = {1, 1};
+  return enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box, estr,
+             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 // Device address of g_s2o_plan_scratch, looked up once per device.
 std::mutex g_scratch_mu;
 constexpr int kMaxDevices = 64;
@@ -194,15 +226,22 @@ s2o_status s2o_attention(const s2o_config* cfg, const uint16_t* Q, const uint16_
   if (set_kernel_attributes() != cudaSuccess) return S2O_ERR_CUDA;
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
   const int G = cfg->Hq / cfg->Hkv;
-  if (G % 2 == 0) {
+  // row coordinates of the tensor maps are 32-bit
+  const bool rows_fit = (int64_t)cfg->B * cfg->Hq * cfg->N < (int64_t)INT32_MAX;
+  if (G % 2 == 0 && rows_fit) {
     // two query heads of a KV group per CTA share every gathered K/V tile
     Attn2Args a;
     a.Q = Q; a.K = K; a.V = V; a.perm = perm; a.nblocks = nblocks; a.O = O;
     a.B = cfg->B; a.Hq = cfg->Hq; a.Hkv = cfg->Hkv; a.N = cfg->N; a.S = nseg(cfg);
     a.T = ncand_total(cfg);
     a.out_f32 = out_dtype == S2O_OUT_F32;
+    CUtensorMap tmQ, tmK, tmV;
+    if (!encode_rows_map(&tmQ, Q, (uint64_t)cfg->B * cfg->Hq * cfg->N, 128) ||
+        !encode_rows_map(&tmK, K, (uint64_t)cfg->B * cfg->Hkv * cfg->N, 1) ||
+        !encode_rows_map(&tmV, V, (uint64_t)cfg->B * cfg->Hkv * cfg->N, 1))
+      return S2O_ERR_CUDA;
     const int64_t ncta = (int64_t)cfg->B * cfg->Hkv * a.S * (G / 2);
-    k_sparse_attn2<<<(unsigned)ncta, kAttn2Threads, kAttn2Smem, s>>>(a);
+    k_sparse_attn2<<<(unsigned)ncta, kAttn2Threads, kAttn2Smem, s>>>(a, tmQ, tmK, tmV);
   } else {
     AttnArgs a;
     a.Q = Q; a.K = K; a.V = V; a.perm = perm; a.nblocks = nblocks; a.O = O;

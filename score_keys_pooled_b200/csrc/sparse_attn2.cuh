@@ -10,30 +10,37 @@
 //   * 128-key tiles: 64-key blocks of the key walk taken two at a time
 //     (diagonal, previous window, sinks, then the kept candidate blocks; an
 //     odd last block leaves an empty, zero-filled and masked half);
-//   * warp roles (352 threads): warps 0-3 and 4-7 run the online softmax of
+//   * warp roles (384 threads): warps 0-3 and 4-7 run the online softmax of
 //     head 0 and head 1 (thread = row = TMEM lane), warp 8 issues tcgen05.mma
-//     from one thread, warps 9-10 gather K/V rows with 16-byte cp.async into a
-//     2-stage ring of 128B-swizzled tiles and signal an mbarrier on completion;
+//     from one thread, warp 9 gathers K/V rows with TMA (tile::gather4: four
+//     256-byte rows per pair of instructions, one per 64-column half, written
+//     128B-swizzled by the TMA unit) into a 2-stage ring whose mbarriers count
+//     the landed bytes; Q arrives as 2D TMA tiles;
 //   * tensor memory (512 columns): S_i = Q_i K^T in columns [128 i, 128 i+128),
 //     O_i in [256 + 128 i, ...); P_i (bf16, two per column) overwrites the
 //     first 64 columns of S_i and is the A operand of O_i += P_i V straight
 //     from tensor memory, so P never touches shared memory;
 //   * while one head's softmax runs, the tensor core works on the other
-//     head's products (ping-pong through the mbarriers below).
+//     head's products (ping-pong through the mbarriers below);
+//   * registers are rebalanced per warpgroup (setmaxnreg): the launch gives
+//     168 per thread; warps 8-11 drop to 80 and the two softmax warpgroups
+//     rise to 208 (per SM sub-partition 2 x 208 + 80 <= 3 x 168), enough to
+//     hold a thread's 128 scores of a tile at once.
 // Online softmax: exp2 domain, lazy rescale (the row's reference max moves
 // only when it grows by more than 2^8, which leaves the result exact).
 // Every mbarrier wait is bounded; a wait that runs out sets the device error
 // word and the CTA winds down without hanging.
 #pragma once
+#include <cuda.h>  // CUtensorMap (the encoder is fetched from the driver at run time)
+
 #include "s2o_common.cuh"
 
 namespace s2o {
 
 constexpr int kKT2 = 128;                 // keys per tile
-constexpr int kAttn2Threads = 352;
+constexpr int kAttn2Threads = 384;
 constexpr int kMmaWarp = 8;
 constexpr int kLoadWarp0 = 9;
-constexpr int kLoadThreads = 64;  // the row mapping below assumes 2 loader warps
 constexpr int kStages2 = 2;
 constexpr uint32_t kTile2Bytes = 2 * 128 * 128;      // one 128-row operand tile: 2 atoms x 128 rows x 128 B
 constexpr uint32_t kOff2Q = 0;                       // Q0, Q1
@@ -44,9 +51,9 @@ constexpr size_t kAttn2Smem = kAttn2SmemData + 1024;  // + alignment slack
 constexpr uint32_t kTmem2Cols = 512;
 
 // barrier slots (8 bytes each) from kOff2Bar
-constexpr int kBarKvFull = 0;   // [2]  loader -> MMA (count 64, cp.async arrive)
+constexpr int kBarKvFull = 0;   // [2]  loader -> MMA (TMA bytes)
 constexpr int kBarKvEmpty = 2;  // [2]  MMA commit -> loader
-constexpr int kBarQFull = 4;    //      loader -> MMA (count 64)
+constexpr int kBarQFull = 4;    //      loader -> MMA (TMA bytes)
 constexpr int kBarSFull = 5;    // [2]  MMA commit -> softmax i
 constexpr int kBarPFull = 7;    // [2]  softmax i (count 128) -> MMA
 constexpr int kBarODone = 9;    // [2]  MMA commit -> softmax i
@@ -61,12 +68,38 @@ __device__ __forceinline__ void tc_mma_ts(uint32_t d_tmem, uint32_t a_tmem, uint
       "r"(a_tmem), "l"(bdesc), "r"(idesc), "r"(accumulate)
       : "memory");
 }
+template <uint32_t R>
+__device__ __forceinline__ void regs_increase() {
+  asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;\n" ::"n"(R));
+}
+template <uint32_t R>
+__device__ __forceinline__ void regs_decrease() {
+  asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;\n" ::"n"(R));
+}
+constexpr uint32_t kRegsSoftmax = 208, kRegsOther = 80;
+static_assert(2 * kRegsSoftmax + kRegsOther <= 3 * 168, "register split exceeds the launch's budget");
+
 __device__ __forceinline__ void mbar_arrive(uint32_t bar) {
   asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];\n" ::"r"(bar) : "memory");
 }
-// arrive on `bar` once all cp.async of this thread issued so far have landed
-__device__ __forceinline__ void cp_async_arrive(uint32_t bar) {
-  asm volatile("cp.async.mbarrier.arrive.noinc.shared::cta.b64 [%0];\n" ::"r"(bar) : "memory");
+__device__ __forceinline__ void mbar_expect_tx(uint32_t bar, uint32_t bytes) {
+  asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;\n" ::"r"(bar), "r"(bytes) : "memory");
+}
+// 2D tiled TMA load (box of the tensor map) into shared memory
+__device__ __forceinline__ void tma_load_2d(uint32_t dst, const CUtensorMap* map, int x, int y, uint32_t bar) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3}], [%4];\n" ::"r"(dst),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(bar)
+      : "memory");
+}
+// four rows y0..y3, columns [x, x + box width), landing as four consecutive rows
+__device__ __forceinline__ void tma_gather4(uint32_t dst, const CUtensorMap* map, int x, int y0, int y1, int y2,
+                                            int y3, uint32_t bar) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.shared::cluster.global.tile::gather4.mbarrier::complete_tx::bytes"
+      " [%0], [%1, {%2, %3, %4, %5, %6}], [%7];\n" ::"r"(dst),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y0), "r"(y1), "r"(y2), "r"(y3), "r"(bar)
+      : "memory");
 }
 // warp-uniform bounded wait: every lane polls, all agree on the outcome
 __device__ __forceinline__ bool warp_wait(uint32_t bar, uint32_t parity) {
@@ -111,7 +144,9 @@ struct Attn2Args {
   int out_f32;
 };
 
-__global__ void __launch_bounds__(kAttn2Threads, 1) k_sparse_attn2(Attn2Args a) {
+__global__ void __launch_bounds__(kAttn2Threads, 1)
+    k_sparse_attn2(Attn2Args a, const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
+                   const __grid_constant__ CUtensorMap tmV) {
   extern __shared__ uint8_t smem_raw[];
   const uint32_t sbase = (smem_u32(smem_raw) + 1023u) & ~1023u;
   uint8_t* sgen = smem_raw + (sbase - smem_u32(smem_raw));
@@ -142,7 +177,6 @@ __global__ void __launch_bounds__(kAttn2Threads, 1) k_sparse_attn2(Attn2Args a) 
   if (tid == 0) {
     for (int k = 0; k < kSlotTmem; ++k) {
       uint32_t count = 1;
-      if (k == kBarKvFull || k == kBarKvFull + 1 || k == kBarQFull) count = kLoadThreads;
       if (k == kBarPFull || k == kBarPFull + 1) count = 128;
       mbar_init(bar(k), count);
     }
@@ -156,73 +190,68 @@ __global__ void __launch_bounds__(kAttn2Threads, 1) k_sparse_attn2(Attn2Args a) 
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
-
-  if (warp >= kLoadWarp0) {
-    // ------------------------------------------------------------------ loader
-    const int lw = warp - kLoadWarp0;
-    const int c16 = lane & 15, rsub = lane >> 4;
-    const uint32_t atom_off = (uint32_t)(c16 >> 3) * (128 * 128);
-    const uint32_t chunk = (uint32_t)(c16 & 7);
-    // Q tiles of the two heads: 2 x 64 row pairs
-    for (int p = lw; p < 128; p += kLoadThreads / 32) {
-      const int qi = p >> 6;
-      const int r = 2 * (p & 63) + rsub;
-      const bool ok = row0 + r < a.N;
-      const uint16_t* src = a.Q + ((size_t)(b * a.Hq + h0 + qi) * a.N + (size_t)(ok ? row0 + r : 0)) * kD + 8 * c16;
-      cp_async16(sbase + kOff2Q + qi * kTile2Bytes + atom_off + swz128((uint32_t)r, chunk), src, ok ? 16u : 0u);
+  if (warp > kLoadWarp0) {
+    // warps 10-11: no role (they complete the register-donating warpgroup)
+    regs_decrease<kRegsOther>();
+  } else if (warp == kLoadWarp0) {
+    // ------------------------------------------------------------------ loader (TMA)
+    regs_decrease<kRegsOther>();
+    // rows of K/V as [B*Hkv*N, 128]; a row coordinate past the end is out of
+    // bounds and reads as zeros (empty halves, keys past N)
+    const int zero_row = a.B * a.Hkv * a.N;
+    const int kv_row0 = bk * a.N;
+    if (lane == 0) {
+      mbar_expect_tx(bar(kBarQFull), 2 * kTile2Bytes);
+#pragma unroll
+      for (int qi = 0; qi < 2; ++qi)
+#pragma unroll
+        for (int half = 0; half < 2; ++half)
+          tma_load_2d(sbase + kOff2Q + qi * kTile2Bytes + half * (128 * 128), &tmQ, 64 * half,
+                      (b * a.Hq + h0 + qi) * a.N + row0, bar(kBarQFull));
     }
-    cp_async_arrive(bar(kBarQFull));
-    const uint16_t* Kh = a.K + (size_t)bk * a.N * kD;
-    const uint16_t* Vh = a.V + (size_t)bk * a.N * kD;
     const int32_t* pseg = a.perm + (size_t)bk * a.T + cand_offset(s);
     const int cand_hi = kLq * s - kWin;
     for (int t = 0; t < ntiles; ++t) {
       const int st = t & 1;
-      if (!warp_wait(bar(kBarKvEmpty + st), (uint32_t)(((t >> 1) & 1) ^ 1))) {
-        if (lane == 0) set_error(kErrTimeout);
-        break;
-      }
-      const uint32_t sK = sbase + kOff2KV + (2 * st) * kTile2Bytes;
-      // this thread copies chunk c16 of rows r_i = 4 i + 2 lw + rsub (i < 32) of
-      // both K and V; the row indices are fetched first, as independent loads
-      int ja, jb;
-      const int kind_a = walk2_block(wk, s, 2 * t, ja);
-      const int kind_b = walk2_block(wk, s, 2 * t + 1, jb);
-      int jrow[32];
+      // rows 4 lane .. 4 lane + 3 of the tile: their key indices first (these
+      // loads overlap the wait for the stage to drain)
+      const int blk = 2 * t + (lane >> 4);
+      int j0;
+      const int kind = walk2_block(wk, s, blk, j0);
+      int y[4];
 #pragma unroll
-      for (int i = 0; i < 32; ++i) {
-        const int r = 4 * i + 2 * lw + rsub;
-        const int kind = i < 16 ? kind_a : kind_b;
-        const int j0 = i < 16 ? ja : jb;
-        int j = -1;  // -1: zero-fill
+      for (int k = 0; k < 4; ++k) {
+        const int rr = (4 * lane + k) & 63;
+        int j = -1;
         if (kind == 2) {
-          j = pseg[kBk * j0 + (r & 63)];
+          j = pseg[kBk * j0 + rr];
           if (j < kSink || j >= cand_hi) {  // caller-supplied plan out of Cand(s)
             set_error(kErrBadPlan);
             j = kSink;
           }
         } else if (kind != 3) {
-          j = j0 + (r & 63);
+          j = j0 + rr;
           if (j >= a.N) j = -1;
         }
-        jrow[i] = j;
+        y[k] = j >= 0 ? kv_row0 + j : zero_row;
       }
-#pragma unroll
-      for (int m = 0; m < 2; ++m) {
-        const uint16_t* base = m ? Vh : Kh;
-#pragma unroll
-        for (int i = 0; i < 32; ++i) {
-          const int r = 4 * i + 2 * lw + rsub;
-          const int j = jrow[i];
-          const uint16_t* src = base + (size_t)(j >= 0 ? j : 0) * kD + 8 * c16;
-          cp_async16(sK + m * kTile2Bytes + atom_off + swz128((uint32_t)r, chunk), src, j >= 0 ? 16u : 0u);
-        }
+      if (!warp_wait(bar(kBarKvEmpty + st), (uint32_t)(((t >> 1) & 1) ^ 1))) {
+        if (lane == 0) set_error(kErrTimeout);
+        break;
       }
-      cp_async_arrive(bar(kBarKvFull + st));
+      if (lane == 0) mbar_expect_tx(bar(kBarKvFull + st), 2 * kTile2Bytes);
+      __syncwarp();
+      const uint32_t sK = sbase + kOff2KV + (2 * st) * kTile2Bytes;
+#pragma unroll
+      for (int m = 0; m < 2; ++m)
+#pragma unroll
+        for (int half = 0; half < 2; ++half)
+          tma_gather4(sK + m * kTile2Bytes + half * (128 * 128) + lane * (4 * 128), m ? &tmV : &tmK, 64 * half,
+                      y[0], y[1], y[2], y[3], bar(kBarKvFull + st));
     }
-    cp_async_wait_all();
   } else if (warp == kMmaWarp) {
     // ------------------------------------------------------------------ MMA issuer
+    regs_decrease<kRegsOther>();
     if (lane == 0) {
       const uint32_t idesc_qk = idesc_bf16_f32(128, kKT2, false);
       const uint32_t idesc_pv = idesc_bf16_f32(128, 128, true);
@@ -246,7 +275,6 @@ __global__ void __launch_bounds__(kAttn2Threads, 1) k_sparse_attn2(Attn2Args a) 
             if (i == 0) {
               ok = mbar_wait_bounded(bar(kBarKvFull + (t & 1)), (uint32_t)((t >> 1) & 1));
               if (!ok) break;
-              fence_proxy_async_smem();
             }
             const uint32_t sQ = sbase + kOff2Q + i * kTile2Bytes;
             const uint32_t sK = sbase + kOff2KV + (2 * (t & 1)) * kTile2Bytes;
@@ -265,6 +293,7 @@ __global__ void __launch_bounds__(kAttn2Threads, 1) k_sparse_attn2(Attn2Args a) 
     }
   } else {
     // ------------------------------------------------------------------ softmax
+    regs_increase<kRegsSoftmax>();
     const int qi = warp >> 2;               // head of the pair
     const int r = tid & 127;                // row in the segment
     const int row = row0 + r;
@@ -286,18 +315,15 @@ __global__ void __launch_bounds__(kAttn2Threads, 1) k_sparse_attn2(Attn2Args a) 
         const int kb = walk2_block(wk, s, 2 * t + 1, j0);
         lim_b = kb == 3 ? -1 : (kb == 0 ? row - j0 : kBk);
       }
-      // pass 1: row max of the tile, streaming S from tensor memory
+      // the tile's 128 scores of this row, one tensor-memory round trip
+      float x[kKT2];
+#pragma unroll
+      for (int cc = 0; cc < kKT2; cc += 32) tmem_ld32(tS + cc, x + cc);
+      tc_wait_ld();
       float mt = -INFINITY;
 #pragma unroll
-      for (int cc = 0; cc < kKT2; cc += 32) {
-        float v[32];
-        tmem_ld32(tS + cc, v);
-        tc_wait_ld();
-        const int lim = cc < 64 ? lim_a : lim_b;
-#pragma unroll
-        for (int k = 0; k < 32; ++k)
-          if (((cc + k) & 63) <= lim) mt = fmaxf(mt, v[k]);
-      }
+      for (int c = 0; c < kKT2; ++c)
+        if ((c & 63) <= (c < 64 ? lim_a : lim_b)) mt = fmaxf(mt, x[c]);
       mt *= sl2;
       const bool move = mt > m_run + 8.f;
       float alpha = 1.f;
@@ -306,43 +332,36 @@ __global__ void __launch_bounds__(kAttn2Threads, 1) k_sparse_attn2(Attn2Args a) 
         m_run = mt;
         ell *= alpha;
       }
+      // P = exp2(S - m) as bf16 pairs, packed in place into x[0 .. 63]
+      float rs = 0.f;
+#pragma unroll
+      for (int c = 0; c < kKT2; c += 2) {
+        const int lim = c < 64 ? lim_a : lim_b;
+        const float p0 = ((c & 63) <= lim) ? ex2_approx(fmaf(x[c], sl2, -m_run)) : 0.f;
+        const float p1 = (((c + 1) & 63) <= lim) ? ex2_approx(fmaf(x[c + 1], sl2, -m_run)) : 0.f;
+        rs += p0 + p1;
+        x[c / 2] = __uint_as_float(pack_bf16x2(p0, p1));
+      }
+      ell += rs;
       // the previous P V must be done before P_i and O_i are rewritten (it was
       // issued before this tile's S, so this wait normally returns at once)
       if (t > 0) {
         if (!warp_wait(bar(kBarODone + qi), (uint32_t)((t - 1) & 1))) { ok = false; break; }
         tc_fence_after();
-        if (__any_sync(0xffffffffu, move)) {
+      }
+      tmem_st32(tS, x);
+      tmem_st32(tS + 32, x + 32);
+      if (t > 0 && __any_sync(0xffffffffu, move)) {
 #pragma unroll
-          for (int cc = 0; cc < 128; cc += 32) {
-            float o[32];
-            tmem_ld32(tO + cc, o);
-            tc_wait_ld();
+        for (int cc = 0; cc < 128; cc += 32) {
+          float o[32];
+          tmem_ld32(tO + cc, o);
+          tc_wait_ld();
 #pragma unroll
-            for (int k = 0; k < 32; ++k) o[k] *= alpha;
-            tmem_st32(tO + cc, o);
-          }
+          for (int k = 0; k < 32; ++k) o[k] *= alpha;
+          tmem_st32(tO + cc, o);
         }
       }
-      // pass 2: P = exp2(S - m), packed bf16 pairs written over the S columns
-      // already read (P chunk k lands in columns [16k, 16k+16) < 32(k+1))
-      float rs = 0.f;
-#pragma unroll
-      for (int cc = 0; cc < kKT2; cc += 32) {
-        float v[32];
-        tmem_ld32(tS + cc, v);
-        tc_wait_ld();
-        const int lim = cc < 64 ? lim_a : lim_b;
-        uint32_t pk[16];
-#pragma unroll
-        for (int k = 0; k < 32; k += 2) {
-          const float p0 = (((cc + k) & 63) <= lim) ? ex2_approx(v[k] * sl2 - m_run) : 0.f;
-          const float p1 = (((cc + k + 1) & 63) <= lim) ? ex2_approx(v[k + 1] * sl2 - m_run) : 0.f;
-          rs += p0 + p1;
-          pk[k / 2] = pack_bf16x2(p0, p1);
-        }
-        tmem_st16(tS + cc / 2, pk);
-      }
-      ell += rs;
       tc_wait_st();
       tc_fence_before();
       mbar_arrive(bar(kBarPFull + qi));
