@@ -147,7 +147,7 @@ s2o_status s2o_plan(const s2o_config* cfg, const uint16_t* Q, const uint16_t* K,
  *   Scratch: a 32 MiB array in the library's device memory (a file-scope
  *   __device__ buffer that every GPU loading the library holds until the
  *   process exits).  Configs whose plan workspace (s2o_plan_workspace_size)
- *   exceeds 32 MiB -- e.g. B=1, 8 KV heads, N above ~8K -- are rejected with
+ *   exceeds 32 MiB -- e.g. B=1, 8 KV heads, N above ~7K -- are rejected with
  *   S2O_ERR_WORKSPACE_TOO_SMALL before anything is launched.
  *   The first call on a device looks up the buffer's device address for that
  *   device (make that first call before any stream capture).  Nothing in the

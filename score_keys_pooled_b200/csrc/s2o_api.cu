@@ -9,6 +9,7 @@
 #include "s2o_common.cuh"
 #include "pool_score.cuh"
 #include "seg_sort.cuh"
+#include "seg_sort2.cuh"
 #include "sparse_attn.cuh"
 #include "sparse_attn2.cuh"
 
@@ -50,6 +51,11 @@ struct PlanWs {
   float* segM;
   double* segZ;
   uint32_t *keyA, *keyB, *valA, *valB;
+  float* sorted;
+  BucketSlot* slots;
+  int* mode;
+  float2* range;
+  int64_t nslots;
   size_t bytes;
 };
 
@@ -70,6 +76,13 @@ PlanWs plan_layout(const s2o_config* c, void* base) {
   w.keyB = static_cast<uint32_t*>(take(BH * T * 4 + 16));
   w.valA = static_cast<uint32_t*>(take(BH * T * 4 + 16));
   w.valB = static_cast<uint32_t*>(take(BH * T * 4 + 16));
+  w.sorted = static_cast<float*>(take(BH * T * 4 + 16));
+  int64_t per_bk = 0;
+  for (int s = 0; s < (int)S; ++s) per_bk += bucket_slots(num_cand(s));
+  w.nslots = per_bk * (int64_t)BH;
+  w.slots = static_cast<BucketSlot*>(take((size_t)w.nslots * sizeof(BucketSlot) + 16));
+  w.mode = static_cast<int*>(take(BH * S * sizeof(int)));
+  w.range = static_cast<float2*>(take(BH * S * sizeof(float2)));
   w.bytes = off;
   return w;
 }
@@ -84,6 +97,8 @@ cudaError_t set_kernel_attributes() {
       e = cudaFuncSetAttribute(k_sparse_attn, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kAttnSmem);
     if (e == cudaSuccess)
       e = cudaFuncSetAttribute(k_sparse_attn2, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kAttn2Smem);
+    if (e == cudaSuccess)
+      e = cudaFuncSetAttribute(k_bucket_sort, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kBucketSmem);
     if (e == cudaSuccess)
       e = cudaFuncSetAttribute(k_contig_plan, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                (int)(kContigMaxBlocks * sizeof(unsigned long long)));
@@ -187,8 +202,18 @@ s2o_status s2o_plan(const s2o_config* cfg, const uint16_t* Q, const uint16_t* K,
   const int nwarps = BH * S;
   k_seg_stats<<<(nwarps * 32 + 255) / 256, 256, 0, s>>>(w.part, w.segM, w.segZ, seg_stats, BH, S);
   ++t_launches;
-  k_sort<<<BH * S, kSortThreads, 0, s>>>(scores, w.segM, w.segZ, w.keyA, w.keyB, w.valA, w.valB, perm, nblocks,
-                                         BH, S, T, cfg->tau);
+  k_bucket_plan<<<BH * S, kBucketThreads, 0, s>>>(scores, w.sorted, perm, w.slots, w.mode, w.range, w.keyB, w.valB,
+                                                   BH, S, T);
+  ++t_launches;
+  if (w.nslots > 0) {
+    k_bucket_sort<<<(unsigned)w.nslots, kBucketThreads, kBucketSmem, s>>>(w.keyB, w.valB, w.slots, w.sorted, perm,
+                                                                          T);
+    ++t_launches;
+  }
+  k_sort<<<BH * S, kSortThreads, 0, s>>>(scores, w.segM, w.segZ, w.keyA, w.keyB, w.valA, w.valB, perm, w.sorted,
+                                         w.mode, kModeFallback, BH, S, T);
+  ++t_launches;
+  k_mass_stop<<<BH * S, 256, 0, s>>>(w.sorted, w.segM, w.segZ, nblocks, BH, S, T, cfg->tau);
   ++t_launches;
   return launch_status();
 }

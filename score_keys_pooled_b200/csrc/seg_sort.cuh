@@ -11,8 +11,8 @@
 //   M = max_{A(s)} s_j, Z = sum_{A(s)} exp(s_j - M)       (k_seg_stats)
 //   perm = candidates by s_j descending, ties to the lower index: a stable
 //          LSD radix sort (4 x 8-bit digits) of an order-reversing 32-bit
-//          key over index-ascending input                  (k_sort)
-//   m_b  = sum_{j in block b} exp(s_j - M) / Z,  C = first b with m_b < tau
+//          key over index-ascending input, in global memory (k_sort, the
+//          fallback of the bucketed sorter in seg_sort2.cuh)
 #pragma once
 #include "s2o_common.cuh"
 
@@ -59,7 +59,9 @@ __global__ void k_seg_stats(const float2* __restrict__ part, float* __restrict__
 }
 
 // ---------------------------------------------------------------------------
-// Sort + masses + stop: one 1024-thread CTA per (b, kvh, s), largest first.
+// Global-memory sort: one 1024-thread CTA per (b, kvh, s), largest first.
+// Used for the segments the bucketed sorter hands over (mode[seg] == only):
+// writes perm and the sorted scores; the stop is taken by k_mass_stop.
 // ---------------------------------------------------------------------------
 constexpr int kSortThreads = 1024;
 constexpr int kSortWarps = kSortThreads / 32;
@@ -69,24 +71,20 @@ struct SortSmem {
   uint32_t base[256];             // running bucket starts
   uint32_t total[256];
   int trivial;
-  int cmin;
 };
 
 __global__ void __launch_bounds__(kSortThreads, 2)
     k_sort(const float* __restrict__ scores, const float* __restrict__ segM, const double* __restrict__ segZ,
            uint32_t* __restrict__ keyA, uint32_t* __restrict__ keyB, uint32_t* __restrict__ valA,
-           uint32_t* __restrict__ valB, int32_t* __restrict__ perm, int32_t* __restrict__ nblocks, int BHkv, int S,
-           int64_t T, double tau) {
+           uint32_t* __restrict__ valB, int32_t* __restrict__ perm, float* __restrict__ sorted,
+           const int* __restrict__ mode, int only, int BHkv, int S, int64_t T) {
   __shared__ SortSmem sm;
   const int q = blockIdx.x;
   const int s = S - 1 - q / BHkv;
   const int bk = q % BHkv;
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int n = (int)num_cand(s);
-  if (n == 0) {
-    if (tid == 0) nblocks[(size_t)bk * S + s] = 0;
-    return;
-  }
+  if (n == 0 || mode[(size_t)bk * S + s] != only) return;
   const size_t base = (size_t)bk * T + cand_offset(s);
   const float* sc = scores + base;
   uint32_t* kb[2] = {keyA + base, keyB + base};
@@ -167,27 +165,11 @@ __global__ void __launch_bounds__(kSortThreads, 2)
     cur = out;
   }
 
-  // importance order as absolute key indices
-  for (int i = tid; i < n; i += kSortThreads)
+  // importance order as absolute key indices, and the scores in that order
+  for (int i = tid; i < n; i += kSortThreads) {
     perm[base + i] = kSink + (int32_t)(cur < 0 ? (uint32_t)i : vb[cur][i]);
-
-  // block masses and the stop point
-  const float M = segM[(size_t)bk * S + s];
-  const double Z = segZ[(size_t)bk * S + s];
-  const int nb = n / kBk;  // every candidate block is full
-  if (tid == 0) sm.cmin = nb;
-  __syncthreads();
-  for (int blk = warp; blk < nb; blk += kSortWarps) {
-    const int i0 = blk * kBk + lane, i1 = i0 + 32;
-    const uint32_t k0 = cur < 0 ? desc_key(sc[i0]) : kb[cur][i0];
-    const uint32_t k1 = cur < 0 ? desc_key(sc[i1]) : kb[cur][i1];
-    float e = exp_shifted(key_score(k0), M) + exp_shifted(key_score(k1), M);
-#pragma unroll
-    for (int o = 16; o >= 1; o >>= 1) e += __shfl_xor_sync(0xffffffffu, e, o);
-    if (lane == 0 && (double)e / Z < tau) atomicMin(&sm.cmin, blk);
+    sorted[base + i] = cur < 0 ? sc[i] : key_score(kb[cur][i]);
   }
-  __syncthreads();
-  if (tid == 0) nblocks[(size_t)bk * S + s] = sm.cmin;
 }
 
 // ---------------------------------------------------------------------------

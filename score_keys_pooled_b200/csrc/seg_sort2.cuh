@@ -1,0 +1,475 @@
+// Kernel (2), bucketed form: the importance order of each segment's
+// candidates (gist.science technical summary, section 1: KV_perm; the ranking
+// step that dominates the preprocessing, "Resultats Experimentaux"), sorted
+// mostly on chip.
+//
+//   k_bucket_plan  one CTA per segment: the min and max candidate score, a
+//                  2048-bin histogram that is linear in the score between them
+//                  (bins are monotone in the score, so bin b holds only scores
+//                  >= those of bin b+1, and equal scores share a bin), and
+//                  buckets = runs of consecutive bins whose starting rank falls
+//                  in the same window of kBucketHalf ranks (a bucket holds at
+//                  most kBucketHalf + one bin <= kBucketCap elements); then a
+//                  stable multisplit of the segment into its buckets: (key,
+//                  index) pairs land at the bucket's rank range, in index order;
+//   k_bucket_sort  one CTA per bucket: loads its range into shared memory and
+//                  sorts it there: a counting sort into 4096 fine bins linear
+//                  in the score, then each fine bin (a few elements) by
+//                  (key, index); a bucket with a crowded fine bin is sorted by
+//                  a stable LSD radix sort over the bucket-relative key
+//                  instead; writes perm and the sorted scores at the bucket's
+//                  global rank;
+//   k_mass_stop    block masses of the sorted scores and the stop point C(s).
+// A segment whose scores are all equal is already in index order.  A segment
+// with a bin larger than kBucketCap - kBucketHalf (a heavy cluster of nearly
+// equal scores) is sorted by the global-memory LSD kernel k_sort instead.
+#pragma once
+#include "s2o_common.cuh"
+#include "seg_sort.cuh"
+
+namespace s2o {
+
+constexpr int kNumBins = 2048;
+constexpr int kBucketCap = 11264;             // elements a bucket CTA sorts in shared memory
+constexpr int kBucketHalf = kBucketCap / 2;   // rank window of a bucket
+constexpr int kBucketThreads = 1024;
+constexpr int kMaxBuckets = 128;              // bucket ids per segment (N <= 2^19)
+
+enum SegMode : int { kModeDone = 0, kModeBuckets = 1, kModeFallback = 2 };
+
+struct BucketSlot {
+  int bk, s, bin_lo, bin_hi, base, count;
+};
+
+// slots reserved for a segment of n candidates
+__host__ __device__ __forceinline__ int bucket_slots(int64_t n) {
+  return n == 0 ? 0 : (int)(n / kBucketHalf) + 2;
+}
+
+__device__ __forceinline__ int score_bin(float x, float hi, float scale) {
+  const int b = (int)((hi - x) * scale);
+  return min(max(b, 0), kNumBins - 1);
+}
+
+// block-wide exclusive scan of one value per thread (1024 threads)
+__device__ __forceinline__ int block_excl_scan(int v, int* warp_tot, int& total) {
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  int incl = v;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const int y = __shfl_up_sync(0xffffffffu, incl, o);
+    if (lane >= o) incl += y;
+  }
+  if (lane == 31) warp_tot[warp] = incl;
+  __syncthreads();
+  if (warp == 0) {
+    int w = warp_tot[lane];
+    int wi = w;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int y = __shfl_up_sync(0xffffffffu, wi, o);
+      if (lane >= o) wi += y;
+    }
+    warp_tot[lane] = wi - w;  // exclusive prefix of the warp totals
+    if (lane == 31) warp_tot[32] = wi;
+  }
+  __syncthreads();
+  const int r = warp_tot[warp] + incl - v;
+  total = warp_tot[32];
+  __syncthreads();
+  return r;
+}
+
+// ---------------------------------------------------------------------------
+// planner: one 1024-thread CTA per (b, kvh, s), largest segments first
+// ---------------------------------------------------------------------------
+__global__ void __launch_bounds__(kBucketThreads) k_bucket_plan(const float* __restrict__ scores,
+                                                              float* __restrict__ sorted, int32_t* __restrict__ perm,
+                                                              BucketSlot* __restrict__ slots, int* __restrict__ mode,
+                                                              float2* __restrict__ range,
+                                                              uint32_t* __restrict__ stage_key,
+                                                              uint32_t* __restrict__ stage_val, int BHkv, int S,
+                                                              int64_t T) {
+  __shared__ int hist[kNumBins];
+  __shared__ int wtot[33];
+  __shared__ float red[64];
+  __shared__ int flag;
+  __shared__ uint8_t bin2bkt[kNumBins];
+  __shared__ uint16_t wcnt[kSortWarps][kMaxBuckets];
+  __shared__ int cursor[kMaxBuckets];
+  const int q = blockIdx.x;
+  const int s = S - 1 - q / BHkv;
+  const int bk = q % BHkv;
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int n = (int)num_cand(s);
+  const size_t base = (size_t)bk * T + cand_offset(s);
+  const float* sc = scores + base;
+
+  // slot range of this segment: segments with larger s come first, heads interleaved
+  int before = 0;
+  for (int t = s + 1 + tid; t < S; t += kBucketThreads) before += bucket_slots(num_cand(t));
+  int tot_before;
+  block_excl_scan(before, wtot, tot_before);
+  const int my_slots = bucket_slots(n);
+  BucketSlot* myslot = slots + (size_t)tot_before * BHkv + (size_t)bk * my_slots;
+  for (int k = tid; k < my_slots; k += kBucketThreads) myslot[k].count = 0;
+  if (n == 0) {
+    if (tid == 0) mode[(size_t)bk * S + s] = kModeDone;
+    return;
+  }
+
+  // min and max candidate score
+  float lo = INFINITY, hi = -INFINITY;
+  for (int i = tid; i < n; i += kBucketThreads) {
+    const float x = sc[i];
+    lo = fminf(lo, x);
+    hi = fmaxf(hi, x);
+  }
+#pragma unroll
+  for (int o = 16; o >= 1; o >>= 1) {
+    lo = fminf(lo, __shfl_xor_sync(0xffffffffu, lo, o));
+    hi = fmaxf(hi, __shfl_xor_sync(0xffffffffu, hi, o));
+  }
+  if (lane == 0) { red[warp] = lo; red[32 + warp] = hi; }
+  for (int k = tid; k < kNumBins; k += kBucketThreads) hist[k] = 0;
+  __syncthreads();
+  if (warp == 0) {
+    lo = red[lane];
+    hi = red[32 + lane];
+#pragma unroll
+    for (int o = 16; o >= 1; o >>= 1) {
+      lo = fminf(lo, __shfl_xor_sync(0xffffffffu, lo, o));
+      hi = fmaxf(hi, __shfl_xor_sync(0xffffffffu, hi, o));
+    }
+    if (lane == 0) { red[0] = lo; red[32] = hi; }
+  }
+  __syncthreads();
+  lo = red[0];
+  hi = red[32];
+  if (tid == 0) range[(size_t)bk * S + s] = make_float2(lo, hi);
+  if (!(hi > lo)) {
+    // one value (or non-finite, already flagged by the score kernel): the
+    // importance order is the index order
+    for (int i = tid; i < n; i += kBucketThreads) {
+      sorted[base + i] = sc[i];
+      perm[base + i] = kSink + i;
+    }
+    if (tid == 0) mode[(size_t)bk * S + s] = kModeDone;
+    return;
+  }
+  const float scale = (float)kNumBins / (hi - lo);
+  for (int i = tid; i < n; i += kBucketThreads) atomicAdd(&hist[score_bin(sc[i], hi, scale)], 1);
+  __syncthreads();
+  // exclusive scan over the bins: 2 per thread
+  const int c0 = hist[2 * tid], c1 = hist[2 * tid + 1];
+  int total;
+  const int st0 = block_excl_scan(c0 + c1, wtot, total);
+  const int st1 = st0 + c0;
+  if (tid == 0) flag = 0;
+  __syncthreads();
+  if (c0 > kBucketCap - kBucketHalf || c1 > kBucketCap - kBucketHalf) atomicOr(&flag, 1);
+  __syncthreads();
+  if (flag) {
+    if (tid == 0) mode[(size_t)bk * S + s] = kModeFallback;
+    return;
+  }
+  // a bucket = the bins whose start rank lies in [k*H, (k+1)*H); the thread
+  // of its first bin records the first bin and base rank, the thread of its
+  // last bin the end bin, then (after a barrier) the size
+  hist[2 * tid] = st0;
+  hist[2 * tid + 1] = st1;
+  __syncthreads();
+  int end_id = -1, end_rank = 0;
+#pragma unroll
+  for (int e = 0; e < 2; ++e) {
+    const int b = 2 * tid + e;
+    const int stb = e ? st1 : st0;
+    const int id = stb / kBucketHalf;
+    const bool first = (b == 0) || (hist[b - 1] / kBucketHalf != id);
+    const bool last = (b == kNumBins - 1) || (hist[b + 1] / kBucketHalf != id);
+    if (first) {
+      myslot[id].bk = bk;
+      myslot[id].s = s;
+      myslot[id].bin_lo = b;
+      myslot[id].base = stb;
+    }
+    if (last) {
+      myslot[id].bin_hi = b + 1;
+      end_id = id;
+      end_rank = stb + (e ? c1 : c0);
+    }
+  }
+  __syncthreads();
+  if (end_id >= 0) myslot[end_id].count = end_rank - myslot[end_id].base;
+  // stable multisplit into the buckets, 1024 elements per step in index order
+  bin2bkt[2 * tid] = (uint8_t)(st0 / kBucketHalf);
+  bin2bkt[2 * tid + 1] = (uint8_t)(st1 / kBucketHalf);
+  __syncthreads();
+  // cursor[k] = base rank of bucket k = start rank of its first bin
+#pragma unroll
+  for (int e = 0; e < 2; ++e) {
+    const int b = 2 * tid + e;
+    const int id = bin2bkt[b];
+    if (b == 0 || bin2bkt[b - 1] != id) cursor[id] = e ? st1 : st0;
+  }
+  __syncthreads();
+  const uint32_t lt_mask = (1u << lane) - 1u;
+  uint32_t* skey = stage_key + base;
+  uint32_t* sval = stage_val + base;
+  for (int t0 = 0; t0 < n; t0 += kBucketThreads) {
+    const int i = t0 + tid;
+    const bool valid = i < n;
+    const float x = valid ? sc[i] : 0.f;
+    const uint32_t d = valid ? bin2bkt[score_bin(x, hi, scale)] : 0u;
+    for (int k = lane; k < kMaxBuckets; k += 32) wcnt[warp][k] = 0;
+    __syncwarp();
+    const uint32_t peers = __match_any_sync(0xffffffffu, valid ? d : 1024u + lane);
+    const uint32_t rank = __popc(peers & lt_mask);
+    if (valid && (__ffs(peers) - 1) == lane) wcnt[warp][d] = (uint16_t)__popc(peers);
+    __syncthreads();
+    if (tid < kMaxBuckets) {
+      int run = cursor[tid];
+      for (int w2 = 0; w2 < kSortWarps; ++w2) {
+        const int c = wcnt[w2][tid];
+        wcnt[w2][tid] = (uint16_t)(run - cursor[tid]);
+        run += c;
+      }
+      // offsets within this step are relative to the bucket cursor; the
+      // cursor itself advances after everyone has read it
+      hist[tid] = run;
+    }
+    __syncthreads();
+    if (valid) {
+      const int pos = cursor[d] + wcnt[warp][d] + (int)rank;
+      skey[pos] = desc_key(x);
+      sval[pos] = (uint32_t)i;
+    }
+    __syncthreads();
+    if (tid < kMaxBuckets) cursor[tid] = hist[tid];
+    __syncthreads();
+  }
+  if (tid == 0) mode[(size_t)bk * S + s] = kModeBuckets;
+}
+
+// ---------------------------------------------------------------------------
+// bucket sorter: one 1024-thread CTA per slot
+// ---------------------------------------------------------------------------
+constexpr int kFine = 4096;     // fine bins of a bucket
+constexpr int kFineMax = 64;    // larger fine bins send the bucket to the radix path
+
+__device__ __forceinline__ int fine_bin(float x, float hi, float scale) {
+  const int b = (int)((hi - x) * scale);
+  return min(max(b, 0), kFine - 1);
+}
+
+struct BucketSmem {
+  uint32_t key[2][kBucketCap];
+  uint32_t val[2][kBucketCap];
+  uint32_t cnt[kSortWarps][256];  // radix digit counts, or the kFine fine-bin counters
+  uint32_t dbase[256];
+  int wtot[33];
+  uint32_t kmin, kmax;
+  int big;
+};
+constexpr size_t kBucketSmem = sizeof(BucketSmem);
+
+__global__ void __launch_bounds__(kBucketThreads, 1) k_bucket_sort(const uint32_t* __restrict__ stage_key,
+                                                                  const uint32_t* __restrict__ stage_val,
+                                                                  const BucketSlot* __restrict__ slots,
+                                                                  float* __restrict__ sorted,
+                                                                  int32_t* __restrict__ perm, int64_t T) {
+  extern __shared__ uint8_t bsm_raw[];
+  BucketSmem& sm = *reinterpret_cast<BucketSmem*>(bsm_raw);
+  const BucketSlot slot = slots[blockIdx.x];
+  if (slot.count == 0) return;
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const size_t base = (size_t)slot.bk * T + cand_offset(slot.s);
+  if (tid == 0) { sm.kmin = 0xFFFFFFFFu; sm.kmax = 0u; }
+
+  // the bucket's pairs, already in index order at its rank range
+  const int m = slot.count;
+  uint32_t kmin = 0xFFFFFFFFu, kmax = 0u;
+  for (int i = tid; i < m; i += kBucketThreads) {
+    const uint32_t key = stage_key[base + slot.base + i];
+    kmin = min(kmin, key);
+    kmax = max(kmax, key);
+    sm.key[0][i] = key;
+    sm.val[0][i] = stage_val[base + slot.base + i];
+  }
+  __syncthreads();
+  atomicMin(&sm.kmin, kmin);
+  atomicMax(&sm.kmax, kmax);
+  __syncthreads();
+  const uint32_t k0 = sm.kmin;
+  const uint32_t span = sm.kmax - k0;
+  const uint32_t lt_mask = (1u << lane) - 1u;
+  int cur = 0;
+  if (span == 0) goto write_out;  // one key: the index order is the order
+
+  // Fine counting sort: kFine bins linear in the score between the bucket's
+  // extremes (monotone, ties share a bin), a stable-free scatter, then each
+  // bin sorted by (key, index) -- a total order, so the result is unique.
+  {
+    const float xhi = key_score(k0), xlo = key_score(sm.kmax);
+    uint32_t* fcnt = &sm.cnt[0][0];  // kFine counters, then cursors
+    const float fscale = (float)kFine / (xhi - xlo);
+    for (int k = tid; k < kFine; k += kBucketThreads) fcnt[k] = 0;
+    if (tid == 0) sm.big = 0;
+    __syncthreads();
+    for (int i = tid; i < m; i += kBucketThreads)
+      atomicAdd(&fcnt[fine_bin(key_score(sm.key[0][i]), xhi, fscale)], 1u);
+    __syncthreads();
+    uint32_t c[kFine / kBucketThreads];
+    int mine = 0, big = 0;
+#pragma unroll
+    for (int e = 0; e < kFine / kBucketThreads; ++e) {
+      c[e] = fcnt[tid * (kFine / kBucketThreads) + e];
+      mine += (int)c[e];
+      big |= c[e] > kFineMax;
+    }
+    if (big) atomicOr(&sm.big, 1);
+    int total;
+    int run = block_excl_scan(mine, sm.wtot, total);
+    if (!sm.big) {
+      // counters become cursors (start ranks) and the bins are scattered
+#pragma unroll
+      for (int e = 0; e < kFine / kBucketThreads; ++e) {
+        fcnt[tid * (kFine / kBucketThreads) + e] = (uint32_t)run;
+        run += (int)c[e];
+      }
+      __syncthreads();
+      for (int i = tid; i < m; i += kBucketThreads) {
+        const uint32_t key = sm.key[0][i];
+        const uint32_t pos = atomicAdd(&fcnt[fine_bin(key_score(key), xhi, fscale)], 1u);
+        sm.key[1][pos] = key;
+        sm.val[1][pos] = sm.val[0][i];
+      }
+      __syncthreads();
+      // insertion sort of every fine bin (typically 1-3 elements)
+#pragma unroll
+      for (int e = 0; e < kFine / kBucketThreads; ++e) {
+        const int end = (int)fcnt[tid * (kFine / kBucketThreads) + e];
+        const int beg = end - (int)c[e];
+        for (int a2 = beg + 1; a2 < end; ++a2) {
+          const uint32_t kk = sm.key[1][a2], vv = sm.val[1][a2];
+          int b2 = a2 - 1;
+          while (b2 >= beg && (sm.key[1][b2] > kk || (sm.key[1][b2] == kk && sm.val[1][b2] > vv))) {
+            sm.key[1][b2 + 1] = sm.key[1][b2];
+            sm.val[1][b2 + 1] = sm.val[1][b2];
+            --b2;
+          }
+          sm.key[1][b2 + 1] = kk;
+          sm.val[1][b2 + 1] = vv;
+        }
+      }
+      __syncthreads();
+      cur = 1;
+      goto write_out;
+    }
+    __syncthreads();
+  }
+
+  // a heavy fine bin: stable LSD radix sort over the bucket-relative key
+  {
+  const int nbits = 32 - __clz(span);
+  const int passes = (nbits + 7) / 8;
+  for (int pass = 0; pass < passes; ++pass) {
+    const int shift = 8 * pass;
+    // digit totals
+    for (int k = tid; k < kSortWarps * 256; k += kBucketThreads) (&sm.cnt[0][0])[k] = 0;
+    __syncthreads();
+    for (int i = tid; i < m; i += kBucketThreads) atomicAdd(&sm.cnt[warp][((sm.key[cur][i] - k0) >> shift) & 255u], 1u);
+    __syncthreads();
+    if (tid < 256) {
+      uint32_t t = 0;
+      for (int w = 0; w < kSortWarps; ++w) t += sm.cnt[w][tid];
+      sm.dbase[tid] = t;
+    }
+    __syncthreads();
+    if (warp == 0) {
+      uint32_t v[8], run = 0;
+#pragma unroll
+      for (int k = 0; k < 8; ++k) { v[k] = run; run += sm.dbase[lane * 8 + k]; }
+      uint32_t incl = run;
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        const uint32_t y = __shfl_up_sync(0xffffffffu, incl, o);
+        if (lane >= o) incl += y;
+      }
+      const uint32_t excl = incl - run;
+      __syncwarp();
+#pragma unroll
+      for (int k = 0; k < 8; ++k) sm.dbase[lane * 8 + k] = excl + v[k];
+    }
+    __syncthreads();
+    // stable scatter, one element per thread per step
+    const int out = cur ^ 1;
+    for (int t0 = 0; t0 < m; t0 += kBucketThreads) {
+      const int i = t0 + tid;
+      const bool valid = i < m;
+      const uint32_t key = valid ? sm.key[cur][i] : 0u;
+      const uint32_t val = valid ? sm.val[cur][i] : 0u;
+      const uint32_t dg = ((key - k0) >> shift) & 255u;
+#pragma unroll
+      for (int k = 0; k < 8; ++k) sm.cnt[warp][lane * 8 + k] = 0;
+      __syncwarp();
+      const uint32_t peers = __match_any_sync(0xffffffffu, valid ? dg : 256u + lane);
+      const uint32_t rank = __popc(peers & lt_mask);
+      if (valid && (__ffs(peers) - 1) == lane) sm.cnt[warp][dg] = __popc(peers);
+      __syncthreads();
+      if (tid < 256) {
+        uint32_t run = sm.dbase[tid];
+        for (int w = 0; w < kSortWarps; ++w) {
+          const uint32_t c = sm.cnt[w][tid];
+          sm.cnt[w][tid] = run;
+          run += c;
+        }
+        sm.dbase[tid] = run;
+      }
+      __syncthreads();
+      if (valid) {
+        const uint32_t pos = sm.cnt[warp][dg] + rank;
+        sm.key[out][pos] = key;
+        sm.val[out][pos] = val;
+      }
+      __syncthreads();
+    }
+    cur = out;
+  }
+  }
+write_out:
+  for (int i = tid; i < m; i += kBucketThreads) {
+    sorted[base + slot.base + i] = key_score(sm.key[cur][i]);
+    perm[base + slot.base + i] = kSink + (int32_t)sm.val[cur][i];
+  }
+}
+
+// ---------------------------------------------------------------------------
+// block masses of the sorted scores and the stop point: one CTA per segment
+// ---------------------------------------------------------------------------
+__global__ void __launch_bounds__(256) k_mass_stop(const float* __restrict__ sorted, const float* __restrict__ segM,
+                                                  const double* __restrict__ segZ, int32_t* __restrict__ nblocks,
+                                                  int BHkv, int S, int64_t T, double tau) {
+  __shared__ int cmin;
+  const int q = blockIdx.x;
+  const int s = S - 1 - q / BHkv;
+  const int bk = q % BHkv;
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const int n = (int)num_cand(s);
+  const int nb = n / kBk;
+  if (threadIdx.x == 0) cmin = nb;
+  __syncthreads();
+  const float* ss = sorted + (size_t)bk * T + cand_offset(s);
+  const float M = segM[(size_t)bk * S + s];
+  const double Z = segZ[(size_t)bk * S + s];
+  for (int blk = warp; blk < nb; blk += 8) {
+    float e = exp_shifted(ss[blk * kBk + lane], M) + exp_shifted(ss[blk * kBk + 32 + lane], M);
+#pragma unroll
+    for (int o = 16; o >= 1; o >>= 1) e += __shfl_xor_sync(0xffffffffu, e, o);
+    if (lane == 0 && (double)e / Z < tau) atomicMin(&cmin, blk);
+  }
+  __syncthreads();
+  if (threadIdx.x == 0) nblocks[(size_t)bk * S + s] = cmin;
+}
+
+}  // namespace s2o

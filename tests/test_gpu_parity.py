@@ -28,7 +28,7 @@ def run_path(Q, K, V, tau, out_dtype=s2o.OUT_BF16):
     cfg = s2o.make_config(B, Hq, K.shape[1], N, tau=tau)
     q, k, v = dev(Q), dev(K), dev(V)
     bufs = s2o.plan(cfg, q, k)
-    assert s2o.last_launch_count() == 4
+    assert s2o.last_launch_count() >= 6
     out = s2o.attention(cfg, q, k, v, bufs["perm"], bufs["nblocks"], out_dtype=out_dtype)
     assert s2o.last_launch_count() == 1
     assert s2o.last_device_error() == 0

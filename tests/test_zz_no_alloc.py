@@ -49,11 +49,12 @@ def test_noalloc_plan_matches_workspace_plan_on_consecutive_calls(shape):
         Q, K, _ = synth.generate(B, Hq, Hkv, N, 128, planted=True, band=True, n_stripe=8, seed=seed)
         q, k = _dev(Q), _dev(K)
         ref = s2o.plan(cfg, q, k)
+        ref_launches = s2o.last_launch_count()
         assert s2o.last_device_error() == 0
         got = s2o.alloc_plan(cfg, q.device, workspace=False)
         before = torch.cuda.memory_allocated()
         s2o.plan_noalloc(cfg, q, k, got)
-        assert s2o.last_launch_count() == 4
+        assert s2o.last_launch_count() == ref_launches
         assert s2o.last_device_error() == 0
         assert torch.cuda.memory_allocated() == before
         T = cfg.B * cfg.Hkv * s2o.num_candidates(cfg)
