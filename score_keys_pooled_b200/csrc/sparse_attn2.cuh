@@ -12,10 +12,13 @@
 //     odd last block leaves an empty, zero-filled and masked half);
 //   * warp roles (384 threads): warps 0-3 and 4-7 run the online softmax of
 //     head 0 and head 1 (thread = row = TMEM lane), warp 8 issues tcgen05.mma
-//     from one thread, warp 9 gathers K/V rows with TMA (tile::gather4: four
-//     256-byte rows per pair of instructions, one per 64-column half, written
-//     128B-swizzled by the TMA unit) into a 2-stage ring whose mbarriers count
-//     the landed bytes; Q arrives as 2D TMA tiles;
+//     from one thread, warps 9 and 10 gather K and V rows with TMA
+//     (tile::gather4: four 256-byte rows per pair of instructions, one per
+//     64-column half, written 128B-swizzled by the TMA unit) into a 3-stage K
+//     ring and a 2-stage V ring whose mbarriers count the landed bytes (K is
+//     released as soon as both heads' S are computed, so its loads run up to
+//     three tiles ahead); the row indices of the next tile are fetched while
+//     a stage drains; Q arrives as 2D TMA tiles;
 //   * tensor memory (512 columns): S_i = Q_i K^T in columns [128 i, 128 i+128),
 //     O_i in [256 + 128 i, ...); P_i (bf16, two per column) overwrites the
 //     first 64 columns of S_i and is the A operand of O_i += P_i V straight
@@ -41,23 +44,27 @@ constexpr int kKT2 = 128;                 // keys per tile
 constexpr int kAttn2Threads = 384;
 constexpr int kMmaWarp = 8;
 constexpr int kLoadWarp0 = 9;
-constexpr int kStages2 = 2;
+constexpr int kStagesK = 3;                          // K ring (freed once Q K^T of both heads is done)
+constexpr int kStagesV = 2;                          // V ring (freed once P V of both heads is done)
 constexpr uint32_t kTile2Bytes = 2 * 128 * 128;      // one 128-row operand tile: 2 atoms x 128 rows x 128 B
 constexpr uint32_t kOff2Q = 0;                       // Q0, Q1
-constexpr uint32_t kOff2KV = 2 * kTile2Bytes;        // stage st: K at +2*st*tile, V at +(2*st+1)*tile
-constexpr uint32_t kOff2Bar = kOff2KV + 2 * kStages2 * kTile2Bytes;
+constexpr uint32_t kOff2K = 2 * kTile2Bytes;         // K stages
+constexpr uint32_t kOff2V = kOff2K + kStagesK * kTile2Bytes;
+constexpr uint32_t kOff2Bar = kOff2V + kStagesV * kTile2Bytes;
 constexpr uint32_t kAttn2SmemData = kOff2Bar + 256;
 constexpr size_t kAttn2Smem = kAttn2SmemData + 1024;  // + alignment slack
 constexpr uint32_t kTmem2Cols = 512;
 
 // barrier slots (8 bytes each) from kOff2Bar
-constexpr int kBarKvFull = 0;   // [2]  loader -> MMA (TMA bytes)
-constexpr int kBarKvEmpty = 2;  // [2]  MMA commit -> loader
-constexpr int kBarQFull = 4;    //      loader -> MMA (TMA bytes)
-constexpr int kBarSFull = 5;    // [2]  MMA commit -> softmax i
-constexpr int kBarPFull = 7;    // [2]  softmax i (count 128) -> MMA
-constexpr int kBarODone = 9;    // [2]  MMA commit -> softmax i
-constexpr int kSlotTmem = 11;
+constexpr int kBarKFull = 0;    // [3]  K loader -> MMA (TMA bytes)
+constexpr int kBarKEmpty = 3;   // [3]  MMA commit -> K loader
+constexpr int kBarVFull = 6;    // [2]  V loader -> MMA (TMA bytes)
+constexpr int kBarVEmpty = 8;   // [2]  MMA commit -> V loader
+constexpr int kBarQFull = 10;   //      K loader -> MMA (TMA bytes)
+constexpr int kBarSFull = 11;   // [2]  MMA commit -> softmax i
+constexpr int kBarPFull = 13;   // [2]  softmax i (count 128) -> MMA
+constexpr int kBarODone = 15;   // [2]  MMA commit -> softmax i
+constexpr int kSlotTmem = 17;
 
 __device__ __forceinline__ void tc_mma_ts(uint32_t d_tmem, uint32_t a_tmem, uint64_t bdesc, uint32_t idesc,
                                           uint32_t accumulate) {
@@ -156,11 +163,15 @@ __global__ void __launch_bounds__(kAttn2Threads, 1)
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int G = a.Hq / a.Hkv;
   const int pairs = G / 2;
+  // work order: KV head by KV head (the CTAs running together then share one
+  // head's K/V, which stays in L2), segments longest first, the pairs of a
+  // segment adjacent (they gather the same rows)
   const int w = blockIdx.x;
-  const int per_s = a.B * a.Hkv * pairs;
-  const int s = a.S - 1 - w / per_s;
-  const int rest = w % per_s;
-  const int bk = rest / pairs, pair = rest % pairs;
+  const int per_bk = a.S * pairs;
+  const int bk = w / per_bk;
+  const int rest = w % per_bk;
+  const int s = a.S - 1 - rest / pairs;
+  const int pair = rest % pairs;
   const int b = bk / a.Hkv, kvh = bk % a.Hkv;
   const int h0 = kvh * G + 2 * pair;
 
@@ -178,6 +189,7 @@ __global__ void __launch_bounds__(kAttn2Threads, 1)
     for (int k = 0; k < kSlotTmem; ++k) {
       uint32_t count = 1;
       if (k == kBarPFull || k == kBarPFull + 1) count = 128;
+      if (k == kSlotTmem) break;
       mbar_init(bar(k), count);
     }
     fence_mbar_init();
@@ -190,17 +202,24 @@ __global__ void __launch_bounds__(kAttn2Threads, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
-  if (warp > kLoadWarp0) {
-    // warps 10-11: no role (they complete the register-donating warpgroup)
+  if (warp > kLoadWarp0 + 1) {
+    // warp 11: no role (it completes the register-donating warpgroup)
     regs_decrease<kRegsOther>();
-  } else if (warp == kLoadWarp0) {
-    // ------------------------------------------------------------------ loader (TMA)
+  } else if (warp >= kLoadWarp0) {
+    // ------------------------------------------------------------------ loaders (TMA)
+    // warp 9 loads Q and the K ring, warp 10 the V ring
     regs_decrease<kRegsOther>();
+    const bool is_k = warp == kLoadWarp0;
+    const int nst = is_k ? kStagesK : kStagesV;
+    const int bar_full = is_k ? kBarKFull : kBarVFull;
+    const int bar_empty = is_k ? kBarKEmpty : kBarVEmpty;
+    const uint32_t ring = sbase + (is_k ? kOff2K : kOff2V);
+    const CUtensorMap* map = is_k ? &tmK : &tmV;
     // rows of K/V as [B*Hkv*N, 128]; a row coordinate past the end is out of
     // bounds and reads as zeros (empty halves, keys past N)
     const int zero_row = a.B * a.Hkv * a.N;
     const int kv_row0 = bk * a.N;
-    if (lane == 0) {
+    if (is_k && lane == 0) {
       mbar_expect_tx(bar(kBarQFull), 2 * kTile2Bytes);
 #pragma unroll
       for (int qi = 0; qi < 2; ++qi)
@@ -211,14 +230,10 @@ __global__ void __launch_bounds__(kAttn2Threads, 1)
     }
     const int32_t* pseg = a.perm + (size_t)bk * a.T + cand_offset(s);
     const int cand_hi = kLq * s - kWin;
-    for (int t = 0; t < ntiles; ++t) {
-      const int st = t & 1;
-      // rows 4 lane .. 4 lane + 3 of the tile: their key indices first (these
-      // loads overlap the wait for the stage to drain)
-      const int blk = 2 * t + (lane >> 4);
+    // key rows of tile t handled by this lane: rows 4 lane .. 4 lane + 3
+    auto tile_rows = [&](int t, int* y) {
       int j0;
-      const int kind = walk2_block(wk, s, blk, j0);
-      int y[4];
+      const int kind = walk2_block(wk, s, 2 * t + (lane >> 4), j0);
 #pragma unroll
       for (int k = 0; k < 4; ++k) {
         const int rr = (4 * lane + k) & 63;
@@ -235,19 +250,23 @@ __global__ void __launch_bounds__(kAttn2Threads, 1)
         }
         y[k] = j >= 0 ? kv_row0 + j : zero_row;
       }
-      if (!warp_wait(bar(kBarKvEmpty + st), (uint32_t)(((t >> 1) & 1) ^ 1))) {
+    };
+    int y[4];
+    if (ntiles > 0) tile_rows(0, y);
+    for (int t = 0; t < ntiles; ++t) {
+      const int st = t % nst;
+      const int round = t / nst;
+      if (!warp_wait(bar(bar_empty + st), (uint32_t)((round & 1) ^ 1))) {
         if (lane == 0) set_error(kErrTimeout);
         break;
       }
-      if (lane == 0) mbar_expect_tx(bar(kBarKvFull + st), 2 * kTile2Bytes);
+      if (lane == 0) mbar_expect_tx(bar(bar_full + st), kTile2Bytes);
       __syncwarp();
-      const uint32_t sK = sbase + kOff2KV + (2 * st) * kTile2Bytes;
+      const uint32_t dst = ring + st * kTile2Bytes + lane * (4 * 128);
 #pragma unroll
-      for (int m = 0; m < 2; ++m)
-#pragma unroll
-        for (int half = 0; half < 2; ++half)
-          tma_gather4(sK + m * kTile2Bytes + half * (128 * 128) + lane * (4 * 128), m ? &tmV : &tmK, 64 * half,
-                      y[0], y[1], y[2], y[3], bar(kBarKvFull + st));
+      for (int half = 0; half < 2; ++half)
+        tma_gather4(dst + half * (128 * 128), map, 64 * half, y[0], y[1], y[2], y[3], bar(bar_full + st));
+      if (t + 1 < ntiles) tile_rows(t + 1, y);  // loads overlap the next stage's drain
     }
   } else if (warp == kMmaWarp) {
     // ------------------------------------------------------------------ MMA issuer
@@ -260,24 +279,29 @@ __global__ void __launch_bounds__(kAttn2Threads, 1)
         for (int i = 0; ok && i < 2; ++i) {
           if (t > 0) {
             const int tp = t - 1;
+            if (i == 0) {
+              ok = mbar_wait_bounded(bar(kBarVFull + tp % kStagesV), (uint32_t)((tp / kStagesV) & 1));
+              if (!ok) break;
+            }
             ok = mbar_wait_bounded(bar(kBarPFull + i), (uint32_t)(tp & 1));
             if (!ok) break;
             tc_fence_after();
-            const uint32_t sV = sbase + kOff2KV + (2 * (tp & 1) + 1) * kTile2Bytes;
+            const uint32_t sV = sbase + kOff2V + (tp % kStagesV) * kTile2Bytes;
 #pragma unroll
             for (int kk = 0; kk < kKT2 / 16; ++kk) {
               const uint64_t bd = sdesc_sw128(sV + kk * (16 * 128), 128 * 128, 1024);
               tc_mma_ts(tmem + 256 + 128 * i, tmem + 128 * i + 8 * kk, bd, idesc_pv, (tp > 0 || kk > 0) ? 1u : 0u);
             }
             tc_commit(bar(kBarODone + i));
+            if (i == 1) tc_commit(bar(kBarVEmpty + tp % kStagesV));
           }
           if (t < ntiles) {
             if (i == 0) {
-              ok = mbar_wait_bounded(bar(kBarKvFull + (t & 1)), (uint32_t)((t >> 1) & 1));
+              ok = mbar_wait_bounded(bar(kBarKFull + t % kStagesK), (uint32_t)((t / kStagesK) & 1));
               if (!ok) break;
             }
             const uint32_t sQ = sbase + kOff2Q + i * kTile2Bytes;
-            const uint32_t sK = sbase + kOff2KV + (2 * (t & 1)) * kTile2Bytes;
+            const uint32_t sK = sbase + kOff2K + (t % kStagesK) * kTile2Bytes;
 #pragma unroll
             for (int kk = 0; kk < 8; ++kk) {
               const uint64_t ad = sdesc_sw128(sQ + (kk >> 2) * (128 * 128) + (kk & 3) * 32, 16, 1024);
@@ -285,9 +309,9 @@ __global__ void __launch_bounds__(kAttn2Threads, 1)
               tc_mma_ss(tmem + 128 * i, ad, bd, idesc_qk, kk > 0 ? 1u : 0u);
             }
             tc_commit(bar(kBarSFull + i));
+            if (i == 1) tc_commit(bar(kBarKEmpty + t % kStagesK));
           }
         }
-        if (ok && t > 0) tc_commit(bar(kBarKvEmpty + ((t - 1) & 1)));
       }
       if (!ok) set_error(kErrTimeout);
     }
