@@ -86,6 +86,29 @@ __device__ __forceinline__ void regs_decrease() {
 constexpr uint32_t kRegsSoftmax = 208, kRegsOther = 80;
 static_assert(2 * kRegsSoftmax + kRegsOther <= 3 * 168, "register split exceeds the launch's budget");
 
+// packed pairs of fp32 (sm_100 f32x2 arithmetic): one instruction, two lanes
+__device__ __forceinline__ uint64_t f2_pack(float lo, float hi) {
+  return ((uint64_t)__float_as_uint(hi) << 32) | (uint64_t)__float_as_uint(lo);
+}
+__device__ __forceinline__ uint64_t f2_fma(uint64_t a, uint64_t b, uint64_t c) {
+  uint64_t d;
+  asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(d) : "l"(a), "l"(b), "l"(c));
+  return d;
+}
+__device__ __forceinline__ uint64_t f2_add(uint64_t a, uint64_t b) {
+  uint64_t d;
+  asm("add.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+  return d;
+}
+// three-input max (sm_100)
+__device__ __forceinline__ float fmax3(float a, float b, float c) {
+  float d;
+  asm("max.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
+  return d;
+}
+__device__ __forceinline__ float f2_lo(uint64_t v) { return __uint_as_float((uint32_t)v); }
+__device__ __forceinline__ float f2_hi(uint64_t v) { return __uint_as_float((uint32_t)(v >> 32)); }
+
 __device__ __forceinline__ void mbar_arrive(uint32_t bar) {
   asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];\n" ::"r"(bar) : "memory");
 }
@@ -344,10 +367,18 @@ __global__ void __launch_bounds__(kAttn2Threads, 1)
 #pragma unroll
       for (int cc = 0; cc < kKT2; cc += 32) tmem_ld32(tS + cc, x + cc);
       tc_wait_ld();
+      const bool full_tile = lim_a >= kBk && lim_b >= kBk;  // no key masked
       float mt = -INFINITY;
+      if (full_tile) {
+        float m4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
 #pragma unroll
-      for (int c = 0; c < kKT2; ++c)
-        if ((c & 63) <= (c < 64 ? lim_a : lim_b)) mt = fmaxf(mt, x[c]);
+        for (int c = 0; c < kKT2; c += 2) m4[(c >> 1) & 3] = fmax3(m4[(c >> 1) & 3], x[c], x[c + 1]);
+        mt = fmaxf(fmax3(m4[0], m4[1], m4[2]), m4[3]);
+      } else {
+#pragma unroll
+        for (int c = 0; c < kKT2; ++c)
+          if ((c & 63) <= (c < 64 ? lim_a : lim_b)) mt = fmaxf(mt, x[c]);
+      }
       mt *= sl2;
       const bool move = mt > m_run + 8.f;
       float alpha = 1.f;
@@ -357,14 +388,28 @@ __global__ void __launch_bounds__(kAttn2Threads, 1)
         ell *= alpha;
       }
       // P = exp2(S - m) as bf16 pairs, packed in place into x[0 .. 63]
-      float rs = 0.f;
+      float rs;
+      if (full_tile) {
+        const uint64_t s2 = f2_pack(sl2, sl2), nm2 = f2_pack(-m_run, -m_run);
+        uint64_t rs2 = 0;
 #pragma unroll
-      for (int c = 0; c < kKT2; c += 2) {
-        const int lim = c < 64 ? lim_a : lim_b;
-        const float p0 = ((c & 63) <= lim) ? ex2_approx(fmaf(x[c], sl2, -m_run)) : 0.f;
-        const float p1 = (((c + 1) & 63) <= lim) ? ex2_approx(fmaf(x[c + 1], sl2, -m_run)) : 0.f;
-        rs += p0 + p1;
-        x[c / 2] = __uint_as_float(pack_bf16x2(p0, p1));
+        for (int c = 0; c < kKT2; c += 2) {
+          const uint64_t v = f2_fma(f2_pack(x[c], x[c + 1]), s2, nm2);
+          const float p0 = ex2_approx(f2_lo(v)), p1 = ex2_approx(f2_hi(v));
+          rs2 = f2_add(rs2, f2_pack(p0, p1));
+          x[c / 2] = __uint_as_float(pack_bf16x2(p0, p1));
+        }
+        rs = f2_lo(rs2) + f2_hi(rs2);
+      } else {
+        rs = 0.f;
+#pragma unroll
+        for (int c = 0; c < kKT2; c += 2) {
+          const int lim = c < 64 ? lim_a : lim_b;
+          const float p0 = ((c & 63) <= lim) ? ex2_approx(fmaf(x[c], sl2, -m_run)) : 0.f;
+          const float p1 = (((c + 1) & 63) <= lim) ? ex2_approx(fmaf(x[c + 1], sl2, -m_run)) : 0.f;
+          rs += p0 + p1;
+          x[c / 2] = __uint_as_float(pack_bf16x2(p0, p1));
+        }
       }
       ell += rs;
       // the previous P V must be done before P_i and O_i are rewritten (it was
