@@ -143,7 +143,7 @@ __global__ void __launch_bounds__(256, 2) k_score(const uint16_t* __restrict__ K
 
   float* sc_bk = scores + (size_t)bk * T;
   float2* part_bk = part + (size_t)bk * S * S;
-  const double sqrt_d = 11.313708498984761;  // sqrt(128)
+  const double inv_sqrt_d = 0.08838834764831845;  // 1/sqrt(128), rounded to fp64
 #pragma unroll
   for (int q = 0; q < 4; ++q) {
     const int s = s_lo + ts + 16 * q;
@@ -154,7 +154,7 @@ __global__ void __launch_bounds__(256, 2) k_score(const uint16_t* __restrict__ K
 #pragma unroll
     for (int a = 0; a < 8; ++a) {
       const int j = t * kScoreKeys + tk + 16 * a;
-      v[a] = (float)(acc[a][q] / sqrt_d);
+      v[a] = (float)(acc[a][q] * inv_sqrt_d);
       const bool adm = seg_ok && (j < N);
       if (adm) {
         if (!isfinite(v[a])) set_error(kErrNonFinite);

@@ -206,7 +206,7 @@ s2o_status s2o_plan(const s2o_config* cfg, const uint16_t* Q, const uint16_t* K,
                                                    BH, S, T);
   ++t_launches;
   if (w.nslots > 0) {
-    k_bucket_sort<<<(unsigned)w.nslots, kBucketThreads, kBucketSmem, s>>>(w.keyB, w.valB, w.slots, w.sorted, perm,
+    k_bucket_sort<<<(unsigned)w.nslots, kSorterThreads, kBucketSmem, s>>>(w.keyB, w.valB, w.slots, w.sorted, perm,
                                                                           T);
     ++t_launches;
   }

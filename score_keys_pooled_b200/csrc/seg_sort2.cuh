@@ -30,10 +30,12 @@
 namespace s2o {
 
 constexpr int kNumBins = 2048;
-constexpr int kBucketCap = 11264;             // elements a bucket CTA sorts in shared memory
+constexpr int kBucketCap = 5632;              // elements a bucket CTA sorts in shared memory
 constexpr int kBucketHalf = kBucketCap / 2;   // rank window of a bucket
-constexpr int kBucketThreads = 1024;
-constexpr int kMaxBuckets = 128;              // bucket ids per segment (N <= 2^19)
+constexpr int kBucketThreads = 1024;          // planner CTA
+constexpr int kSorterThreads = 512;           // bucket-sorter CTA (two per SM)
+constexpr int kSorterWarps = kSorterThreads / 32;
+constexpr int kMaxBuckets = 256;              // bucket ids per segment (N <= 2^19)
 
 enum SegMode : int { kModeDone = 0, kModeBuckets = 1, kModeFallback = 2 };
 
@@ -51,7 +53,8 @@ __device__ __forceinline__ int score_bin(float x, float hi, float scale) {
   return min(max(b, 0), kNumBins - 1);
 }
 
-// block-wide exclusive scan of one value per thread (1024 threads)
+// block-wide exclusive scan of one value per thread (NWARPS full warps)
+template <int NWARPS = 32>
 __device__ __forceinline__ int block_excl_scan(int v, int* warp_tot, int& total) {
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   int incl = v;
@@ -63,14 +66,14 @@ __device__ __forceinline__ int block_excl_scan(int v, int* warp_tot, int& total)
   if (lane == 31) warp_tot[warp] = incl;
   __syncthreads();
   if (warp == 0) {
-    int w = warp_tot[lane];
+    int w = lane < NWARPS ? warp_tot[lane] : 0;
     int wi = w;
 #pragma unroll
     for (int o = 1; o < 32; o <<= 1) {
       const int y = __shfl_up_sync(0xffffffffu, wi, o);
       if (lane >= o) wi += y;
     }
-    warp_tot[lane] = wi - w;  // exclusive prefix of the warp totals
+    if (lane < NWARPS) warp_tot[lane] = wi - w;  // exclusive prefix of the warp totals
     if (lane == 31) warp_tot[32] = wi;
   }
   __syncthreads();
@@ -94,7 +97,7 @@ __global__ void __launch_bounds__(kBucketThreads) k_bucket_plan(const float* __r
   __shared__ int wtot[33];
   __shared__ float red[64];
   __shared__ int flag;
-  __shared__ uint8_t bin2bkt[kNumBins];
+  __shared__ uint8_t bin2bkt[kNumBins];  // bucket id of each bin (< kMaxBuckets = 256)
   __shared__ uint16_t wcnt[kSortWarps][kMaxBuckets];
   __shared__ int cursor[kMaxBuckets];
   const int q = blockIdx.x;
@@ -254,7 +257,7 @@ __global__ void __launch_bounds__(kBucketThreads) k_bucket_plan(const float* __r
 // ---------------------------------------------------------------------------
 // bucket sorter: one 1024-thread CTA per slot
 // ---------------------------------------------------------------------------
-constexpr int kFine = 4096;     // fine bins of a bucket
+constexpr int kFine = 4096;     // fine bins of a bucket (= kSorterWarps * 256 counters)
 constexpr int kFineMax = 64;    // larger fine bins send the bucket to the radix path
 
 __device__ __forceinline__ int fine_bin(float x, float hi, float scale) {
@@ -265,7 +268,7 @@ __device__ __forceinline__ int fine_bin(float x, float hi, float scale) {
 struct BucketSmem {
   uint32_t key[2][kBucketCap];
   uint32_t val[2][kBucketCap];
-  uint32_t cnt[kSortWarps][256];  // radix digit counts, or the kFine fine-bin counters
+  uint32_t cnt[kSorterWarps][256];  // radix digit counts, or the kFine fine-bin counters
   uint32_t dbase[256];
   int wtot[33];
   uint32_t kmin, kmax;
@@ -273,7 +276,7 @@ struct BucketSmem {
 };
 constexpr size_t kBucketSmem = sizeof(BucketSmem);
 
-__global__ void __launch_bounds__(kBucketThreads, 1) k_bucket_sort(const uint32_t* __restrict__ stage_key,
+__global__ void __launch_bounds__(kSorterThreads, 2) k_bucket_sort(const uint32_t* __restrict__ stage_key,
                                                                   const uint32_t* __restrict__ stage_val,
                                                                   const BucketSlot* __restrict__ slots,
                                                                   float* __restrict__ sorted,
@@ -289,7 +292,7 @@ __global__ void __launch_bounds__(kBucketThreads, 1) k_bucket_sort(const uint32_
   // the bucket's pairs, already in index order at its rank range
   const int m = slot.count;
   uint32_t kmin = 0xFFFFFFFFu, kmax = 0u;
-  for (int i = tid; i < m; i += kBucketThreads) {
+  for (int i = tid; i < m; i += kSorterThreads) {
     const uint32_t key = stage_key[base + slot.base + i];
     kmin = min(kmin, key);
     kmax = max(kmax, key);
@@ -313,32 +316,32 @@ __global__ void __launch_bounds__(kBucketThreads, 1) k_bucket_sort(const uint32_
     const float xhi = key_score(k0), xlo = key_score(sm.kmax);
     uint32_t* fcnt = &sm.cnt[0][0];  // kFine counters, then cursors
     const float fscale = (float)kFine / (xhi - xlo);
-    for (int k = tid; k < kFine; k += kBucketThreads) fcnt[k] = 0;
+    for (int k = tid; k < kFine; k += kSorterThreads) fcnt[k] = 0;
     if (tid == 0) sm.big = 0;
     __syncthreads();
-    for (int i = tid; i < m; i += kBucketThreads)
+    for (int i = tid; i < m; i += kSorterThreads)
       atomicAdd(&fcnt[fine_bin(key_score(sm.key[0][i]), xhi, fscale)], 1u);
     __syncthreads();
-    uint32_t c[kFine / kBucketThreads];
+    uint32_t c[kFine / kSorterThreads];
     int mine = 0, big = 0;
 #pragma unroll
-    for (int e = 0; e < kFine / kBucketThreads; ++e) {
-      c[e] = fcnt[tid * (kFine / kBucketThreads) + e];
+    for (int e = 0; e < kFine / kSorterThreads; ++e) {
+      c[e] = fcnt[tid * (kFine / kSorterThreads) + e];
       mine += (int)c[e];
       big |= c[e] > kFineMax;
     }
     if (big) atomicOr(&sm.big, 1);
     int total;
-    int run = block_excl_scan(mine, sm.wtot, total);
+    int run = block_excl_scan<kSorterWarps>(mine, sm.wtot, total);
     if (!sm.big) {
       // counters become cursors (start ranks) and the bins are scattered
 #pragma unroll
-      for (int e = 0; e < kFine / kBucketThreads; ++e) {
-        fcnt[tid * (kFine / kBucketThreads) + e] = (uint32_t)run;
+      for (int e = 0; e < kFine / kSorterThreads; ++e) {
+        fcnt[tid * (kFine / kSorterThreads) + e] = (uint32_t)run;
         run += (int)c[e];
       }
       __syncthreads();
-      for (int i = tid; i < m; i += kBucketThreads) {
+      for (int i = tid; i < m; i += kSorterThreads) {
         const uint32_t key = sm.key[0][i];
         const uint32_t pos = atomicAdd(&fcnt[fine_bin(key_score(key), xhi, fscale)], 1u);
         sm.key[1][pos] = key;
@@ -347,8 +350,8 @@ __global__ void __launch_bounds__(kBucketThreads, 1) k_bucket_sort(const uint32_
       __syncthreads();
       // insertion sort of every fine bin (typically 1-3 elements)
 #pragma unroll
-      for (int e = 0; e < kFine / kBucketThreads; ++e) {
-        const int end = (int)fcnt[tid * (kFine / kBucketThreads) + e];
+      for (int e = 0; e < kFine / kSorterThreads; ++e) {
+        const int end = (int)fcnt[tid * (kFine / kSorterThreads) + e];
         const int beg = end - (int)c[e];
         for (int a2 = beg + 1; a2 < end; ++a2) {
           const uint32_t kk = sm.key[1][a2], vv = sm.val[1][a2];
@@ -376,13 +379,13 @@ __global__ void __launch_bounds__(kBucketThreads, 1) k_bucket_sort(const uint32_
   for (int pass = 0; pass < passes; ++pass) {
     const int shift = 8 * pass;
     // digit totals
-    for (int k = tid; k < kSortWarps * 256; k += kBucketThreads) (&sm.cnt[0][0])[k] = 0;
+    for (int k = tid; k < kSorterWarps * 256; k += kSorterThreads) (&sm.cnt[0][0])[k] = 0;
     __syncthreads();
-    for (int i = tid; i < m; i += kBucketThreads) atomicAdd(&sm.cnt[warp][((sm.key[cur][i] - k0) >> shift) & 255u], 1u);
+    for (int i = tid; i < m; i += kSorterThreads) atomicAdd(&sm.cnt[warp][((sm.key[cur][i] - k0) >> shift) & 255u], 1u);
     __syncthreads();
     if (tid < 256) {
       uint32_t t = 0;
-      for (int w = 0; w < kSortWarps; ++w) t += sm.cnt[w][tid];
+      for (int w = 0; w < kSorterWarps; ++w) t += sm.cnt[w][tid];
       sm.dbase[tid] = t;
     }
     __syncthreads();
@@ -404,7 +407,7 @@ __global__ void __launch_bounds__(kBucketThreads, 1) k_bucket_sort(const uint32_
     __syncthreads();
     // stable scatter, one element per thread per step
     const int out = cur ^ 1;
-    for (int t0 = 0; t0 < m; t0 += kBucketThreads) {
+    for (int t0 = 0; t0 < m; t0 += kSorterThreads) {
       const int i = t0 + tid;
       const bool valid = i < m;
       const uint32_t key = valid ? sm.key[cur][i] : 0u;
@@ -419,7 +422,7 @@ __global__ void __launch_bounds__(kBucketThreads, 1) k_bucket_sort(const uint32_
       __syncthreads();
       if (tid < 256) {
         uint32_t run = sm.dbase[tid];
-        for (int w = 0; w < kSortWarps; ++w) {
+        for (int w = 0; w < kSorterWarps; ++w) {
           const uint32_t c = sm.cnt[w][tid];
           sm.cnt[w][tid] = run;
           run += c;
@@ -438,7 +441,7 @@ __global__ void __launch_bounds__(kBucketThreads, 1) k_bucket_sort(const uint32_
   }
   }
 write_out:
-  for (int i = tid; i < m; i += kBucketThreads) {
+  for (int i = tid; i < m; i += kSorterThreads) {
     sorted[base + slot.base + i] = key_score(sm.key[cur][i]);
     perm[base + slot.base + i] = kSink + (int32_t)sm.val[cur][i];
   }
