@@ -69,7 +69,7 @@ __global__ void __launch_bounds__(256) k_pool(const uint16_t* __restrict__ Q, do
 // the importance order is checked against.)
 // The d = 128 reduction runs in two halves of 64 so that the transposed key
 // tile (fp64) and pooled queries (fp64) fit twice per SM.  Thread (tk, ts)
-// accumulates keys tk + 16 a (a < 8) x segments ts + 16 b (b < 4).
+// accumulates keys 2 tk + 32 a + {0, 1} (a < 4) x segments ts + 16 b (b < 4).
 // Outputs:
 //   scores[bk][off(s) + j - 64] for candidate keys j of segment s
 //   part[bk][s][t] = (max over the tile's admissible keys,
@@ -78,7 +78,8 @@ __global__ void __launch_bounds__(256) k_pool(const uint16_t* __restrict__ Q, do
 constexpr int kScoreKeys = 128;
 constexpr int kScoreSegs = 64;
 constexpr int kScoreHalf = 64;  // d per pass
-constexpr size_t kScoreSmem = sizeof(double) * (kScoreHalf * kScoreKeys + kScoreHalf * kScoreSegs);
+constexpr int kQtStride = kScoreSegs + 2;  // padded rows: the transposed fill is conflict-free
+constexpr size_t kScoreSmem = sizeof(double) * (kScoreHalf * kScoreKeys + kScoreHalf * kQtStride);
 
 __global__ void __launch_bounds__(256, 2) k_score(const uint16_t* __restrict__ K, const double* __restrict__ qbar,
                                                  float* __restrict__ scores, float2* __restrict__ part,
@@ -92,7 +93,7 @@ __global__ void __launch_bounds__(256, 2) k_score(const uint16_t* __restrict__ K
 
   extern __shared__ double smd[];
   double* Kt = smd;                               // [64 d][128 keys]
-  double* Qt = smd + kScoreHalf * kScoreKeys;     // [64 d][64 segs]
+  double* Qt = smd + kScoreHalf * kScoreKeys;     // [64 d][64 segs], rows padded to kQtStride
   const int tid = threadIdx.x;
   const int tk = tid & 15;
   const int ts = tid >> 4;
@@ -124,16 +125,20 @@ __global__ void __launch_bounds__(256, 2) k_score(const uint16_t* __restrict__ K
     for (int q = tid; q < kScoreSegs * kScoreHalf; q += 256) {
       const int seg = q / kScoreHalf, dd = q % kScoreHalf;
       const int s = s_lo + seg;
-      Qt[dd * kScoreSegs + seg] = (s < S) ? qb[(size_t)s * kD + half * kScoreHalf + dd] : 0.0;
+      Qt[dd * kQtStride + seg] = (s < S) ? qb[(size_t)s * kD + half * kScoreHalf + dd] : 0.0;
     }
     __syncthreads();
 #pragma unroll 2
     for (int dd = 0; dd < kScoreHalf; ++dd) {
       double kk[8], qq[4];
 #pragma unroll
-      for (int a = 0; a < 8; ++a) kk[a] = Kt[dd * kScoreKeys + tk + 16 * a];
+      for (int a = 0; a < 4; ++a) {  // keys 2 tk + 32 a and 2 tk + 32 a + 1, one 16-byte load
+        const double2 k2 = *reinterpret_cast<const double2*>(Kt + dd * kScoreKeys + 2 * tk + 32 * a);
+        kk[2 * a] = k2.x;
+        kk[2 * a + 1] = k2.y;
+      }
 #pragma unroll
-      for (int q = 0; q < 4; ++q) qq[q] = Qt[dd * kScoreSegs + ts + 16 * q];
+      for (int q = 0; q < 4; ++q) qq[q] = Qt[dd * kQtStride + ts + 16 * q];
 #pragma unroll
       for (int a = 0; a < 8; ++a)
 #pragma unroll
@@ -153,7 +158,7 @@ __global__ void __launch_bounds__(256, 2) k_score(const uint16_t* __restrict__ K
     float mloc = -INFINITY;
 #pragma unroll
     for (int a = 0; a < 8; ++a) {
-      const int j = t * kScoreKeys + tk + 16 * a;
+      const int j = t * kScoreKeys + 2 * tk + 32 * (a >> 1) + (a & 1);
       v[a] = (float)(acc[a][q] * inv_sqrt_d);
       const bool adm = seg_ok && (j < N);
       if (adm) {
