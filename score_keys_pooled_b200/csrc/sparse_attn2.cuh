@@ -61,10 +61,11 @@ constexpr int kBarKEmpty = 3;   // [3]  MMA commit -> K loader
 constexpr int kBarVFull = 6;    // [2]  V loader -> MMA (TMA bytes)
 constexpr int kBarVEmpty = 8;   // [2]  MMA commit -> V loader
 constexpr int kBarQFull = 10;   //      K loader -> MMA (TMA bytes)
-constexpr int kBarSFull = 11;   // [2]  MMA commit -> softmax i
-constexpr int kBarPFull = 13;   // [2]  softmax i (count 128) -> MMA
-constexpr int kBarODone = 15;   // [2]  MMA commit -> softmax i
-constexpr int kSlotTmem = 17;
+// per 64-key half h of a tile and head i: slot + 2 h + i
+constexpr int kBarSFull = 11;   // [2][2]  MMA commit -> softmax i
+constexpr int kBarPFull = 15;   // [2][2]  softmax i (count 128) -> MMA
+constexpr int kBarODone = 19;   // [2][2]  MMA commit -> softmax i
+constexpr int kSlotTmem = 23;
 
 __device__ __forceinline__ void tc_mma_ts(uint32_t d_tmem, uint32_t a_tmem, uint64_t bdesc, uint32_t idesc,
                                           uint32_t accumulate) {
@@ -211,8 +212,7 @@ __global__ void __launch_bounds__(kAttn2Threads, 1)
   if (tid == 0) {
     for (int k = 0; k < kSlotTmem; ++k) {
       uint32_t count = 1;
-      if (k == kBarPFull || k == kBarPFull + 1) count = 128;
-      if (k == kSlotTmem) break;
+      if (k >= kBarPFull && k < kBarPFull + 4) count = 128;
       mbar_init(bar(k), count);
     }
     fence_mbar_init();
@@ -295,44 +295,48 @@ __global__ void __launch_bounds__(kAttn2Threads, 1)
     // ------------------------------------------------------------------ MMA issuer
     regs_decrease<kRegsOther>();
     if (lane == 0) {
-      const uint32_t idesc_qk = idesc_bf16_f32(128, kKT2, false);
+      const uint32_t idesc_qk = idesc_bf16_f32(128, kBk, false);   // one 64-key half
       const uint32_t idesc_pv = idesc_bf16_f32(128, 128, true);
       bool ok = mbar_wait_bounded(bar(kBarQFull), 0);
+      // per tile and half: the P V of the previous tile, then this tile's S
       for (int t = 0; ok && t <= ntiles; ++t) {
-        for (int i = 0; ok && i < 2; ++i) {
-          if (t > 0) {
-            const int tp = t - 1;
-            if (i == 0) {
-              ok = mbar_wait_bounded(bar(kBarVFull + tp % kStagesV), (uint32_t)((tp / kStagesV) & 1));
+        for (int h = 0; ok && h < 2; ++h) {
+          for (int i = 0; ok && i < 2; ++i) {
+            if (t > 0) {
+              const int tp = t - 1;
+              if (h == 0 && i == 0) {
+                ok = mbar_wait_bounded(bar(kBarVFull + tp % kStagesV), (uint32_t)((tp / kStagesV) & 1));
+                if (!ok) break;
+              }
+              ok = mbar_wait_bounded(bar(kBarPFull + 2 * h + i), (uint32_t)(tp & 1));
               if (!ok) break;
-            }
-            ok = mbar_wait_bounded(bar(kBarPFull + i), (uint32_t)(tp & 1));
-            if (!ok) break;
-            tc_fence_after();
-            const uint32_t sV = sbase + kOff2V + (tp % kStagesV) * kTile2Bytes;
+              tc_fence_after();
+              const uint32_t sV = sbase + kOff2V + (tp % kStagesV) * kTile2Bytes;
 #pragma unroll
-            for (int kk = 0; kk < kKT2 / 16; ++kk) {
-              const uint64_t bd = sdesc_sw128(sV + kk * (16 * 128), 128 * 128, 1024);
-              tc_mma_ts(tmem + 256 + 128 * i, tmem + 128 * i + 8 * kk, bd, idesc_pv, (tp > 0 || kk > 0) ? 1u : 0u);
+              for (int kk = 0; kk < kBk / 16; ++kk) {
+                const uint64_t bd = sdesc_sw128(sV + (kBk * h + 16 * kk) * 128, 128 * 128, 1024);
+                tc_mma_ts(tmem + 256 + 128 * i, tmem + 128 * i + 64 * h + 8 * kk, bd, idesc_pv,
+                          (tp > 0 || h > 0 || kk > 0) ? 1u : 0u);
+              }
+              tc_commit(bar(kBarODone + 2 * h + i));
+              if (h == 1 && i == 1) tc_commit(bar(kBarVEmpty + tp % kStagesV));
             }
-            tc_commit(bar(kBarODone + i));
-            if (i == 1) tc_commit(bar(kBarVEmpty + tp % kStagesV));
-          }
-          if (t < ntiles) {
-            if (i == 0) {
-              ok = mbar_wait_bounded(bar(kBarKFull + t % kStagesK), (uint32_t)((t / kStagesK) & 1));
-              if (!ok) break;
-            }
-            const uint32_t sQ = sbase + kOff2Q + i * kTile2Bytes;
-            const uint32_t sK = sbase + kOff2K + (t % kStagesK) * kTile2Bytes;
+            if (t < ntiles) {
+              if (h == 0 && i == 0) {
+                ok = mbar_wait_bounded(bar(kBarKFull + t % kStagesK), (uint32_t)((t / kStagesK) & 1));
+                if (!ok) break;
+              }
+              const uint32_t sQ = sbase + kOff2Q + i * kTile2Bytes;
+              const uint32_t sK = sbase + kOff2K + (t % kStagesK) * kTile2Bytes + kBk * h * 128;
 #pragma unroll
-            for (int kk = 0; kk < 8; ++kk) {
-              const uint64_t ad = sdesc_sw128(sQ + (kk >> 2) * (128 * 128) + (kk & 3) * 32, 16, 1024);
-              const uint64_t bd = sdesc_sw128(sK + (kk >> 2) * (128 * 128) + (kk & 3) * 32, 16, 1024);
-              tc_mma_ss(tmem + 128 * i, ad, bd, idesc_qk, kk > 0 ? 1u : 0u);
+              for (int kk = 0; kk < 8; ++kk) {
+                const uint64_t ad = sdesc_sw128(sQ + (kk >> 2) * (128 * 128) + (kk & 3) * 32, 16, 1024);
+                const uint64_t bd = sdesc_sw128(sK + (kk >> 2) * (128 * 128) + (kk & 3) * 32, 16, 1024);
+                tc_mma_ss(tmem + 128 * i + 64 * h, ad, bd, idesc_qk, kk > 0 ? 1u : 0u);
+              }
+              tc_commit(bar(kBarSFull + 2 * h + i));
+              if (h == 1 && i == 1) tc_commit(bar(kBarKEmpty + t % kStagesK));
             }
-            tc_commit(bar(kBarSFull + i));
-            if (i == 1) tc_commit(bar(kBarKEmpty + t % kStagesK));
           }
         }
       }
@@ -350,92 +354,95 @@ __global__ void __launch_bounds__(kAttn2Threads, 1)
     const float sl2 = 1.4426950408889634f * 0.08838834764831845f;  // log2(e) / sqrt(d)
     float m_run = -INFINITY, ell = 0.f;
     bool ok = true;
-    for (int t = 0; t < ntiles; ++t) {
-      if (!warp_wait(bar(kBarSFull + qi), (uint32_t)(t & 1))) { ok = false; break; }
-      tc_fence_after();
-      // key c of a half is visible iff (c mod 64) <= lim of that half
-      int lim_a, lim_b;
-      {
+    for (int t = 0; ok && t < ntiles; ++t) {
+      // key c of a half is visible iff c <= lim of that half
+      int lim_h[2];
+#pragma unroll
+      for (int h = 0; h < 2; ++h) {
         int j0;
-        const int ka = walk2_block(wk, s, 2 * t, j0);
-        lim_a = ka == 3 ? -1 : (ka == 0 ? row - j0 : kBk);
-        const int kb = walk2_block(wk, s, 2 * t + 1, j0);
-        lim_b = kb == 3 ? -1 : (kb == 0 ? row - j0 : kBk);
+        const int kind = walk2_block(wk, s, 2 * t + h, j0);
+        lim_h[h] = kind == 3 ? -1 : (kind == 0 ? row - j0 : kBk);
       }
-      // the tile's 128 scores of this row, one tensor-memory round trip
-      float x[kKT2];
-#pragma unroll
-      for (int cc = 0; cc < kKT2; cc += 32) tmem_ld32(tS + cc, x + cc);
-      tc_wait_ld();
-      const bool full_tile = lim_a >= kBk && lim_b >= kBk;  // no key masked
-      float mt = -INFINITY;
-      if (full_tile) {
-        float m4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
-#pragma unroll
-        for (int c = 0; c < kKT2; c += 2) m4[(c >> 1) & 3] = fmax3(m4[(c >> 1) & 3], x[c], x[c + 1]);
-        mt = fmaxf(fmax3(m4[0], m4[1], m4[2]), m4[3]);
-      } else {
-#pragma unroll
-        for (int c = 0; c < kKT2; ++c)
-          if ((c & 63) <= (c < 64 ? lim_a : lim_b)) mt = fmaxf(mt, x[c]);
-      }
-      mt *= sl2;
-      const bool move = mt > m_run + 8.f;
-      float alpha = 1.f;
-      if (move) {
-        alpha = (m_run == -INFINITY) ? 0.f : ex2_approx(m_run - mt);
-        m_run = mt;
-        ell *= alpha;
-      }
-      // P = exp2(S - m) as bf16 pairs, packed in place into x[0 .. 63]
-      float rs;
-      if (full_tile) {
-        const uint64_t s2 = f2_pack(sl2, sl2), nm2 = f2_pack(-m_run, -m_run);
-        uint64_t rs2 = 0;
-#pragma unroll
-        for (int c = 0; c < kKT2; c += 2) {
-          const uint64_t v = f2_fma(f2_pack(x[c], x[c + 1]), s2, nm2);
-          const float p0 = ex2_approx(f2_lo(v)), p1 = ex2_approx(f2_hi(v));
-          rs2 = f2_add(rs2, f2_pack(p0, p1));
-          x[c / 2] = __uint_as_float(pack_bf16x2(p0, p1));
-        }
-        rs = f2_lo(rs2) + f2_hi(rs2);
-      } else {
-        rs = 0.f;
-#pragma unroll
-        for (int c = 0; c < kKT2; c += 2) {
-          const int lim = c < 64 ? lim_a : lim_b;
-          const float p0 = ((c & 63) <= lim) ? ex2_approx(fmaf(x[c], sl2, -m_run)) : 0.f;
-          const float p1 = (((c + 1) & 63) <= lim) ? ex2_approx(fmaf(x[c + 1], sl2, -m_run)) : 0.f;
-          rs += p0 + p1;
-          x[c / 2] = __uint_as_float(pack_bf16x2(p0, p1));
-        }
-      }
-      ell += rs;
-      // the previous P V must be done before P_i and O_i are rewritten (it was
-      // issued before this tile's S, so this wait normally returns at once)
-      if (t > 0) {
-        if (!warp_wait(bar(kBarODone + qi), (uint32_t)((t - 1) & 1))) { ok = false; break; }
+#pragma unroll 1
+      for (int h = 0; h < 2; ++h) {
+        if (!warp_wait(bar(kBarSFull + 2 * h + qi), (uint32_t)(t & 1))) { ok = false; break; }
         tc_fence_after();
-      }
-      tmem_st32(tS, x);
-      tmem_st32(tS + 32, x + 32);
-      if (t > 0 && __any_sync(0xffffffffu, move)) {
+        const int lim = lim_h[h];
+        float x[kBk];
+        tmem_ld32(tS + 64 * h, x);
+        tmem_ld32(tS + 64 * h + 32, x + 32);
+        tc_wait_ld();
+        const bool full = lim >= kBk;  // no key masked
+        float mt = -INFINITY;
+        if (full) {
+          float m4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
 #pragma unroll
-        for (int cc = 0; cc < 128; cc += 32) {
-          float o[32];
-          tmem_ld32(tO + cc, o);
-          tc_wait_ld();
+          for (int c = 0; c < kBk; c += 2) m4[(c >> 1) & 3] = fmax3(m4[(c >> 1) & 3], x[c], x[c + 1]);
+          mt = fmaxf(fmax3(m4[0], m4[1], m4[2]), m4[3]);
+        } else {
 #pragma unroll
-          for (int k = 0; k < 32; ++k) o[k] *= alpha;
-          tmem_st32(tO + cc, o);
+          for (int c = 0; c < kBk; ++c)
+            if (c <= lim) mt = fmaxf(mt, x[c]);
         }
+        mt *= sl2;
+        const bool move = mt > m_run + 8.f;
+        float alpha = 1.f;
+        if (move) {
+          alpha = (m_run == -INFINITY) ? 0.f : ex2_approx(m_run - mt);
+          m_run = mt;
+          ell *= alpha;
+        }
+        // a moved reference rescales O once every P V issued so far is done:
+        // half a waits for the previous tile's half-b product, half b for this
+        // tile's half-a product (the other products are already complete)
+        if ((t > 0 || h == 1) && __any_sync(0xffffffffu, move)) {
+          const int oh = 1 - h;
+          const int ot = h ? t : t - 1;
+          if (!warp_wait(bar(kBarODone + 2 * oh + qi), (uint32_t)(ot & 1))) { ok = false; break; }
+          tc_fence_after();
+#pragma unroll
+          for (int cc = 0; cc < 128; cc += 32) {
+            float o[32];
+            tmem_ld32(tO + cc, o);
+            tc_wait_ld();
+#pragma unroll
+            for (int k = 0; k < 32; ++k) o[k] *= alpha;
+            tmem_st32(tO + cc, o);
+          }
+        }
+        // P = exp2(S - m) as bf16 pairs, packed in place into x[0 .. 31]
+        float rs;
+        if (full) {
+          const uint64_t s2 = f2_pack(sl2, sl2), nm2 = f2_pack(-m_run, -m_run);
+          uint64_t rs2 = 0;
+#pragma unroll
+          for (int c = 0; c < kBk; c += 2) {
+            const uint64_t v = f2_fma(f2_pack(x[c], x[c + 1]), s2, nm2);
+            const float p0 = ex2_approx(f2_lo(v)), p1 = ex2_approx(f2_hi(v));
+            rs2 = f2_add(rs2, f2_pack(p0, p1));
+            x[c / 2] = __uint_as_float(pack_bf16x2(p0, p1));
+          }
+          rs = f2_lo(rs2) + f2_hi(rs2);
+        } else {
+          rs = 0.f;
+#pragma unroll
+          for (int c = 0; c < kBk; c += 2) {
+            const float p0 = (c <= lim) ? ex2_approx(fmaf(x[c], sl2, -m_run)) : 0.f;
+            const float p1 = (c + 1 <= lim) ? ex2_approx(fmaf(x[c + 1], sl2, -m_run)) : 0.f;
+            rs += p0 + p1;
+            x[c / 2] = __uint_as_float(pack_bf16x2(p0, p1));
+          }
+        }
+        ell += rs;
+        // P of this half over the S columns already read; the previous P of
+        // these columns was consumed before this S was computed
+        tmem_st32(tS + 64 * h, x);
+        tc_wait_st();
+        tc_fence_before();
+        mbar_arrive(bar(kBarPFull + 2 * h + qi));
       }
-      tc_wait_st();
-      tc_fence_before();
-      mbar_arrive(bar(kBarPFull + qi));
     }
-    if (ok) ok = warp_wait(bar(kBarODone + qi), (uint32_t)((ntiles - 1) & 1));
+    if (ok) ok = warp_wait(bar(kBarODone + 2 + qi), (uint32_t)((ntiles - 1) & 1));
     if (!ok) {
       if (lane == 0) set_error(kErrTimeout);
     } else {
