@@ -260,13 +260,11 @@ s2o_status s2o_attention(const s2o_config* cfg, const uint16_t* Q, const uint16_
     a.B = cfg->B; a.Hq = cfg->Hq; a.Hkv = cfg->Hkv; a.N = cfg->N; a.S = nseg(cfg);
     a.T = ncand_total(cfg);
     a.out_f32 = out_dtype == S2O_OUT_F32;
-    CUtensorMap tmQ, tmK, tmV;
-    if (!encode_rows_map(&tmQ, Q, (uint64_t)cfg->B * cfg->Hq * cfg->N, 128) ||
-        !encode_rows_map(&tmK, K, (uint64_t)cfg->B * cfg->Hkv * cfg->N, 1) ||
-        !encode_rows_map(&tmV, V, (uint64_t)cfg->B * cfg->Hkv * cfg->N, 1))
+    CUtensorMap tmQ;
+    if (!encode_rows_map(&tmQ, Q, (uint64_t)cfg->B * cfg->Hq * cfg->N, 128))
       return S2O_ERR_CUDA;
     const int64_t ncta = (int64_t)cfg->B * cfg->Hkv * a.S * (G / 2);
-    k_sparse_attn2<<<(unsigned)ncta, kAttn2Threads, kAttn2Smem, s>>>(a, tmQ, tmK, tmV);
+    k_sparse_attn2<<<(unsigned)ncta, kAttn2Threads, kAttn2Smem, s>>>(a, tmQ);
   } else {
     AttnArgs a;
     a.Q = Q; a.K = K; a.V = V; a.perm = perm; a.nblocks = nblocks; a.O = O;

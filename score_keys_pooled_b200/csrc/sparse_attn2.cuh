@@ -9,22 +9,29 @@
 //     share every gathered K/V tile (each tile is fetched once for 256 rows);
 //   * 128-key tiles: 64-key blocks of the key walk taken two at a time
 //     (diagonal, previous window, sinks, then the kept candidate blocks; an
-//     odd last block leaves an empty, zero-filled and masked half);
+//     odd last block leaves an empty, zero-filled and masked half); the
+//     tensor core and the softmax step through them one 64-key chunk (one
+//     block, half a tile) at a time;
 //   * warp roles (384 threads): warps 0-3 and 4-7 run the online softmax of
-//     head 0 and head 1 (thread = row = TMEM lane), warp 8 issues tcgen05.mma
-//     from one thread, warps 9 and 10 gather K and V rows with TMA
-//     (tile::gather4: four 256-byte rows per pair of instructions, one per
-//     64-column half, written 128B-swizzled by the TMA unit) into a 3-stage K
-//     ring and a 2-stage V ring whose mbarriers count the landed bytes (K is
-//     released as soon as both heads' S are computed, so its loads run up to
-//     three tiles ahead); the row indices of the next tile are fetched while
-//     a stage drains; Q arrives as 2D TMA tiles;
-//   * tensor memory (512 columns): S_i = Q_i K^T in columns [128 i, 128 i+128),
-//     O_i in [256 + 128 i, ...); P_i (bf16, two per column) overwrites the
-//     first 64 columns of S_i and is the A operand of O_i += P_i V straight
-//     from tensor memory, so P never touches shared memory;
-//   * while one head's softmax runs, the tensor core works on the other
-//     head's products (ping-pong through the mbarriers below);
+//     head 0 and head 1 (thread = row = TMEM lane), one thread of warp 8 and
+//     one of warp 11 issue the tcgen05.mma of head 0 and head 1 (a single
+//     issuer stalls the tensor pipe whenever it waits on one head's softmax,
+//     and one thread cannot issue fast enough to keep it busy anyway), warps
+//     9 and 10 gather K and V rows with cp.async (16 bytes a lane, written in
+//     the tensor core's 128B-swizzled layout) into a 3-stage K ring and a
+//     2-stage V ring; a loader arrives on a stage's mbarrier once its copies
+//     have landed (K is released as soon as both heads' S are computed, so
+//     its loads run up to three tiles ahead); the key indices of the next
+//     tile are fetched while the copies of this one fly; Q arrives as 2D
+//     TMA tiles;
+//   * tensor memory (512 columns): O_i in [128 i, 128 i + 128); S_i of one
+//     chunk in [256 + 64 i, +64); two P buffers per head (bf16, two per
+//     column) in [384 + 64 i + 32 b, +32).  P is the A operand of
+//     O_i += P_i V straight from tensor memory, so it never touches shared
+//     memory.  S_i is released as soon as the softmax has read it into
+//     registers, so Q K^T of the next chunk runs while the softmax of this
+//     one computes; the exp2 work (bound by the special-function unit) and
+//     the tensor core then overlap instead of waiting on each other;
 //   * registers are rebalanced per warpgroup (setmaxnreg): the launch gives
 //     168 per thread; warps 8-11 drop to 80 and the two softmax warpgroups
 //     rise to 208 (per SM sub-partition 2 x 208 + 80 <= 3 x 168), enough to
@@ -42,7 +49,8 @@ namespace s2o {
 
 constexpr int kKT2 = 128;                 // keys per tile
 constexpr int kAttn2Threads = 384;
-constexpr int kMmaWarp = 8;
+constexpr int kMmaWarp = 8;                          // issuer of head 0 (and TMEM owner)
+constexpr int kMmaWarp1 = 11;                        // issuer of head 1
 constexpr int kLoadWarp0 = 9;
 constexpr int kStagesK = 3;                          // K ring (freed once Q K^T of both heads is done)
 constexpr int kStagesV = 2;                          // V ring (freed once P V of both heads is done)
@@ -56,16 +64,21 @@ constexpr size_t kAttn2Smem = kAttn2SmemData + 1024;  // + alignment slack
 constexpr uint32_t kTmem2Cols = 512;
 
 // barrier slots (8 bytes each) from kOff2Bar
-constexpr int kBarKFull = 0;    // [3]  K loader -> MMA (TMA bytes)
-constexpr int kBarKEmpty = 3;   // [3]  MMA commit -> K loader
-constexpr int kBarVFull = 6;    // [2]  V loader -> MMA (TMA bytes)
-constexpr int kBarVEmpty = 8;   // [2]  MMA commit -> V loader
+constexpr int kBarKFull = 0;    // [3]  K loader (after its copies landed) -> MMA
+constexpr int kBarKEmpty = 3;   // [3]  MMA commits of both issuers (count 2) -> K loader
+constexpr int kBarVFull = 6;    // [2]  V loader (after its copies landed) -> MMA
+constexpr int kBarVEmpty = 8;   // [2]  MMA commits of both issuers (count 2) -> V loader
 constexpr int kBarQFull = 10;   //      K loader -> MMA (TMA bytes)
-// per 64-key half h of a tile and head i: slot + 2 h + i
-constexpr int kBarSFull = 11;   // [2][2]  MMA commit -> softmax i
-constexpr int kBarPFull = 15;   // [2][2]  softmax i (count 128) -> MMA
-constexpr int kBarODone = 19;   // [2][2]  MMA commit -> softmax i
+// per head i (and P buffer b)
+constexpr int kBarSFull = 11;   // [2]     MMA commit (S_i written) -> softmax i
+constexpr int kBarSEmpty = 13;  // [2]     softmax i, one arrive per warp (S_i read) -> MMA
+constexpr int kBarPFull = 15;   // [2][2]  softmax i, one arrive per warp (P_i,b written) -> MMA; slot + 2 i + b
+constexpr int kBarODone = 19;   // [2][2]  MMA commit (P_i,b consumed, O_i updated) -> softmax i
 constexpr int kSlotTmem = 23;
+// tensor-memory columns
+__device__ __forceinline__ uint32_t col_o(int i) { return 128u * i; }
+__device__ __forceinline__ uint32_t col_s(int i) { return 256u + 64u * i; }
+__device__ __forceinline__ uint32_t col_p(int i, int b) { return 384u + 64u * i + 32u * b; }
 
 __device__ __forceinline__ void tc_mma_ts(uint32_t d_tmem, uint32_t a_tmem, uint64_t bdesc, uint32_t idesc,
                                           uint32_t accumulate) {
@@ -123,15 +136,6 @@ __device__ __forceinline__ void tma_load_2d(uint32_t dst, const CUtensorMap* map
       "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(bar)
       : "memory");
 }
-// four rows y0..y3, columns [x, x + box width), landing as four consecutive rows
-__device__ __forceinline__ void tma_gather4(uint32_t dst, const CUtensorMap* map, int x, int y0, int y1, int y2,
-                                            int y3, uint32_t bar) {
-  asm volatile(
-      "cp.async.bulk.tensor.2d.shared::cluster.global.tile::gather4.mbarrier::complete_tx::bytes"
-      " [%0], [%1, {%2, %3, %4, %5, %6}], [%7];\n" ::"r"(dst),
-      "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y0), "r"(y1), "r"(y2), "r"(y3), "r"(bar)
-      : "memory");
-}
 // warp-uniform bounded wait: every lane polls, all agree on the outcome
 __device__ __forceinline__ bool warp_wait(uint32_t bar, uint32_t parity) {
   const bool ok = mbar_wait_bounded(bar, parity);
@@ -176,8 +180,7 @@ struct Attn2Args {
 };
 
 __global__ void __launch_bounds__(kAttn2Threads, 1)
-    k_sparse_attn2(Attn2Args a, const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
-                   const __grid_constant__ CUtensorMap tmV) {
+    k_sparse_attn2(Attn2Args a, const __grid_constant__ CUtensorMap tmQ) {
   extern __shared__ uint8_t smem_raw[];
   const uint32_t sbase = (smem_u32(smem_raw) + 1023u) & ~1023u;
   uint8_t* sgen = smem_raw + (sbase - smem_u32(smem_raw));
@@ -212,7 +215,8 @@ __global__ void __launch_bounds__(kAttn2Threads, 1)
   if (tid == 0) {
     for (int k = 0; k < kSlotTmem; ++k) {
       uint32_t count = 1;
-      if (k >= kBarPFull && k < kBarPFull + 4) count = 128;
+      if ((k >= kBarSEmpty && k < kBarSEmpty + 2) || (k >= kBarPFull && k < kBarPFull + 4)) count = 4;
+      if ((k >= kBarKEmpty && k < kBarKEmpty + kStagesK) || (k >= kBarVEmpty && k < kBarVEmpty + kStagesV)) count = 2;
       mbar_init(bar(k), count);
     }
     fence_mbar_init();
@@ -225,23 +229,20 @@ __global__ void __launch_bounds__(kAttn2Threads, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
-  if (warp > kLoadWarp0 + 1) {
-    // warp 11: no role (it completes the register-donating warpgroup)
-    regs_decrease<kRegsOther>();
-  } else if (warp >= kLoadWarp0) {
-    // ------------------------------------------------------------------ loaders (TMA)
-    // warp 9 loads Q and the K ring, warp 10 the V ring
+  if (warp >= kLoadWarp0 && warp < kMmaWarp1) {
+    // ------------------------------------------------------------------ loaders
+    // warp 9 loads Q (2D TMA) and the K ring, warp 10 the V ring.  The
+    // gathered rows go through cp.async, 16 bytes per lane: lanes 0-15 copy
+    // one 256-byte row, lanes 16-31 the next, written in the 128B-swizzled
+    // layout the tensor core reads (one TMA gather4 per four rows issues far
+    // slower than the load/store unit takes these copies).
     regs_decrease<kRegsOther>();
     const bool is_k = warp == kLoadWarp0;
     const int nst = is_k ? kStagesK : kStagesV;
     const int bar_full = is_k ? kBarKFull : kBarVFull;
     const int bar_empty = is_k ? kBarKEmpty : kBarVEmpty;
     const uint32_t ring = sbase + (is_k ? kOff2K : kOff2V);
-    const CUtensorMap* map = is_k ? &tmK : &tmV;
-    // rows of K/V as [B*Hkv*N, 128]; a row coordinate past the end is out of
-    // bounds and reads as zeros (empty halves, keys past N)
-    const int zero_row = a.B * a.Hkv * a.N;
-    const int kv_row0 = bk * a.N;
+    const uint16_t* kv = (is_k ? a.K : a.V) + (size_t)bk * a.N * kD;
     if (is_k && lane == 0) {
       mbar_expect_tx(bar(kBarQFull), 2 * kTile2Bytes);
 #pragma unroll
@@ -253,8 +254,9 @@ __global__ void __launch_bounds__(kAttn2Threads, 1)
     }
     const int32_t* pseg = a.perm + (size_t)bk * a.T + cand_offset(s);
     const int cand_hi = kLq * s - kWin;
-    // key rows of tile t handled by this lane: rows 4 lane .. 4 lane + 3
-    auto tile_rows = [&](int t, int* y) {
+    // keys of tile rows 4 lane .. 4 lane + 3 (-1: a zero row, for an empty
+    // half or a key past N)
+    auto tile_keys = [&](int t, int* y) {
       int j0;
       const int kind = walk2_block(wk, s, 2 * t + (lane >> 4), j0);
 #pragma unroll
@@ -271,11 +273,14 @@ __global__ void __launch_bounds__(kAttn2Threads, 1)
           j = j0 + rr;
           if (j >= a.N) j = -1;
         }
-        y[k] = j >= 0 ? kv_row0 + j : zero_row;
+        y[k] = j;
       }
     };
+    // this lane's 16-byte chunk q of a row: swizzle atom q / 8, chunk q % 8
+    const int q = lane & 15, sel = lane >> 4;
+    const uint32_t lane_off = (uint32_t)(q >> 3) * (128 * 128);
     int y[4];
-    if (ntiles > 0) tile_rows(0, y);
+    if (ntiles > 0) tile_keys(0, y);
     for (int t = 0; t < ntiles; ++t) {
       const int st = t % nst;
       const int round = t / nst;
@@ -283,61 +288,78 @@ __global__ void __launch_bounds__(kAttn2Threads, 1)
         if (lane == 0) set_error(kErrTimeout);
         break;
       }
-      if (lane == 0) mbar_expect_tx(bar(bar_full + st), kTile2Bytes);
-      __syncwarp();
-      const uint32_t dst = ring + st * kTile2Bytes + lane * (4 * 128);
+      const uint32_t dst0 = ring + st * kTile2Bytes + lane_off;
 #pragma unroll
-      for (int half = 0; half < 2; ++half)
-        tma_gather4(dst + half * (128 * 128), map, 64 * half, y[0], y[1], y[2], y[3], bar(bar_full + st));
-      if (t + 1 < ntiles) tile_rows(t + 1, y);  // loads overlap the next stage's drain
+      for (int jj = 0; jj < 64; ++jj) {
+        // tile row r = 2 jj + sel; its key sits in lane r / 4, register r % 4
+        const int v0 = __shfl_sync(0xffffffffu, y[2 * (jj & 1)], jj >> 1);
+        const int v1 = __shfl_sync(0xffffffffu, y[2 * (jj & 1) + 1], jj >> 1);
+        const int key = sel ? v1 : v0;
+        const int r = 2 * jj + sel;
+        const uint32_t dst = dst0 + (uint32_t)r * 128 + ((uint32_t)((q & 7) ^ (r & 7)) << 4);
+        const uint16_t* src = kv + (size_t)(key < 0 ? 0 : key) * kD + 8 * q;
+        cp_async16(dst, src, key < 0 ? 0u : 16u);
+      }
+      if (t + 1 < ntiles) tile_keys(t + 1, y);  // index loads overlap the copies
+      cp_async_wait_all();
+      fence_proxy_async_smem();  // generic-proxy writes -> tensor-core reads
+      __syncwarp();
+      if (lane == 0) mbar_arrive(bar(bar_full + st));
     }
-  } else if (warp == kMmaWarp) {
-    // ------------------------------------------------------------------ MMA issuer
+  } else if (warp == kMmaWarp || warp == kMmaWarp1) {
+    // ------------------------------------------------------------------ MMA issuers
+    // head i's products, in order: its P V of tile t-1 and half h precedes its
+    // Q K^T of tile t and half h, which overwrites that P.  The two issuers
+    // share only the K/V stages (both commit before a stage is refilled).
     regs_decrease<kRegsOther>();
+    const int i = warp == kMmaWarp ? 0 : 1;
     if (lane == 0) {
       const uint32_t idesc_qk = idesc_bf16_f32(128, kBk, false);   // one 64-key half
       const uint32_t idesc_pv = idesc_bf16_f32(128, 128, true);
       bool ok = mbar_wait_bounded(bar(kBarQFull), 0);
-      // per tile and half: the P V of the previous tile, then this tile's S
-      for (int t = 0; ok && t <= ntiles; ++t) {
-        for (int h = 0; ok && h < 2; ++h) {
-          for (int i = 0; ok && i < 2; ++i) {
-            if (t > 0) {
-              const int tp = t - 1;
-              if (h == 0 && i == 0) {
-                ok = mbar_wait_bounded(bar(kBarVFull + tp % kStagesV), (uint32_t)((tp / kStagesV) & 1));
-                if (!ok) break;
-              }
-              ok = mbar_wait_bounded(bar(kBarPFull + 2 * h + i), (uint32_t)(tp & 1));
-              if (!ok) break;
-              tc_fence_after();
-              const uint32_t sV = sbase + kOff2V + (tp % kStagesV) * kTile2Bytes;
-#pragma unroll
-              for (int kk = 0; kk < kBk / 16; ++kk) {
-                const uint64_t bd = sdesc_sw128(sV + (kBk * h + 16 * kk) * 128, 128 * 128, 1024);
-                tc_mma_ts(tmem + 256 + 128 * i, tmem + 128 * i + 64 * h + 8 * kk, bd, idesc_pv,
-                          (tp > 0 || h > 0 || kk > 0) ? 1u : 0u);
-              }
-              tc_commit(bar(kBarODone + 2 * h + i));
-              if (h == 1 && i == 1) tc_commit(bar(kBarVEmpty + tp % kStagesV));
-            }
-            if (t < ntiles) {
-              if (h == 0 && i == 0) {
-                ok = mbar_wait_bounded(bar(kBarKFull + t % kStagesK), (uint32_t)((t / kStagesK) & 1));
-                if (!ok) break;
-              }
-              const uint32_t sQ = sbase + kOff2Q + i * kTile2Bytes;
-              const uint32_t sK = sbase + kOff2K + (t % kStagesK) * kTile2Bytes + kBk * h * 128;
-#pragma unroll
-              for (int kk = 0; kk < 8; ++kk) {
-                const uint64_t ad = sdesc_sw128(sQ + (kk >> 2) * (128 * 128) + (kk & 3) * 32, 16, 1024);
-                const uint64_t bd = sdesc_sw128(sK + (kk >> 2) * (128 * 128) + (kk & 3) * 32, 16, 1024);
-                tc_mma_ss(tmem + 128 * i + 64 * h, ad, bd, idesc_qk, kk > 0 ? 1u : 0u);
-              }
-              tc_commit(bar(kBarSFull + 2 * h + i));
-              if (h == 1 && i == 1) tc_commit(bar(kBarKEmpty + t % kStagesK));
-            }
+      // chunk c = half c & 1 of tile c >> 1: S of chunk c as soon as the
+      // softmax has read S of chunk c - 1, then P V of chunk c - 1
+      const int nch = 2 * ntiles;
+      for (int c = 0; ok && c <= nch; ++c) {
+        if (c < nch) {
+          const int t = c >> 1, h = c & 1;
+          if (h == 0) {
+            ok = mbar_wait_bounded(bar(kBarKFull + t % kStagesK), (uint32_t)((t / kStagesK) & 1));
+            if (!ok) break;
           }
+          if (c > 0) {
+            ok = mbar_wait_bounded(bar(kBarSEmpty + i), (uint32_t)((c - 1) & 1));
+            if (!ok) break;
+            tc_fence_after();
+          }
+          const uint32_t sQ = sbase + kOff2Q + i * kTile2Bytes;
+          const uint32_t sK = sbase + kOff2K + (t % kStagesK) * kTile2Bytes + kBk * h * 128;
+#pragma unroll
+          for (int kk = 0; kk < 8; ++kk) {
+            const uint64_t ad = sdesc_sw128(sQ + (kk >> 2) * (128 * 128) + (kk & 3) * 32, 16, 1024);
+            const uint64_t bd = sdesc_sw128(sK + (kk >> 2) * (128 * 128) + (kk & 3) * 32, 16, 1024);
+            tc_mma_ss(tmem + col_s(i), ad, bd, idesc_qk, kk > 0 ? 1u : 0u);
+          }
+          tc_commit(bar(kBarSFull + i));
+          if (h == 1) tc_commit(bar(kBarKEmpty + t % kStagesK));
+        }
+        if (c > 0) {
+          const int cp = c - 1, tp = cp >> 1, hp = cp & 1;
+          if (hp == 0) {
+            ok = mbar_wait_bounded(bar(kBarVFull + tp % kStagesV), (uint32_t)((tp / kStagesV) & 1));
+            if (!ok) break;
+          }
+          ok = mbar_wait_bounded(bar(kBarPFull + 2 * i + hp), (uint32_t)((cp >> 1) & 1));
+          if (!ok) break;
+          tc_fence_after();
+          const uint32_t sV = sbase + kOff2V + (tp % kStagesV) * kTile2Bytes;
+#pragma unroll
+          for (int kk = 0; kk < kBk / 16; ++kk) {
+            const uint64_t bd = sdesc_sw128(sV + (kBk * hp + 16 * kk) * 128, 128 * 128, 1024);
+            tc_mma_ts(tmem + col_o(i), tmem + col_p(i, hp) + 8 * kk, bd, idesc_pv, (cp > 0 || kk > 0) ? 1u : 0u);
+          }
+          tc_commit(bar(kBarODone + 2 * i + hp));
+          if (hp == 1) tc_commit(bar(kBarVEmpty + tp % kStagesV));
         }
       }
       if (!ok) set_error(kErrTimeout);
@@ -349,100 +371,99 @@ __global__ void __launch_bounds__(kAttn2Threads, 1)
     const int r = tid & 127;                // row in the segment
     const int row = row0 + r;
     const uint32_t lane_base = (uint32_t)((warp & 3) * 32) << 16;
-    const uint32_t tS = tmem + 128 * qi + lane_base;
-    const uint32_t tO = tmem + 256 + 128 * qi + lane_base;
+    const uint32_t tS = tmem + col_s(qi) + lane_base;
+    const uint32_t tO = tmem + col_o(qi) + lane_base;
     const float sl2 = 1.4426950408889634f * 0.08838834764831845f;  // log2(e) / sqrt(d)
     float m_run = -INFINITY, ell = 0.f;
     bool ok = true;
-    for (int t = 0; ok && t < ntiles; ++t) {
-      // key c of a half is visible iff c <= lim of that half
-      int lim_h[2];
+    const int nch = 2 * ntiles;
+    for (int c = 0; ok && c < nch; ++c) {
+      // key k of the chunk is visible iff k <= lim
+      int j0;
+      const int kind = walk2_block(wk, s, c, j0);
+      const int lim = kind == 3 ? -1 : (kind == 0 ? row - j0 : kBk);
+      if (!warp_wait(bar(kBarSFull + qi), (uint32_t)(c & 1))) { ok = false; break; }
+      tc_fence_after();
+      float x[kBk];
+      tmem_ld32(tS, x);
+      tmem_ld32(tS + 32, x + 32);
+      tc_wait_ld();
+      // S_i is free for the next chunk's Q K^T
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(bar(kBarSEmpty + qi));
+      const bool full = lim >= kBk;  // no key masked
+      float mt = -INFINITY;
+      if (full) {
+        float m4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
 #pragma unroll
-      for (int h = 0; h < 2; ++h) {
-        int j0;
-        const int kind = walk2_block(wk, s, 2 * t + h, j0);
-        lim_h[h] = kind == 3 ? -1 : (kind == 0 ? row - j0 : kBk);
+        for (int k = 0; k < kBk; k += 2) m4[(k >> 1) & 3] = fmax3(m4[(k >> 1) & 3], x[k], x[k + 1]);
+        mt = fmaxf(fmax3(m4[0], m4[1], m4[2]), m4[3]);
+      } else {
+#pragma unroll
+        for (int k = 0; k < kBk; ++k)
+          if (k <= lim) mt = fmaxf(mt, x[k]);
       }
-#pragma unroll 1
-      for (int h = 0; h < 2; ++h) {
-        if (!warp_wait(bar(kBarSFull + 2 * h + qi), (uint32_t)(t & 1))) { ok = false; break; }
+      mt *= sl2;
+      const bool move = mt > m_run + 8.f;
+      float alpha = 1.f;
+      if (move) {
+        alpha = (m_run == -INFINITY) ? 0.f : ex2_approx(m_run - mt);
+        m_run = mt;
+        ell *= alpha;
+      }
+      // a moved reference rescales O once every P V issued so far (the last
+      // one is chunk c - 1's) is done
+      if (c > 0 && __any_sync(0xffffffffu, move)) {
+        if (!warp_wait(bar(kBarODone + 2 * qi + ((c - 1) & 1)), (uint32_t)(((c - 1) >> 1) & 1))) { ok = false; break; }
         tc_fence_after();
-        const int lim = lim_h[h];
-        float x[kBk];
-        tmem_ld32(tS + 64 * h, x);
-        tmem_ld32(tS + 64 * h + 32, x + 32);
-        tc_wait_ld();
-        const bool full = lim >= kBk;  // no key masked
-        float mt = -INFINITY;
-        if (full) {
-          float m4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
 #pragma unroll
-          for (int c = 0; c < kBk; c += 2) m4[(c >> 1) & 3] = fmax3(m4[(c >> 1) & 3], x[c], x[c + 1]);
-          mt = fmaxf(fmax3(m4[0], m4[1], m4[2]), m4[3]);
-        } else {
+        for (int cc = 0; cc < 128; cc += 32) {
+          float o[32];
+          tmem_ld32(tO + cc, o);
+          tc_wait_ld();
 #pragma unroll
-          for (int c = 0; c < kBk; ++c)
-            if (c <= lim) mt = fmaxf(mt, x[c]);
+          for (int k = 0; k < 32; ++k) o[k] *= alpha;
+          tmem_st32(tO + cc, o);
         }
-        mt *= sl2;
-        const bool move = mt > m_run + 8.f;
-        float alpha = 1.f;
-        if (move) {
-          alpha = (m_run == -INFINITY) ? 0.f : ex2_approx(m_run - mt);
-          m_run = mt;
-          ell *= alpha;
-        }
-        // a moved reference rescales O once every P V issued so far is done:
-        // half a waits for the previous tile's half-b product, half b for this
-        // tile's half-a product (the other products are already complete)
-        if ((t > 0 || h == 1) && __any_sync(0xffffffffu, move)) {
-          const int oh = 1 - h;
-          const int ot = h ? t : t - 1;
-          if (!warp_wait(bar(kBarODone + 2 * oh + qi), (uint32_t)(ot & 1))) { ok = false; break; }
-          tc_fence_after();
-#pragma unroll
-          for (int cc = 0; cc < 128; cc += 32) {
-            float o[32];
-            tmem_ld32(tO + cc, o);
-            tc_wait_ld();
-#pragma unroll
-            for (int k = 0; k < 32; ++k) o[k] *= alpha;
-            tmem_st32(tO + cc, o);
-          }
-        }
-        // P = exp2(S - m) as bf16 pairs, packed in place into x[0 .. 31]
-        float rs;
-        if (full) {
-          const uint64_t s2 = f2_pack(sl2, sl2), nm2 = f2_pack(-m_run, -m_run);
-          uint64_t rs2 = 0;
-#pragma unroll
-          for (int c = 0; c < kBk; c += 2) {
-            const uint64_t v = f2_fma(f2_pack(x[c], x[c + 1]), s2, nm2);
-            const float p0 = ex2_approx(f2_lo(v)), p1 = ex2_approx(f2_hi(v));
-            rs2 = f2_add(rs2, f2_pack(p0, p1));
-            x[c / 2] = __uint_as_float(pack_bf16x2(p0, p1));
-          }
-          rs = f2_lo(rs2) + f2_hi(rs2);
-        } else {
-          rs = 0.f;
-#pragma unroll
-          for (int c = 0; c < kBk; c += 2) {
-            const float p0 = (c <= lim) ? ex2_approx(fmaf(x[c], sl2, -m_run)) : 0.f;
-            const float p1 = (c + 1 <= lim) ? ex2_approx(fmaf(x[c + 1], sl2, -m_run)) : 0.f;
-            rs += p0 + p1;
-            x[c / 2] = __uint_as_float(pack_bf16x2(p0, p1));
-          }
-        }
-        ell += rs;
-        // P of this half over the S columns already read; the previous P of
-        // these columns was consumed before this S was computed
-        tmem_st32(tS + 64 * h, x);
-        tc_wait_st();
-        tc_fence_before();
-        mbar_arrive(bar(kBarPFull + 2 * h + qi));
       }
+      // P = exp2(S - m) as bf16 pairs, packed in place into x[0 .. 31]
+      float rs;
+      if (full) {
+        const uint64_t s2 = f2_pack(sl2, sl2), nm2 = f2_pack(-m_run, -m_run);
+        uint64_t rs2 = 0;
+#pragma unroll
+        for (int k = 0; k < kBk; k += 2) {
+          const uint64_t v = f2_fma(f2_pack(x[k], x[k + 1]), s2, nm2);
+          const float p0 = ex2_approx(f2_lo(v)), p1 = ex2_approx(f2_hi(v));
+          rs2 = f2_add(rs2, f2_pack(p0, p1));
+          x[k / 2] = __uint_as_float(pack_bf16x2(p0, p1));
+        }
+        rs = f2_lo(rs2) + f2_hi(rs2);
+      } else {
+        rs = 0.f;
+#pragma unroll
+        for (int k = 0; k < kBk; k += 2) {
+          const float p0 = (k <= lim) ? ex2_approx(fmaf(x[k], sl2, -m_run)) : 0.f;
+          const float p1 = (k + 1 <= lim) ? ex2_approx(fmaf(x[k + 1], sl2, -m_run)) : 0.f;
+          rs += p0 + p1;
+          x[k / 2] = __uint_as_float(pack_bf16x2(p0, p1));
+        }
+      }
+      ell += rs;
+      // P buffer c & 1 was last read by chunk c - 2's P V
+      if (c >= 2) {
+        if (!warp_wait(bar(kBarODone + 2 * qi + (c & 1)), (uint32_t)(((c - 2) >> 1) & 1))) { ok = false; break; }
+        tc_fence_after();
+      }
+      tmem_st32(tmem + col_p(qi, c & 1) + lane_base, x);
+      tc_wait_st();
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(bar(kBarPFull + 2 * qi + (c & 1)));
     }
-    if (ok) ok = warp_wait(bar(kBarODone + 2 + qi), (uint32_t)((ntiles - 1) & 1));
+    if (ok && nch > 0)
+      ok = warp_wait(bar(kBarODone + 2 * qi + ((nch - 1) & 1)), (uint32_t)(((nch - 1) >> 1) & 1));
     if (!ok) {
       if (lane == 0) set_error(kErrTimeout);
     } else {
