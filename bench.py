@@ -203,6 +203,9 @@ def main():
     ap.add_argument("--impl", default="s2o", choices=["s2o", "reference"])
     ap.add_argument("--e2e-steps", type=int, default=3)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--plan", default="filtered", choices=["full", "filtered"],
+                    help="s2o_plan (every segment fully ordered) or s2o_plan_filtered (only the prefix the "
+                         "stop rule can reach; same kept sets and output)")
     args = ap.parse_args()
     if args.warmup < 3 and args.impl == "s2o":
         ap.error("--warmup must be >= 3")
@@ -237,8 +240,10 @@ def main():
     O = torch.empty(Q.shape, dtype=torch.bfloat16, device=dev)
     stream = torch.cuda.current_stream(dev)
 
+    filtered = args.plan == "filtered"
+
     def step():
-        s2o.plan(cfg, Q, K, bufs)
+        s2o.plan(cfg, Q, K, bufs, filtered=filtered)
         s2o.attention(cfg, Q, K, V, bufs["perm"], bufs["nblocks"], O)
 
     for _ in range(args.warmup):
@@ -258,7 +263,7 @@ def main():
         t_start.record(stream)
         for k in range(args.steps):
             ev[k][0].record(stream)
-            s2o.plan(cfg, Q, K, bufs)
+            s2o.plan(cfg, Q, K, bufs, filtered=filtered)
             launches += s2o.last_launch_count()
             ev[k][1].record(stream)
             s2o.attention(cfg, Q, K, V, bufs["perm"], bufs["nblocks"], O)
@@ -275,6 +280,16 @@ def main():
     st = s2o.last_device_error()
     if st != 0:
         raise RuntimeError(f"device error in the timed region: {s2o.status_string(st)}")
+
+    # the other plan entry point, timed alone for the report (same inputs)
+    other = [[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in range(3)]
+    for e0, e1 in other:
+        e0.record(stream)
+        s2o.plan(cfg, Q, K, bufs, filtered=not filtered)
+        e1.record(stream)
+    torch.cuda.synchronize()
+    other_ms = float(np.median([e0.elapsed_time(e1) for e0, e1 in other]))
+    s2o.plan(cfg, Q, K, bufs, filtered=filtered)
 
     nb = bufs["nblocks"].cpu().numpy().reshape(w.B, w.Hkv, -1)
     G = w.Hq // w.Hkv
@@ -339,8 +354,9 @@ def main():
             "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
             "config": {"workload": w.name, "B": w.B, "Hq": w.Hq, "Hkv": w.Hkv, "N": w.N, "d": w.d, "tau": w.tau,
                        "global_batch": w.B * world, "seq_len": w.N, "parallelism": f"independent x{world}",
-                       "l2": "inputs larger than L2 (Q alone is 1 GiB)"},
+                       "l2": "inputs larger than L2 (Q alone is 1 GiB)", "plan": args.plan},
             "plan_ms": float(np.mean(plan_ms)), "attention_ms": attn_mean,
+            "plan_other": {"kind": "full" if filtered else "filtered", "ms": other_ms},
             "attention_only_tflops": whole_job_tflops(world, dense, attn_mean),
             "kept_pair_fraction": density,
             "roofline": roofline, "cpu_baseline": cpu, "e2e": e2e, "gpu_launches": launches,

@@ -136,6 +136,25 @@ s2o_status s2o_plan(const s2o_config* cfg, const uint16_t* Q, const uint16_t* K,
                     void* workspace, size_t workspace_bytes, s2o_stream_t stream);
 
 /*
+ * s2o_plan_filtered -- s2o_plan that sorts only the part of each segment's
+ * order the stop rule can reach (the pages describe the preprocessing as very
+ * light: pith.science abstract; gist.science technical summary, "Resultats
+ * Experimentaux").  A candidate of pooled mass exp(s - M)/Z below tau/Bk
+ * cannot lift a block to tau, so with n_hi candidates at or above that level
+ * the block starting at Bk*ceil(n_hi/Bk) fails the test and C(s) can be no
+ * larger; the rest of the segment is never ordered.
+ *   Arguments, layouts, workspace size and errors: as s2o_plan.
+ *   Results: scores, seg_stats and nblocks equal s2o_plan's; perm equals
+ *   s2o_plan's on the first Bk * nblocks[b,kvh,s] entries of every segment
+ *   (all that s2o_attention reads); later entries of a segment are
+ *   unspecified (they may hold anything, including stale data).
+ *   With tau = 0 every candidate counts and the result is s2o_plan's.
+ */
+s2o_status s2o_plan_filtered(const s2o_config* cfg, const uint16_t* Q, const uint16_t* K,
+                             float* scores, int32_t* perm, int32_t* nblocks, float* seg_stats,
+                             void* workspace, size_t workspace_bytes, s2o_stream_t stream);
+
+/*
  * s2o_plan_noalloc -- s2o_plan without a caller-supplied workspace, for
  * callers that may not allocate device memory: plugins inside an engine or
  * framework that owns all device memory through its own pool (a cudaMalloc of
@@ -198,7 +217,9 @@ s2o_status s2o_prefill_arena_size(const s2o_config* cfg, int32_t out_dtype, size
 
 /*
  * s2o_prefill_host -- the whole path from HOST buffers: copies Q, K, V to
- * the device arena, plans, runs the attention and copies O back to host O.
+ * the device arena, plans (s2o_plan_filtered: it returns no perm, and O and
+ * C(s) equal those of s2o_plan), runs the attention and copies O back to
+ * host O.
  * Host buffers should be page-locked for full copy speed.  The arena is
  * caller-allocated device memory of s2o_prefill_arena_size() bytes, 256-byte
  * aligned.  Synchronises the stream before returning and reports device

@@ -63,6 +63,7 @@ def lib() -> ctypes.CDLL:
         L.s2o_candidate_offset.restype = ctypes.c_int64
         L.s2o_plan_workspace_size.argtypes = [_CFG, ctypes.POINTER(ctypes.c_size_t)]
         L.s2o_plan.argtypes = [_CFG, _P, _P, _P, _P, _P, _P, _P, ctypes.c_size_t, _P]
+        L.s2o_plan_filtered.argtypes = [_CFG, _P, _P, _P, _P, _P, _P, _P, ctypes.c_size_t, _P]
         L.s2o_plan_noalloc.argtypes = [_CFG, _P, _P, _P, _P, _P, _P, _P]
         L.s2o_plan_contiguous.argtypes = [_CFG, _P, _P, _P, _P, _P]
         L.s2o_attention.argtypes = [_CFG, _P, _P, _P, _P, _P, _P, ctypes.c_int32, _P]
@@ -72,7 +73,7 @@ def lib() -> ctypes.CDLL:
         L.s2o_status_string.restype = ctypes.c_char_p
         L.s2o_last_device_error.argtypes = [_P]
         L.s2o_last_launch_count.restype = ctypes.c_int32
-        for name in ("s2o_plan_workspace_size", "s2o_plan", "s2o_plan_noalloc", "s2o_plan_contiguous", "s2o_attention",
+        for name in ("s2o_plan_workspace_size", "s2o_plan", "s2o_plan_filtered", "s2o_plan_noalloc", "s2o_plan_contiguous", "s2o_attention",
                      "s2o_prefill_arena_size", "s2o_prefill_host", "s2o_last_device_error"):
             getattr(L, name).restype = ctypes.c_int
         _lib = L
@@ -141,13 +142,14 @@ def alloc_plan(cfg: Config, device="cuda", workspace=True):
     return out
 
 
-def plan(cfg: Config, Q, K, bufs=None, stream=None):
-    """Run s2o_plan; returns the buffer dict (scores, perm, nblocks, seg_stats)."""
+def plan(cfg: Config, Q, K, bufs=None, stream=None, filtered: bool = False):
+    """Run s2o_plan (or s2o_plan_filtered); returns the buffer dict (scores,
+    perm, nblocks, seg_stats)."""
     bufs = alloc_plan(cfg, Q.device) if bufs is None else bufs
     ws = bufs["workspace"]
-    _check(lib().s2o_plan(ctypes.byref(cfg), _ptr(Q), _ptr(K), _ptr(bufs["scores"]), _ptr(bufs["perm"]),
-                          _ptr(bufs["nblocks"]), _ptr(bufs.get("seg_stats")), _ptr(ws), ws.numel(),
-                          _stream(stream)), "s2o_plan")
+    fn, name = (lib().s2o_plan_filtered, "s2o_plan_filtered") if filtered else (lib().s2o_plan, "s2o_plan")
+    _check(fn(ctypes.byref(cfg), _ptr(Q), _ptr(K), _ptr(bufs["scores"]), _ptr(bufs["perm"]),
+              _ptr(bufs["nblocks"]), _ptr(bufs.get("seg_stats")), _ptr(ws), ws.numel(), _stream(stream)), name)
     return bufs
 
 

@@ -54,6 +54,7 @@ struct PlanWs {
   float* sorted;
   BucketSlot* slots;
   int* mode;
+  int* plen;
   float2* range;
   int64_t nslots;
   size_t bytes;
@@ -82,6 +83,7 @@ PlanWs plan_layout(const s2o_config* c, void* base) {
   w.nslots = per_bk * (int64_t)BH;
   w.slots = static_cast<BucketSlot*>(take((size_t)w.nslots * sizeof(BucketSlot) + 16));
   w.mode = static_cast<int*>(take(BH * S * sizeof(int)));
+  w.plen = static_cast<int*>(take(BH * S * sizeof(int)));
   w.range = static_cast<float2*>(take(BH * S * sizeof(float2)));
   w.bytes = off;
   return w;
@@ -175,9 +177,11 @@ s2o_status s2o_plan_workspace_size(const s2o_config* cfg, size_t* bytes) {
   return S2O_OK;
 }
 
-s2o_status s2o_plan(const s2o_config* cfg, const uint16_t* Q, const uint16_t* K, float* scores, int32_t* perm,
+// the plan's launches; `filtered` sorts only the prefix of each segment's
+// order that the stop rule can reach
+static s2o_status run_plan(const s2o_config* cfg, const uint16_t* Q, const uint16_t* K, float* scores, int32_t* perm,
                     int32_t* nblocks, float* seg_stats, void* workspace, size_t workspace_bytes,
-                    s2o_stream_t stream) {
+                    s2o_stream_t stream, int filtered) {
   t_launches = 0;
   s2o_status st = check_cfg(cfg);
   if (st != S2O_OK) return st;
@@ -203,7 +207,7 @@ s2o_status s2o_plan(const s2o_config* cfg, const uint16_t* Q, const uint16_t* K,
   k_seg_stats<<<(nwarps * 32 + 255) / 256, 256, 0, s>>>(w.part, w.segM, w.segZ, seg_stats, BH, S);
   ++t_launches;
   k_bucket_plan<<<BH * S, kBucketThreads, 0, s>>>(scores, w.sorted, perm, w.slots, w.mode, w.range, w.keyB, w.valB,
-                                                   BH, S, T);
+                                                   w.segM, w.segZ, w.plen, cfg->tau, filtered, BH, S, T);
   ++t_launches;
   if (w.nslots > 0) {
     k_bucket_sort<<<(unsigned)w.nslots, kSorterThreads, kBucketSmem, s>>>(w.keyB, w.valB, w.slots, w.sorted, perm,
@@ -213,9 +217,21 @@ s2o_status s2o_plan(const s2o_config* cfg, const uint16_t* Q, const uint16_t* K,
   k_sort<<<BH * S, kSortThreads, 0, s>>>(scores, w.segM, w.segZ, w.keyA, w.keyB, w.valA, w.valB, perm, w.sorted,
                                          w.mode, kModeFallback, BH, S, T);
   ++t_launches;
-  k_mass_stop<<<BH * S, 256, 0, s>>>(w.sorted, w.segM, w.segZ, nblocks, BH, S, T, cfg->tau);
+  k_mass_stop<<<BH * S, 256, 0, s>>>(w.sorted, w.segM, w.segZ, w.plen, nblocks, BH, S, T, cfg->tau);
   ++t_launches;
   return launch_status();
+}
+
+s2o_status s2o_plan(const s2o_config* cfg, const uint16_t* Q, const uint16_t* K, float* scores, int32_t* perm,
+                    int32_t* nblocks, float* seg_stats, void* workspace, size_t workspace_bytes,
+                    s2o_stream_t stream) {
+  return run_plan(cfg, Q, K, scores, perm, nblocks, seg_stats, workspace, workspace_bytes, stream, 0);
+}
+
+s2o_status s2o_plan_filtered(const s2o_config* cfg, const uint16_t* Q, const uint16_t* K, float* scores,
+                             int32_t* perm, int32_t* nblocks, float* seg_stats, void* workspace,
+                             size_t workspace_bytes, s2o_stream_t stream) {
+  return run_plan(cfg, Q, K, scores, perm, nblocks, seg_stats, workspace, workspace_bytes, stream, 1);
 }
 
 s2o_status s2o_plan_contiguous(const s2o_config* cfg, const float* scores, const float* seg_stats,
@@ -322,7 +338,7 @@ s2o_status s2o_prefill_host(const s2o_config* cfg, const uint16_t* Q_host, const
       cudaMemcpyAsync(dK, K_host, kv * 2, cudaMemcpyHostToDevice, s) != cudaSuccess ||
       cudaMemcpyAsync(dV, V_host, kv * 2, cudaMemcpyHostToDevice, s) != cudaSuccess)
     return S2O_ERR_CUDA;
-  st = s2o_plan(cfg, dQ, dK, dscores, dperm, dnb, nullptr, ws, wsb, stream);
+  st = run_plan(cfg, dQ, dK, dscores, dperm, dnb, nullptr, ws, wsb, stream, 1);
   if (st != S2O_OK) return st;
   const int32_t n_plan = t_launches;
   st = s2o_attention(cfg, dQ, dK, dV, dperm, dnb, dO, out_dtype, stream);

@@ -20,6 +20,16 @@
 //                  instead; writes perm and the sorted scores at the bucket's
 //                  global rank;
 //   k_mass_stop    block masses of the sorted scores and the stop point C(s).
+// Filtered form (the planner's `filtered` flag): a candidate of pooled mass
+// exp(s - M)/Z below tau/Bk cannot lift a block to tau, so a block made only
+// of such candidates fails the stop test.  With n_hi candidates at or above
+// that level (counted with a small safety margin), the first block starting
+// at or after n_hi fails, hence C(s) <= ceil(n_hi/Bk), and only the first
+// L = Bk ceil(n_hi/Bk) entries of the order are needed.  The planner then
+// buckets and moves only the score bins that start below rank L; the rest of
+// the segment is never sorted.  perm[0, Bk C) and C are those of the full
+// sort (the pith.science abstract calls the preprocessing very light; this
+// keeps its cost proportional to what the stop rule can keep).
 // A segment whose scores are all equal is already in index order.  A segment
 // with a bin larger than kBucketCap - kBucketHalf (a heavy cluster of nearly
 // equal scores) is sorted by the global-memory LSD kernel k_sort instead.
@@ -91,8 +101,11 @@ __global__ void __launch_bounds__(kBucketThreads) k_bucket_plan(const float* __r
                                                               BucketSlot* __restrict__ slots, int* __restrict__ mode,
                                                               float2* __restrict__ range,
                                                               uint32_t* __restrict__ stage_key,
-                                                              uint32_t* __restrict__ stage_val, int BHkv, int S,
-                                                              int64_t T) {
+                                                              uint32_t* __restrict__ stage_val,
+                                                              const float* __restrict__ segM,
+                                                              const double* __restrict__ segZ,
+                                                              int* __restrict__ plen, double tau, int filtered,
+                                                              int BHkv, int S, int64_t T) {
   __shared__ int hist[kNumBins];
   __shared__ int wtot[33];
   __shared__ float red[64];
@@ -100,6 +113,7 @@ __global__ void __launch_bounds__(kBucketThreads) k_bucket_plan(const float* __r
   __shared__ uint8_t bin2bkt[kNumBins];  // bucket id of each bin (< kMaxBuckets = 256)
   __shared__ uint16_t wcnt[kSortWarps][kMaxBuckets];
   __shared__ int cursor[kMaxBuckets];
+  __shared__ int bin_cut;  // first bin left out of the order (filtered form)
   const int q = blockIdx.x;
   const int s = S - 1 - q / BHkv;
   const int bk = q % BHkv;
@@ -116,17 +130,25 @@ __global__ void __launch_bounds__(kBucketThreads) k_bucket_plan(const float* __r
   const int my_slots = bucket_slots(n);
   BucketSlot* myslot = slots + (size_t)tot_before * BHkv + (size_t)bk * my_slots;
   for (int k = tid; k < my_slots; k += kBucketThreads) myslot[k].count = 0;
+  if (tid == 0) plen[(size_t)bk * S + s] = n;
   if (n == 0) {
     if (tid == 0) mode[(size_t)bk * S + s] = kModeDone;
     return;
   }
 
-  // min and max candidate score
+  // min and max candidate score; the number of candidates whose pooled mass
+  // may reach tau/Bk: s >= M + ln(tau Z / Bk), less a margin of 1e-3 that
+  // covers the rounding of the masses computed in k_mass_stop
+  double cut = -INFINITY;
+  if (filtered && tau > 0.0)
+    cut = (double)segM[(size_t)bk * S + s] + log(tau * segZ[(size_t)bk * S + s] / (double)kBk) - 1e-3;
   float lo = INFINITY, hi = -INFINITY;
+  int nhi = 0;
   for (int i = tid; i < n; i += kBucketThreads) {
     const float x = sc[i];
     lo = fminf(lo, x);
     hi = fmaxf(hi, x);
+    nhi += (double)x >= cut;
   }
 #pragma unroll
   for (int o = 16; o >= 1; o >>= 1) {
@@ -135,6 +157,10 @@ __global__ void __launch_bounds__(kBucketThreads) k_bucket_plan(const float* __r
   }
   if (lane == 0) { red[warp] = lo; red[32 + warp] = hi; }
   for (int k = tid; k < kNumBins; k += kBucketThreads) hist[k] = 0;
+  int nhi_tot;
+  block_excl_scan(nhi, wtot, nhi_tot);  // (synchronises the block)
+  // entries of the order the stop rule can reach: whole blocks up to n_hi
+  const int L = (int)min((int64_t)n, (int64_t)kBk * (((int64_t)nhi_tot + kBk - 1) / kBk));
   __syncthreads();
   if (warp == 0) {
     lo = red[lane];
@@ -176,20 +202,33 @@ __global__ void __launch_bounds__(kBucketThreads) k_bucket_plan(const float* __r
     if (tid == 0) mode[(size_t)bk * S + s] = kModeFallback;
     return;
   }
-  // a bucket = the bins whose start rank lies in [k*H, (k+1)*H); the thread
-  // of its first bin records the first bin and base rank, the thread of its
-  // last bin the end bin, then (after a barrier) the size
+  // bins that start at rank >= L are left out (none when L = n); start ranks
+  // grow with the bin, so they form a suffix
+  if (tid == 0) bin_cut = kNumBins;
+  __syncthreads();
+  if (st0 >= L && (tid == 0 || st0 - hist[2 * tid - 1] < L)) atomicMin(&bin_cut, 2 * tid);
+  else if (st1 >= L && st0 < L) atomicMin(&bin_cut, 2 * tid + 1);
+  __syncthreads();
+  const int bcut = bin_cut;
+  if (tid == 0) plen[(size_t)bk * S + s] = L;
+  // a bucket = the bins below bin_cut whose start rank lies in
+  // [k*H, (k+1)*H); the thread of its first bin records the first bin and
+  // base rank, the thread of its last bin the end bin, then (after a
+  // barrier) the size
   hist[2 * tid] = st0;
   hist[2 * tid + 1] = st1;
   __syncthreads();
-  int end_id = -1, end_rank = 0;
+  // both bins of a thread may end a bucket (a bin that is a bucket by itself,
+  // or the last bin before bin_cut), so each keeps its own record
+  int end_id[2] = {-1, -1}, end_rank[2] = {0, 0};
 #pragma unroll
   for (int e = 0; e < 2; ++e) {
     const int b = 2 * tid + e;
+    if (b >= bcut) break;
     const int stb = e ? st1 : st0;
     const int id = stb / kBucketHalf;
     const bool first = (b == 0) || (hist[b - 1] / kBucketHalf != id);
-    const bool last = (b == kNumBins - 1) || (hist[b + 1] / kBucketHalf != id);
+    const bool last = (b == kNumBins - 1) || (b + 1 == bcut) || (hist[b + 1] / kBucketHalf != id);
     if (first) {
       myslot[id].bk = bk;
       myslot[id].s = s;
@@ -198,12 +237,14 @@ __global__ void __launch_bounds__(kBucketThreads) k_bucket_plan(const float* __r
     }
     if (last) {
       myslot[id].bin_hi = b + 1;
-      end_id = id;
-      end_rank = stb + (e ? c1 : c0);
+      end_id[e] = id;
+      end_rank[e] = stb + (e ? c1 : c0);
     }
   }
   __syncthreads();
-  if (end_id >= 0) myslot[end_id].count = end_rank - myslot[end_id].base;
+#pragma unroll
+  for (int e = 0; e < 2; ++e)
+    if (end_id[e] >= 0) myslot[end_id[e]].count = end_rank[e] - myslot[end_id[e]].base;
   // stable multisplit into the buckets, 1024 elements per step in index order
   bin2bkt[2 * tid] = (uint8_t)(st0 / kBucketHalf);
   bin2bkt[2 * tid + 1] = (uint8_t)(st1 / kBucketHalf);
@@ -213,7 +254,7 @@ __global__ void __launch_bounds__(kBucketThreads) k_bucket_plan(const float* __r
   for (int e = 0; e < 2; ++e) {
     const int b = 2 * tid + e;
     const int id = bin2bkt[b];
-    if (b == 0 || bin2bkt[b - 1] != id) cursor[id] = e ? st1 : st0;
+    if (b < bcut && (b == 0 || bin2bkt[b - 1] != id)) cursor[id] = e ? st1 : st0;
   }
   __syncthreads();
   const uint32_t lt_mask = (1u << lane) - 1u;
@@ -221,9 +262,10 @@ __global__ void __launch_bounds__(kBucketThreads) k_bucket_plan(const float* __r
   uint32_t* sval = stage_val + base;
   for (int t0 = 0; t0 < n; t0 += kBucketThreads) {
     const int i = t0 + tid;
-    const bool valid = i < n;
-    const float x = valid ? sc[i] : 0.f;
-    const uint32_t d = valid ? bin2bkt[score_bin(x, hi, scale)] : 0u;
+    const float x = i < n ? sc[i] : 0.f;
+    const int bin = score_bin(x, hi, scale);
+    const bool valid = i < n && bin < bcut;
+    const uint32_t d = valid ? bin2bkt[bin] : 0u;
     for (int k = lane; k < kMaxBuckets; k += 32) wcnt[warp][k] = 0;
     __syncwarp();
     const uint32_t peers = __match_any_sync(0xffffffffu, valid ? d : 1024u + lane);
@@ -450,16 +492,19 @@ write_out:
 // ---------------------------------------------------------------------------
 // block masses of the sorted scores and the stop point: one CTA per segment
 // ---------------------------------------------------------------------------
+// Blocks past plen[(b,kvh,s)] / Bk are not evaluated: the planner proved the
+// block starting there fails the test (it is the stop point if no earlier
+// block fails).
 __global__ void __launch_bounds__(256) k_mass_stop(const float* __restrict__ sorted, const float* __restrict__ segM,
-                                                  const double* __restrict__ segZ, int32_t* __restrict__ nblocks,
-                                                  int BHkv, int S, int64_t T, double tau) {
+                                                  const double* __restrict__ segZ, const int* __restrict__ plen,
+                                                  int32_t* __restrict__ nblocks, int BHkv, int S, int64_t T,
+                                                  double tau) {
   __shared__ int cmin;
   const int q = blockIdx.x;
   const int s = S - 1 - q / BHkv;
   const int bk = q % BHkv;
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-  const int n = (int)num_cand(s);
-  const int nb = n / kBk;
+  const int nb = min((int)(num_cand(s) / kBk), plen[(size_t)bk * S + s] / kBk);
   if (threadIdx.x == 0) cmin = nb;
   __syncthreads();
   const float* ss = sorted + (size_t)bk * T + cand_offset(s);

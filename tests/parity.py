@@ -28,21 +28,34 @@ def log_near_ties(record: dict):
             f.write(json.dumps(record) + "\n")
 
 
-def compare_segment_plan(gpu_perm: np.ndarray, gpu_C: int, sp: O.SegmentPlan, p: O.Params, full_list=True):
-    """Returns (swapped_positions, C_flip); raises AssertionError on a real mismatch."""
+def compare_segment_plan(gpu_perm: np.ndarray, gpu_C: int, sp: O.SegmentPlan, p: O.Params, full_list=True,
+                         prefix_only=False):
+    """Returns (swapped_positions, C_flip); raises AssertionError on a real mismatch.
+
+    prefix_only: only the first Bk * gpu_C entries are defined (the filtered
+    plan); they must be distinct members of Cand(s) and match the oracle's.
+    """
     n = len(sp.order)
     gpu_perm = np.asarray(gpu_perm, dtype=np.int64)
     assert len(gpu_perm) == n
     if n:
         lo = int(sp.order.min())
-        assert np.array_equal(np.sort(gpu_perm), np.arange(lo, lo + n)), "perm is not a permutation of Cand(s)"
+        if prefix_only:
+            head = gpu_perm[:min(n, p.Bk * gpu_C)]
+            assert np.all((head >= lo) & (head < lo + n)), "perm prefix leaves Cand(s)"
+            assert len(np.unique(head)) == len(head), "perm prefix repeats a key"
+        else:
+            assert np.array_equal(np.sort(gpu_perm), np.arange(lo, lo + n)), "perm is not a permutation of Cand(s)"
     # near-tie runs of the oracle order
     run = np.zeros(n, dtype=np.int64)
     if n > 1:
         brk = np.ones(n - 1, dtype=bool)
         brk[sp.score_ties] = False
         run[1:] = np.cumsum(brk)
-    span = n if full_list else min(n, p.Bk * max(gpu_C, sp.C) + p.Bk)
+    if prefix_only:
+        span = min(n, p.Bk * gpu_C)
+    else:
+        span = n if full_list else min(n, p.Bk * max(gpu_C, sp.C) + p.Bk)
     swapped = 0
     if n:
         pos = np.empty(n, dtype=np.int64)

@@ -45,7 +45,7 @@ def host_plan(cfg, bufs):
     return perm, nb, scores, stats
 
 
-def check_plan(Q, K, cfg, bufs, p, segments=None, kvheads=None, what=""):
+def check_plan(Q, K, cfg, bufs, p, segments=None, kvheads=None, what="", prefix_only=False):
     perm, nb, scores, stats = host_plan(cfg, bufs)
     G = cfg.Hq // cfg.Hkv
     off = O.candidate_offsets(cfg.N, p)
@@ -66,7 +66,8 @@ def check_plan(Q, K, cfg, bufs, p, segments=None, kvheads=None, what=""):
             assert np.all(np.abs(gs - ref) <= half_ulp + 1e-13 * np.abs(ref) + 1e-300)
             assert abs(stats[b, kvh, s, 0] - sp.M) <= 0.5 * float(np.spacing(np.float32(abs(sp.M)))) + 1e-13 * abs(sp.M)
             assert abs(stats[b, kvh, s, 1] / sp.Z - 1.0) <= 1e-5
-            sw, fl = parity.compare_segment_plan(perm[b, kvh, off[s]:off[s + 1]], int(nb[b, kvh, s]), sp, p)
+            sw, fl = parity.compare_segment_plan(perm[b, kvh, off[s]:off[s + 1]], int(nb[b, kvh, s]), sp, p,
+                                                 prefix_only=prefix_only)
             swaps += sw
             flips += fl
     parity.log_near_ties({"case": what, "tau": p.tau, "segments": len(segs) * len(heads),
@@ -261,3 +262,70 @@ def test_sweep_64k_tau_and_contiguous():
                                                                O.candidate_range(w.N, s, p)[1]))
             outc = s2o.attention(cfg, q, k, v, pc, bufs["nblocks"])
             check_output(Q, K, V, cfg, pch, nb, outc, p, segments=segs, kvheads=[5], what=f"contig tau={tau}")
+
+
+# ---------------------------------------------------------------------------
+# s2o_plan_filtered: only the prefix of each order the stop rule can reach
+# ---------------------------------------------------------------------------
+
+def filtered_matches_full(cfg, q, k, v):
+    """Runs both plans and both attentions; the filtered plan's perm buffer
+    starts filled with -1, so an attention that read past a segment's kept
+    prefix would raise the bad-plan error."""
+    full = s2o.plan(cfg, q, k)
+    filt = s2o.alloc_plan(cfg, q.device)
+    filt["perm"].fill_(-1)
+    s2o.plan(cfg, q, k, bufs=filt, filtered=True)
+    assert s2o.last_launch_count() >= 6
+    assert s2o.last_device_error() == 0
+    BH = cfg.B * cfg.Hkv
+    S, T = s2o.num_segments(cfg), s2o.num_candidates(cfg)
+    assert torch.equal(filt["nblocks"], full["nblocks"])
+    assert torch.equal(filt["scores"][:BH * T], full["scores"][:BH * T])
+    assert torch.equal(filt["seg_stats"], full["seg_stats"])
+    # positions inside each segment's kept prefix, compared on the device
+    nb = full["nblocks"].view(BH, S).long()
+    off = torch.tensor([s2o.candidate_offset(cfg, s) for s in range(S + 1)], dtype=torch.int64, device=q.device)
+    pos = torch.arange(T, dtype=torch.int64, device=q.device)
+    seg = torch.searchsorted(off, pos, right=True) - 1
+    inside = (pos - off[seg]).unsqueeze(0) < 64 * nb[:, seg]
+    pf = filt["perm"][:BH * T].view(BH, T)
+    pa = full["perm"][:BH * T].view(BH, T)
+    assert torch.equal(pf[inside], pa[inside])
+    kept = float(inside.float().mean()) if T else 0.0
+    del inside, pos, seg
+    out_a = s2o.attention(cfg, q, k, v, full["perm"], full["nblocks"])
+    out_f = s2o.attention(cfg, q, k, v, filt["perm"], filt["nblocks"])
+    assert s2o.last_device_error() == 0
+    assert torch.equal(out_a, out_f)
+    return filt, kept
+
+
+@pytest.mark.parametrize("B,Hq,Hkv,N,tau,planted,band", SMALL)
+def test_filtered_plan_small_cases(B, Hq, Hkv, N, tau, planted, band):
+    Q, K, V = synth.generate(B, Hq, Hkv, N, 128, planted=planted, band=band, n_stripe=8, seed=3)
+    cfg = s2o.make_config(B, Hq, Hkv, N, tau=tau)
+    filt, _ = filtered_matches_full(cfg, dev(Q), dev(K), dev(V))
+    check_plan(Q, K, cfg, filt, O.Params(tau=tau), what="filtered small", prefix_only=True)
+
+
+@pytest.mark.parametrize("name", ["tiny_1k", "llama_16k", "llama_128k", "flat_128k"])
+def test_filtered_plan_workloads(name):
+    w = synth.WORKLOADS[name]
+    Q, K, V = synth.generate_workload(w)
+    cfg = s2o.make_config(w.B, w.Hq, w.Hkv, w.N, tau=w.tau)
+    filt, kept = filtered_matches_full(cfg, dev(Q), dev(K), dev(V))
+    p = O.Params(tau=w.tau)
+    S = O.num_segments(w.N, p)
+    segs = None if S <= 8 else sampled_segments(S)
+    check_plan(Q, K, cfg, filt, p, segments=segs, kvheads=[0, w.Hkv - 1], what=f"filtered {name}",
+               prefix_only=True)
+
+
+def test_filtered_plan_tau_sweep():
+    w = synth.WORKLOADS["sweep_64k"]
+    Q, K, V = synth.generate_workload(w)
+    q, k, v = dev(Q), dev(K), dev(V)
+    for tau in synth.TAU_SWEEP:
+        cfg = s2o.make_config(w.B, w.Hq, w.Hkv, w.N, tau=tau)
+        filtered_matches_full(cfg, q, k, v)

@@ -368,3 +368,43 @@ def test_kept_pairs_dense_closed_form():
         keep = np.arange(O.admissible_end(N, s, p))
         total += O.kept_pairs_segment(N, s, keep, p)
     assert total == N * (N + 1) // 2
+
+
+# ---------------------------------------------------------------------------
+# the bound behind the filtered plan
+# ---------------------------------------------------------------------------
+
+@pytest.mark.parametrize("tau", [1e-4, 1e-3, 3e-3, 1e-2, 5e-2])
+def test_stop_point_within_threshold_prefix(tau):
+    # A block is a sum of Bk masses; if all of them are below tau/Bk it is
+    # below tau.  So the stop point can be no later than the first block that
+    # starts at or after n_hi = #{candidates with mass >= tau/Bk}, and the
+    # first Bk*ceil(n_hi/Bk) entries of the order decide C.  The masses here
+    # are recomputed from the scores, not taken from the oracle's blocks.
+    p = O.Params(tau=tau)
+    seen_bound = False
+    for seed in (1, 2):
+        Q, K, V = _random_case(seed, N=4096)
+        N = Q.shape[2]
+        res = O.plan(Q, K, p)
+        for s in range(O.num_segments(N, p)):
+            sp = res["plans"][(0, 0, s)]
+            lo, hi = O.candidate_range(N, s, p)
+            if hi <= lo:
+                continue
+            w = np.exp(sp.scores[lo:hi] - sp.M) / sp.Z
+            n_hi = int(np.count_nonzero(w >= tau / p.Bk))
+            bound = -(-n_hi // p.Bk)
+            assert sp.C <= bound
+            # the same C from the prefix alone
+            L = min(hi - lo, p.Bk * bound)
+            head = np.exp(sp.scores[sp.order[:L]] - sp.M) / sp.Z
+            C2 = bound
+            for k in range(L // p.Bk):
+                if head[k * p.Bk:(k + 1) * p.Bk].sum() < tau:
+                    C2 = k
+                    break
+            assert C2 == sp.C
+            seen_bound |= bound < O.num_blocks(hi - lo, p)
+    # at these sizes the bound cuts the order for the larger thresholds
+    assert seen_bound or tau < 3e-3
