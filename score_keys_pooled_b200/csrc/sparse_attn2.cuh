@@ -59,7 +59,8 @@ constexpr uint32_t kOff2Q = 0;                       // Q0, Q1
 constexpr uint32_t kOff2K = 2 * kTile2Bytes;         // K stages
 constexpr uint32_t kOff2V = kOff2K + kStagesK * kTile2Bytes;
 constexpr uint32_t kOff2Bar = kOff2V + kStagesV * kTile2Bytes;
-constexpr uint32_t kAttn2SmemData = kOff2Bar + 256;
+constexpr uint32_t kOff2Keys = kOff2Bar + 256;         // per loader warp: keys of its tile rows, by row parity
+constexpr uint32_t kAttn2SmemData = kOff2Keys + 2 * 512;
 constexpr size_t kAttn2Smem = kAttn2SmemData + 1024;  // + alignment slack
 constexpr uint32_t kTmem2Cols = 512;
 
@@ -254,53 +255,93 @@ __global__ void __launch_bounds__(kAttn2Threads, 1)
     }
     const int32_t* pseg = a.perm + (size_t)bk * a.T + cand_offset(s);
     const int cand_hi = kLq * s - kWin;
-    // keys of tile rows 4 lane .. 4 lane + 3 (-1: a zero row, for an empty
-    // half or a key past N)
-    auto tile_keys = [&](int t, int* y) {
+    // raw key indices of tile rows 4 lane .. 4 lane + 3 (loaded, not yet used)
+    auto fetch_keys = [&](int t, int* y) {
       int j0;
       const int kind = walk2_block(wk, s, 2 * t + (lane >> 4), j0);
+      const int rr = (4 * lane) & 63;
+      if (kind == 2) {
+        const int4 v = *reinterpret_cast<const int4*>(pseg + kBk * j0 + rr);
+        y[0] = v.x; y[1] = v.y; y[2] = v.z; y[3] = v.w;
+      } else {
+#pragma unroll
+        for (int k = 0; k < 4; ++k) y[k] = kind == 3 ? -1 : j0 + rr + k;
+      }
+    };
+    // checked keys (-1: a zero row: an empty half or a key past N) into the
+    // warp's table: row r = 2 jj + p at keys[p][jj]; true if any is -1
+    int32_t* keys = reinterpret_cast<int32_t*>(sgen + kOff2Keys + (is_k ? 0 : 512));
+    const uint32_t keys_s = sbase + kOff2Keys + (is_k ? 0u : 512u);
+    auto stage_keys = [&](int t, const int* y) {
+      int j0;
+      const int kind = walk2_block(wk, s, 2 * t + (lane >> 4), j0);
+      int k4[4];
 #pragma unroll
       for (int k = 0; k < 4; ++k) {
-        const int rr = (4 * lane + k) & 63;
-        int j = -1;
+        int j = y[k];
         if (kind == 2) {
-          j = pseg[kBk * j0 + rr];
           if (j < kSink || j >= cand_hi) {  // caller-supplied plan out of Cand(s)
             set_error(kErrBadPlan);
             j = kSink;
           }
-        } else if (kind != 3) {
-          j = j0 + rr;
-          if (j >= a.N) j = -1;
+        } else if (j >= a.N) {
+          j = -1;
         }
-        y[k] = j;
+        k4[k] = j;
       }
+      // rows 4 lane + k: parity k & 1, slot 2 lane + (k >> 1)
+      *reinterpret_cast<int2*>(keys + 2 * lane) = make_int2(k4[0], k4[2]);
+      *reinterpret_cast<int2*>(keys + 64 + 2 * lane) = make_int2(k4[1], k4[3]);
+      __syncwarp();
+      return __any_sync(0xffffffffu, k4[0] < 0 || k4[1] < 0 || k4[2] < 0 || k4[3] < 0);
     };
-    // this lane's 16-byte chunk q of a row: swizzle atom q / 8, chunk q % 8
+    // this lane copies 16-byte chunk q of rows 2 jj + sel (swizzle atom q / 8,
+    // chunk q % 8 xor row % 8); its destination offsets repeat with jj % 4
     const int q = lane & 15, sel = lane >> 4;
-    const uint32_t lane_off = (uint32_t)(q >> 3) * (128 * 128);
+    uint32_t dsw[4];
+#pragma unroll
+    for (int m = 0; m < 4; ++m)
+      dsw[m] = (uint32_t)(q >> 3) * (128 * 128) + (uint32_t)sel * 128 +
+               ((uint32_t)((q & 7) ^ ((2 * m + sel) & 7)) << 4);
+    const char* src0 = reinterpret_cast<const char*>(kv) + 16 * q;
+    const uint32_t ktab = keys_s + 256u * (uint32_t)sel;
     int y[4];
-    if (ntiles > 0) tile_keys(0, y);
+    if (ntiles > 0) fetch_keys(0, y);
     for (int t = 0; t < ntiles; ++t) {
       const int st = t % nst;
       const int round = t / nst;
+      const bool ragged = stage_keys(t, y);
+      if (t + 1 < ntiles) fetch_keys(t + 1, y);  // in flight while this stage fills
       if (!warp_wait(bar(bar_empty + st), (uint32_t)((round & 1) ^ 1))) {
         if (lane == 0) set_error(kErrTimeout);
         break;
       }
-      const uint32_t dst0 = ring + st * kTile2Bytes + lane_off;
+      const uint32_t dst0 = ring + st * kTile2Bytes;
+      // 64 copies per lane; the key table is read four keys at a time.  A tile
+      // with a zero row (rare: an empty half or keys past N) takes the loop
+      // with per-row source sizes; the branch stays outside the unrolled loop
+      // so that each copy issues once.
+      if (!ragged) {
 #pragma unroll
-      for (int jj = 0; jj < 64; ++jj) {
-        // tile row r = 2 jj + sel; its key sits in lane r / 4, register r % 4
-        const int v0 = __shfl_sync(0xffffffffu, y[2 * (jj & 1)], jj >> 1);
-        const int v1 = __shfl_sync(0xffffffffu, y[2 * (jj & 1) + 1], jj >> 1);
-        const int key = sel ? v1 : v0;
-        const int r = 2 * jj + sel;
-        const uint32_t dst = dst0 + (uint32_t)r * 128 + ((uint32_t)((q & 7) ^ (r & 7)) << 4);
-        const uint16_t* src = kv + (size_t)(key < 0 ? 0 : key) * kD + 8 * q;
-        cp_async16(dst, src, key < 0 ? 0u : 16u);
+        for (int j4 = 0; j4 < 16; ++j4) {
+          int4 kk;
+          asm volatile("ld.shared.v4.s32 {%0, %1, %2, %3}, [%4];\n"
+                       : "=r"(kk.x), "=r"(kk.y), "=r"(kk.z), "=r"(kk.w)
+                       : "r"(ktab + 16u * (uint32_t)j4)
+                       : "memory");
+          const int key4[4] = {kk.x, kk.y, kk.z, kk.w};
+#pragma unroll
+          for (int m = 0; m < 4; ++m)
+            cp_async16(dst0 + dsw[m] + 256u * (uint32_t)(4 * j4 + m), src0 + (size_t)key4[m] * (kD * 2), 16u);
+        }
+      } else {
+#pragma unroll 4
+        for (int jj = 0; jj < 64; ++jj) {
+          const int key = keys[64 * sel + jj];
+          cp_async16(dst0 + dsw[jj & 3] + 256u * (uint32_t)jj, src0 + (size_t)(key < 0 ? 0 : key) * (kD * 2),
+                     key < 0 ? 0u : 16u);
+        }
       }
-      if (t + 1 < ntiles) tile_keys(t + 1, y);  // index loads overlap the copies
       cp_async_wait_all();
       fence_proxy_async_smem();  // generic-proxy writes -> tensor-core reads
       __syncwarp();
@@ -451,11 +492,9 @@ __global__ void __launch_bounds__(kAttn2Threads, 1)
         }
       }
       ell += rs;
-      // P buffer c & 1 was last read by chunk c - 2's P V
-      if (c >= 2) {
-        if (!warp_wait(bar(kBarODone + 2 * qi + (c & 1)), (uint32_t)(((c - 2) >> 1) & 1))) { ok = false; break; }
-        tc_fence_after();
-      }
+      // P buffer c & 1 was last read by chunk c - 2's P V, which this head's
+      // issuer committed before chunk c's Q K^T: the S-full barrier of chunk c
+      // (waited above) already covers it
       tmem_st32(tmem + col_p(qi, c & 1) + lane_base, x);
       tc_wait_st();
       tc_fence_before();
