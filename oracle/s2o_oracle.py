@@ -37,7 +37,14 @@ the following readings (the GPU library takes the same ones):
   * stop: C = index of the first block with m_b < tau (that block is not
     kept), or the number of blocks if none is below tau;
   * attention: every row i of the segment, for every head of the group, gets
-    exact softmax attention over Keep(s) intersected with [0, i].
+    exact softmax attention over Keep(s) intersected with [0, i];
+  * run-time stop (the pages' own rule, an alternative to the planned stop):
+    a tile (the segment's rows of a pair of query heads, or of one head when
+    the group size is odd) processes the always-kept keys, then candidate
+    blocks in the plan's order; after each block every row's gain is the
+    block's share of the exp-sum the row has processed so far (the block
+    included); the tile stops after the first block whose mean gain over its
+    rows is below tau, keeping that block.
 
 All arithmetic is IEEE fp64 on inputs widened exactly from bf16.  Loops are
 plain; numpy's matmul, sort and sum are used as library steps only.  The
@@ -333,6 +340,81 @@ def dense_attention(Qf, Kf, Vf, p: Params, segments=None):
                 r0, r1 = segment_rows(N, s, p)
                 O[b, kvh * G:(kvh + 1) * G, r0:r1] = dense_segment(Qf, Kf, Vf, b, kvh, s, G, p)
     return O
+
+
+# ---------------------------------------------------------------------------
+# Run-time (online) stop rule
+# ---------------------------------------------------------------------------
+
+NEAR_TIE_ONLINE_REL = 1e-4  # relative band around tau for the online block gains
+
+
+@dataclass
+class OnlineStop:
+    C: int                  # candidate blocks processed, the stopping block included
+    gains: np.ndarray       # mean relative gain of each processed candidate block
+    near_ties: np.ndarray   # processed blocks whose gain lies within the band of tau
+
+
+def online_stop_segment(Qf, Kf, b: int, kvh: int, s: int, heads, perm_seg: np.ndarray, p: Params,
+                        phys_of_logical: np.ndarray | None = None) -> OnlineStop:
+    """The pages' run-time stop (gist.science technical summary, section 2;
+    arxivlens "Methodology": stop on the marginal softmax gain).
+
+    The tile is the segment's rows of the query heads in `heads`.  Pass 1
+    takes the always-kept keys (sinks and window; each row sees those <= i).
+    Candidate blocks then follow in the order perm_seg, Bk keys each.  After
+    block b every row i has the gain g_i(b) = W_i(b) / L_i(b): W_i(b) is the
+    sum of exp(q_i . k_j / sqrt(d)) over the block, L_i(b) the same sum over
+    everything the row has processed, block b included.  The tile's gain is
+    the mean of g_i(b) over its rows (rows past N do not exist).  Processing
+    stops after the first block whose tile gain is below tau; that block has
+    been computed and stays in the output.  With no such block every
+    candidate block is processed.
+    """
+    N, d = Qf.shape[2], Qf.shape[3]
+    r0, r1 = segment_rows(N, s, p)
+    rows = np.arange(r0, r1)
+    always = always_kept(N, s, p)
+    perm_seg = np.asarray(perm_seg, dtype=np.int64)
+    nb = num_blocks(len(perm_seg), p)
+    phys = (lambda j: j) if phys_of_logical is None else (lambda j: np.asarray(phys_of_logical)[j])
+    Ka = _f64(Kf[b, kvh][phys(always)])
+    Kc = _f64(Kf[b, kvh][phys(perm_seg)]) if len(perm_seg) else np.zeros((0, d))
+    vis = always[None, :] <= rows[:, None]
+    # per (head, row): a fixed reference (the row's max over everything it
+    # could see) keeps the exponentials in range; the gains do not depend on it
+    Sa, Sc = [], []
+    for h in heads:
+        Qs = _f64(Qf[b, h, r0:r1])
+        Sa.append(np.where(vis, (Qs @ Ka.T) / math.sqrt(d), -np.inf))
+        Sc.append((Qs @ Kc.T) / math.sqrt(d))
+    Sa = np.concatenate(Sa, axis=0)
+    Sc = np.concatenate(Sc, axis=0) if len(perm_seg) else np.zeros((Sa.shape[0], 0))
+    ref = np.maximum(Sa.max(axis=1), Sc.max(axis=1) if Sc.shape[1] else -np.inf)[:, None]
+    L = np.exp(Sa - ref).sum(axis=1)
+    gains = []
+    C = nb
+    for blk in range(nb):
+        W = np.exp(Sc[:, blk * p.Bk:(blk + 1) * p.Bk] - ref).sum(axis=1)
+        L = L + W
+        g = float(np.mean(W / L))
+        gains.append(g)
+        if g < p.tau:
+            C = blk + 1
+            break
+    gains = np.array(gains, dtype=np.float64)
+    ties = np.nonzero(np.abs(gains - p.tau) <= NEAR_TIE_ONLINE_REL * p.tau)[0]
+    return OnlineStop(C=C, gains=gains, near_ties=ties)
+
+
+def tile_heads(kvh: int, G: int, pair: int) -> list:
+    """Query heads of one tile of the online rule: the pair 2*pair, 2*pair+1
+    of the group when G is even (the heads the library's kernel computes
+    together), else the single head `pair`."""
+    if G % 2 == 0:
+        return [kvh * G + 2 * pair, kvh * G + 2 * pair + 1]
+    return [kvh * G + pair]
 
 
 # ---------------------------------------------------------------------------

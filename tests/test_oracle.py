@@ -408,3 +408,125 @@ def test_stop_point_within_threshold_prefix(tau):
             seen_bound |= bound < O.num_blocks(hi - lo, p)
     # at these sizes the bound cuts the order for the larger thresholds
     assert seen_bound or tau < 3e-3
+
+
+# ---------------------------------------------------------------------------
+# run-time (online) stop rule
+# ---------------------------------------------------------------------------
+
+def test_online_tau_zero_processes_every_block_and_is_dense():
+    p = O.Params(tau=0.0)
+    Q, K, V = _random_case(5, Hq=4, Hkv=1, N=896, d=64)
+    N = Q.shape[2]
+    res = O.plan(Q, K, p)
+    off = res["offsets"]
+    for s in range(O.num_segments(N, p)):
+        perm_seg = res["perm"][0, 0, off[s]:off[s + 1]]
+        for pair in range(2):
+            st = O.online_stop_segment(Q, K, 0, 0, s, O.tile_heads(0, 4, pair), perm_seg, p)
+            assert st.C == O.num_blocks(len(perm_seg), p)
+            assert np.all(st.gains > 0)
+        keep = O.keep_set(N, s, perm_seg, st.C, p)
+        got = O.attention_segment(Q, K, V, 0, 0, s, 4, keep, p)
+        want = O.dense_segment(Q, K, V, 0, 0, s, 4, p)
+        assert np.max(np.abs(got - want)) <= 1e-12
+
+
+def test_online_all_ties_closed_form():
+    # Q = 0 makes every score 0, so every key weighs 1: after candidate block b
+    # row i has processed n_i always-kept keys plus Bk (b + 1) candidates and
+    # its gain is Bk / (n_i + Bk (b + 1)).  n_i counts sinks and window keys
+    # <= i directly from the geometry below.
+    N, Lq, Bk, W, ns = 4096, 128, 64, 128, 64
+    tau = 0.03
+    p = O.Params(tau=tau)
+    rng = np.random.default_rng(3)
+    Q = np.zeros((1, 2, N, 64), dtype=np.uint16)
+    K = _bits(rng.standard_normal((1, 1, N, 64)))
+    hit = 0
+    for s in (2, 9, 20, 31):
+        r0 = Lq * s
+        rows = np.arange(r0, min(N, r0 + Lq))
+        n_i = ns + (rows - (r0 - W) + 1)          # sinks, then the window up to row i
+        ncand = max(0, Lq * s - W - ns)
+        nb = ncand // Bk
+        want_C, want_g = nb, []
+        for blk in range(nb):
+            g = float(np.mean(Bk / (n_i + Bk * (blk + 1))))
+            want_g.append(g)
+            if g < tau:
+                want_C = blk + 1
+                break
+        perm_seg = np.arange(ns, ns + ncand)
+        st = O.online_stop_segment(Q, K, 0, 0, s, [0, 1], perm_seg, p)
+        assert st.C == want_C
+        assert np.allclose(st.gains, want_g, rtol=1e-12, atol=0)
+        hit += want_C < nb
+    assert hit >= 2  # the threshold binds in some of these segments
+
+
+def _brute_online(Qv, Kv, heads, s, perm_seg, Lq, Bk, n_sink, W, tau):
+    """Plain-Python gains and stop point of one tile (lists and math.exp)."""
+    N, d = len(Kv), len(Kv[0])
+    r0, r1 = Lq * s, min(N, Lq * s + Lq)
+    e = r1
+    always = sorted(set(range(min(n_sink, e))) | set(range(max(0, Lq * s - W), e)))
+    nb = -(-len(perm_seg) // Bk)  # the last block may be partial
+    L, gains, C = {}, [], nb
+    for h in heads:
+        for i in range(r0, r1):
+            L[(h, i)] = sum(math.exp(sum(Qv[h][i][c] * Kv[j][c] for c in range(d)) / math.sqrt(d))
+                            for j in always if j <= i)
+    for blk in range(nb):
+        tot, cnt = 0.0, 0
+        for h in heads:
+            for i in range(r0, r1):
+                w = sum(math.exp(sum(Qv[h][i][c] * Kv[j][c] for c in range(d)) / math.sqrt(d))
+                        for j in perm_seg[blk * Bk:(blk + 1) * Bk])
+                L[(h, i)] += w
+                tot += w / L[(h, i)]
+                cnt += 1
+        gains.append(tot / cnt)
+        if tot / cnt < tau:
+            C = blk + 1
+            break
+    return C, gains
+
+
+@pytest.mark.parametrize("tau", [0.2, 0.3])
+def test_online_brute_force_n16(tau):
+    p = O.Params(Lq=4, Bk=2, n_sink=1, window_prev=4, tau=tau)
+    rng = np.random.default_rng(9)
+    N, d = 16, 8
+    Q = _bits(rng.standard_normal((1, 2, N, d)) * 1.5)
+    K = _bits(rng.standard_normal((1, 1, N, d)) * 1.5)
+    Qv, Kv = O.widen_bf16(Q)[0].tolist(), O.widen_bf16(K)[0, 0].tolist()
+    res = O.plan(Q, K, p)
+    off = res["offsets"]
+    stopped = 0
+    for s in range(O.num_segments(N, p)):
+        perm_seg = res["perm"][0, 0, off[s]:off[s + 1]]
+        st = O.online_stop_segment(Q, K, 0, 0, s, [0, 1], perm_seg, p)
+        C, g = _brute_online(Qv, Kv, [0, 1], s, [int(x) for x in perm_seg], 4, 2, 1, 4, tau)
+        assert st.C == C
+        assert np.allclose(st.gains, g, rtol=1e-12, atol=0)
+        stopped += C < -(-len(perm_seg) // 2)
+    assert stopped >= 1
+
+
+def test_online_invariant_under_physical_permutation():
+    p = O.Params(tau=0.01)
+    Q, K, V = _random_case(6, Hq=2, Hkv=1, N=1024, d=64)
+    N = Q.shape[2]
+    res = O.plan(Q, K, p)
+    rng = np.random.default_rng(12)
+    pi = rng.permutation(N)
+    Kp = np.empty_like(K)
+    Kp[:, :, pi] = K
+    off = res["offsets"]
+    for s in (2, 4, 7):
+        perm_seg = res["perm"][0, 0, off[s]:off[s + 1]]
+        a = O.online_stop_segment(Q, K, 0, 0, s, [0, 1], perm_seg, p)
+        b = O.online_stop_segment(Q, Kp, 0, 0, s, [0, 1], perm_seg, p, phys_of_logical=pi)
+        assert a.C == b.C
+        assert np.allclose(a.gains, b.gains, rtol=1e-12, atol=0)
