@@ -203,6 +203,9 @@ def main():
     ap.add_argument("--impl", default="s2o", choices=["s2o", "reference"])
     ap.add_argument("--e2e-steps", type=int, default=3)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--online-steps", type=int, default=3,
+                    help="steps of the run-time stop variant (full plan + s2o_attention_online), reported beside "
+                         "the headline; 0 skips it")
     ap.add_argument("--plan", default="filtered", choices=["full", "filtered"],
                     help="s2o_plan (every segment fully ordered) or s2o_plan_filtered (only the prefix the "
                          "stop rule can reach; same kept sets and output)")
@@ -313,6 +316,32 @@ def main():
                 "frac": achieved / peak, "traffic": traffic, "kernel": "k_sparse_attn2",
                 "peak_source": f"{peak_src} bf16 sustained"}
 
+    # the pages' run-time stop: the full order, then the attention kernel
+    # deciding the stop itself; timed after the headline, reported beside it
+    online = None
+    if args.online_steps > 0 and (w.Hq // w.Hkv) % 2 == 0:
+        cout = torch.empty(w.B * w.Hq * s2o.num_segments(cfg), dtype=torch.int32, device=dev)
+        for _ in range(2):
+            s2o.plan(cfg, Q, K, bufs, filtered=False)
+            s2o.attention_online(cfg, Q, K, V, bufs["perm"], O, cout)
+        evo = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(args.online_steps)]
+        for e in evo:
+            e[0].record(stream)
+            s2o.plan(cfg, Q, K, bufs, filtered=False)
+            e[1].record(stream)
+            s2o.attention_online(cfg, Q, K, V, bufs["perm"], O, cout)
+            e[2].record(stream)
+        torch.cuda.synchronize()
+        if s2o.last_device_error() != 0:
+            raise RuntimeError("device error in the run-time stop variant")
+        op = float(np.mean([e[0].elapsed_time(e[1]) for e in evo]))
+        oa = float(np.mean([e[1].elapsed_time(e[2]) for e in evo]))
+        co = cout.cpu().numpy().reshape(w.B, w.Hq, -1)
+        online = {"plan_ms": op, "attention_ms": oa, "value": whole_job_tflops(world, dense, op + oa),
+                  "kept_pair_fraction": kept_pairs(co, w.N, 1) / (w.B * w.Hq * w.N * (w.N + 1) / 2.0),
+                  "rule": "stop after the first candidate block whose mean relative gain over the tile is < tau"}
+        s2o.plan(cfg, Q, K, bufs, filtered=filtered)
+
     # end to end through the host-buffer C ABI call (pinned host memory)
     e2e = None
     if args.e2e_steps > 0:
@@ -357,6 +386,7 @@ def main():
                        "l2": "inputs larger than L2 (Q alone is 1 GiB)", "plan": args.plan},
             "plan_ms": float(np.mean(plan_ms)), "attention_ms": attn_mean,
             "plan_other": {"kind": "full" if filtered else "filtered", "ms": other_ms},
+            "online_stop": online,
             "attention_only_tflops": whole_job_tflops(world, dense, attn_mean),
             "kept_pair_fraction": density,
             "roofline": roofline, "cpu_baseline": cpu, "e2e": e2e, "gpu_launches": launches,

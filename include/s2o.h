@@ -216,6 +216,29 @@ s2o_status s2o_attention(const s2o_config* cfg, const uint16_t* Q, const uint16_
 s2o_status s2o_prefill_arena_size(const s2o_config* cfg, int32_t out_dtype, size_t* bytes);
 
 /*
+ * s2o_attention_online -- the pages' run-time stop in place of the planned one
+ * (gist.science technical summary, section 2 "Regle d'Arret Anticipe"; the
+ * arxivlens "Methodology" facet: stop on the marginal softmax gain).  A tile
+ * is the segment's rows of a pair of query heads of a group.  It processes
+ * the always-kept keys, then the segment's candidate blocks in the order of
+ * perm; after each block, each row's gain is the block's share of the
+ * exp-sum the row has processed so far (the block included), and the tile
+ * stops after the first block whose mean gain over its rows is below
+ * cfg->tau.  That block stays in the output.
+ *   Q, K, V, O, out_dtype  as s2o_attention
+ *   perm         device int32 [B,Hkv,T] from s2o_plan (every segment fully
+ *                ordered; the filtered plan's order is not enough)
+ *   nblocks_out  out, device int32 [B,Hq,S]: candidate blocks processed by
+ *                the tile of each query head (equal within a pair)
+ *   Requires an even group size Hq/Hkv (S2O_ERR_UNSUPPORTED_SHAPE otherwise).
+ *   A perm entry outside Cand(s) is clamped and reported as S2O_ERR_BAD_PLAN
+ *   by s2o_last_device_error.
+ */
+s2o_status s2o_attention_online(const s2o_config* cfg, const uint16_t* Q, const uint16_t* K,
+                                const uint16_t* V, const int32_t* perm, void* O, int32_t out_dtype,
+                                int32_t* nblocks_out, s2o_stream_t stream);
+
+/*
  * s2o_prefill_host -- the whole path from HOST buffers: copies Q, K, V to
  * the device arena, plans (s2o_plan_filtered: it returns no perm, and O and
  * C(s) equal those of s2o_plan), runs the attention and copies O back to

@@ -67,13 +67,14 @@ def lib() -> ctypes.CDLL:
         L.s2o_plan_noalloc.argtypes = [_CFG, _P, _P, _P, _P, _P, _P, _P]
         L.s2o_plan_contiguous.argtypes = [_CFG, _P, _P, _P, _P, _P]
         L.s2o_attention.argtypes = [_CFG, _P, _P, _P, _P, _P, _P, ctypes.c_int32, _P]
+        L.s2o_attention_online.argtypes = [_CFG, _P, _P, _P, _P, _P, ctypes.c_int32, _P, _P]
         L.s2o_prefill_arena_size.argtypes = [_CFG, ctypes.c_int32, ctypes.POINTER(ctypes.c_size_t)]
         L.s2o_prefill_host.argtypes = [_CFG, _P, _P, _P, _P, ctypes.c_int32, _P, _P, ctypes.c_size_t, _P]
         L.s2o_status_string.argtypes = [ctypes.c_int]
         L.s2o_status_string.restype = ctypes.c_char_p
         L.s2o_last_device_error.argtypes = [_P]
         L.s2o_last_launch_count.restype = ctypes.c_int32
-        for name in ("s2o_plan_workspace_size", "s2o_plan", "s2o_plan_filtered", "s2o_plan_noalloc", "s2o_plan_contiguous", "s2o_attention",
+        for name in ("s2o_plan_workspace_size", "s2o_plan", "s2o_plan_filtered", "s2o_plan_noalloc", "s2o_plan_contiguous", "s2o_attention", "s2o_attention_online",
                      "s2o_prefill_arena_size", "s2o_prefill_host", "s2o_last_device_error"):
             getattr(L, name).restype = ctypes.c_int
         _lib = L
@@ -176,6 +177,19 @@ def attention(cfg: Config, Q, K, V, perm, nblocks, O=None, out_dtype: int = OUT_
     _check(lib().s2o_attention(ctypes.byref(cfg), _ptr(Q), _ptr(K), _ptr(V), _ptr(perm), _ptr(nblocks),
                                _ptr(O), out_dtype, _stream(stream)), "s2o_attention")
     return O
+
+
+def attention_online(cfg: Config, Q, K, V, perm, O=None, nblocks_out=None, out_dtype: int = OUT_BF16, stream=None):
+    """s2o_attention_online: the run-time stop; returns (O, nblocks_out [B*Hq*S])."""
+    import torch
+    if O is None:
+        O = torch.empty(Q.shape, dtype=torch.bfloat16 if out_dtype == OUT_BF16 else torch.float32,
+                        device=Q.device)
+    if nblocks_out is None:
+        nblocks_out = torch.empty(cfg.B * cfg.Hq * num_segments(cfg), dtype=torch.int32, device=Q.device)
+    _check(lib().s2o_attention_online(ctypes.byref(cfg), _ptr(Q), _ptr(K), _ptr(V), _ptr(perm), _ptr(O), out_dtype,
+                                      _ptr(nblocks_out), _stream(stream)), "s2o_attention_online")
+    return O, nblocks_out
 
 
 def prefill_host(cfg: Config, Q_host, K_host, V_host, O_host, arena, nblocks_host=None,

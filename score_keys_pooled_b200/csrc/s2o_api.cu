@@ -98,7 +98,9 @@ cudaError_t set_kernel_attributes() {
     if (e == cudaSuccess)
       e = cudaFuncSetAttribute(k_sparse_attn, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kAttnSmem);
     if (e == cudaSuccess)
-      e = cudaFuncSetAttribute(k_sparse_attn2, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kAttn2Smem);
+      e = cudaFuncSetAttribute(k_sparse_attn2<false>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kAttn2Smem);
+    if (e == cudaSuccess)
+      e = cudaFuncSetAttribute(k_sparse_attn2<true>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kAttn2Smem);
     if (e == cudaSuccess)
       e = cudaFuncSetAttribute(k_bucket_sort, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kBucketSmem);
     if (e == cudaSuccess)
@@ -276,11 +278,12 @@ s2o_status s2o_attention(const s2o_config* cfg, const uint16_t* Q, const uint16_
     a.B = cfg->B; a.Hq = cfg->Hq; a.Hkv = cfg->Hkv; a.N = cfg->N; a.S = nseg(cfg);
     a.T = ncand_total(cfg);
     a.out_f32 = out_dtype == S2O_OUT_F32;
+    a.tau = 0.f; a.cout = nullptr;
     CUtensorMap tmQ;
     if (!encode_rows_map(&tmQ, Q, (uint64_t)cfg->B * cfg->Hq * cfg->N, 128))
       return S2O_ERR_CUDA;
     const int64_t ncta = (int64_t)cfg->B * cfg->Hkv * a.S * (G / 2);
-    k_sparse_attn2<<<(unsigned)ncta, kAttn2Threads, kAttn2Smem, s>>>(a, tmQ);
+    k_sparse_attn2<false><<<(unsigned)ncta, kAttn2Threads, kAttn2Smem, s>>>(a, tmQ);
   } else {
     AttnArgs a;
     a.Q = Q; a.K = K; a.V = V; a.perm = perm; a.nblocks = nblocks; a.O = O;
@@ -290,6 +293,36 @@ s2o_status s2o_attention(const s2o_config* cfg, const uint16_t* Q, const uint16_
     const int64_t ncta = (int64_t)cfg->B * cfg->Hq * a.S;
     k_sparse_attn<<<(unsigned)ncta, kAttnThreads, kAttnSmem, s>>>(a);
   }
+  ++t_launches;
+  return launch_status();
+}
+
+s2o_status s2o_attention_online(const s2o_config* cfg, const uint16_t* Q, const uint16_t* K, const uint16_t* V,
+                                const int32_t* perm, void* O, int32_t out_dtype, int32_t* nblocks_out,
+                                s2o_stream_t stream) {
+  t_launches = 0;
+  s2o_status st = check_cfg(cfg);
+  if (st != S2O_OK) return st;
+  if (!Q || !K || !V || !perm || !O || !nblocks_out) return S2O_ERR_INVALID_ARG;
+  if (out_dtype != S2O_OUT_BF16 && out_dtype != S2O_OUT_F32) return S2O_ERR_INVALID_ARG;
+  if (!aligned16(Q) || !aligned16(K) || !aligned16(V) || !aligned16(O) || !aligned16(perm) ||
+      !aligned16(nblocks_out))
+    return S2O_ERR_INVALID_ARG;
+  const int G = cfg->Hq / cfg->Hkv;
+  // the tile of the rule is the pair of query heads one CTA computes
+  if (G % 2 != 0 || (int64_t)cfg->B * cfg->Hq * cfg->N >= (int64_t)INT32_MAX) return S2O_ERR_UNSUPPORTED_SHAPE;
+  if (set_kernel_attributes() != cudaSuccess) return S2O_ERR_CUDA;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  Attn2Args a;
+  a.Q = Q; a.K = K; a.V = V; a.perm = perm; a.nblocks = nullptr; a.O = O;
+  a.B = cfg->B; a.Hq = cfg->Hq; a.Hkv = cfg->Hkv; a.N = cfg->N; a.S = nseg(cfg);
+  a.T = ncand_total(cfg);
+  a.out_f32 = out_dtype == S2O_OUT_F32;
+  a.tau = (float)cfg->tau; a.cout = nblocks_out;
+  CUtensorMap tmQ;
+  if (!encode_rows_map(&tmQ, Q, (uint64_t)cfg->B * cfg->Hq * cfg->N, 128)) return S2O_ERR_CUDA;
+  const int64_t ncta = (int64_t)cfg->B * cfg->Hkv * a.S * (G / 2);
+  k_sparse_attn2<true><<<(unsigned)ncta, kAttn2Threads, kAttn2Smem, s>>>(a, tmQ);
   ++t_launches;
   return launch_status();
 }

@@ -75,7 +75,11 @@ constexpr int kBarSFull = 11;   // [2]     MMA commit (S_i written) -> softmax i
 constexpr int kBarSEmpty = 13;  // [2]     softmax i, one arrive per warp (S_i read) -> MMA
 constexpr int kBarPFull = 15;   // [2][2]  softmax i, one arrive per warp (P_i,b written) -> MMA; slot + 2 i + b
 constexpr int kBarODone = 19;   // [2][2]  MMA commit (P_i,b consumed, O_i updated) -> softmax i
-constexpr int kSlotTmem = 23;
+constexpr int kBarGain = 23;    //      online stop: the 8 softmax warps (count 8) added their rows' gains
+constexpr int kSlotTmem = 24;
+constexpr int kSlotGain = 25;   //      online stop: 3 fp32 gain accumulators (slots 25, 26)
+constexpr int kSlotStop = 27;   //      online stop: index of the chunk after which the tile stops
+constexpr int kNoStop = 0x7fffffff;
 // tensor-memory columns
 __device__ __forceinline__ uint32_t col_o(int i) { return 128u * i; }
 __device__ __forceinline__ uint32_t col_s(int i) { return 256u + 64u * i; }
@@ -178,8 +182,17 @@ struct Attn2Args {
   int B, Hq, Hkv, N, S;
   int64_t T;
   int out_f32;
+  // run-time stop (k_sparse_attn2<true>; gist.science technical summary,
+  // section 2): walk every candidate block of the full order and stop after
+  // the first one whose mean relative gain over the tile's rows is below tau;
+  // blocks processed per query head go to cout [B, Hq, S]
+  float tau;
+  int32_t* cout;
 };
 
+// ONLINE selects the run-time stop; the planned-stop kernel is compiled
+// without any of its code
+template <bool ONLINE>
 __global__ void __launch_bounds__(kAttn2Threads, 1)
     k_sparse_attn2(Attn2Args a, const __grid_constant__ CUtensorMap tmQ) {
   extern __shared__ uint8_t smem_raw[];
@@ -203,8 +216,8 @@ __global__ void __launch_bounds__(kAttn2Threads, 1)
   const int b = bk / a.Hkv, kvh = bk % a.Hkv;
   const int h0 = kvh * G + 2 * pair;
 
-  int C = a.nblocks[(size_t)bk * a.S + s];
   const int cmax = (int)(num_cand(s) / kBk);
+  int C = ONLINE ? cmax : a.nblocks[(size_t)bk * a.S + s];
   if (C < 0 || C > cmax) {
     if (tid == 0) set_error(kErrBadPlan);
     C = C < 0 ? 0 : cmax;
@@ -218,10 +231,15 @@ __global__ void __launch_bounds__(kAttn2Threads, 1)
       uint32_t count = 1;
       if ((k >= kBarSEmpty && k < kBarSEmpty + 2) || (k >= kBarPFull && k < kBarPFull + 4)) count = 4;
       if ((k >= kBarKEmpty && k < kBarKEmpty + kStagesK) || (k >= kBarVEmpty && k < kBarVEmpty + kStagesV)) count = 2;
+      if (k == kBarGain) count = 8;
       mbar_init(bar(k), count);
     }
+    float* gacc = reinterpret_cast<float*>(sgen + kOff2Bar + 8 * kSlotGain);
+    gacc[0] = gacc[1] = gacc[2] = 0.f;
+    *reinterpret_cast<volatile int*>(sgen + kOff2Bar + 8 * kSlotStop) = kNoStop;
     fence_mbar_init();
   }
+  volatile int* stop_word = reinterpret_cast<volatile int*>(sgen + kOff2Bar + 8 * kSlotStop);
   if (warp == kMmaWarp) {
     tmem_alloc(smem_u32((const void*)tmem_slot), kTmem2Cols);
     tmem_relinquish();
@@ -307,12 +325,36 @@ __global__ void __launch_bounds__(kAttn2Threads, 1)
     const uint32_t ktab = keys_s + 256u * (uint32_t)sel;
     int y[4];
     if (ntiles > 0) fetch_keys(0, y);
+    // with the run-time stop a tile past the stop point is not needed: the
+    // last products issued after a stop at chunk c read K of chunk c + 1
+    auto not_needed = [&](int t) {
+      const int sc = *stop_word;
+      return sc != kNoStop && t > sc / 2 + 1;
+    };
     for (int t = 0; t < ntiles; ++t) {
       const int st = t % nst;
       const int round = t / nst;
+      if (ONLINE && not_needed(t)) break;
       const bool ragged = stage_keys(t, y);
       if (t + 1 < ntiles) fetch_keys(t + 1, y);  // in flight while this stage fills
-      if (!warp_wait(bar(bar_empty + st), (uint32_t)((round & 1) ^ 1))) {
+      bool okw;
+      if (!ONLINE) {
+        okw = warp_wait(bar(bar_empty + st), (uint32_t)((round & 1) ^ 1));
+      } else {
+        // lane 0 waits for the stage or for a stop that makes it unneeded;
+        // after a free stage every lane acquires the barrier itself
+        int r = 0;
+        if (lane == 0) {
+          for (uint32_t it = 0; it < kSpinLimit && r == 0; ++it) {
+            if (mbar_try_wait(bar(bar_empty + st), (uint32_t)((round & 1) ^ 1))) r = 1;
+            else if (not_needed(t)) r = 2;
+          }
+        }
+        r = __shfl_sync(0xffffffffu, r, 0);
+        if (r == 2) break;
+        okw = r == 1 && warp_wait(bar(bar_empty + st), (uint32_t)((round & 1) ^ 1));
+      }
+      if (!okw) {
         if (lane == 0) set_error(kErrTimeout);
         break;
       }
@@ -401,6 +443,12 @@ __global__ void __launch_bounds__(kAttn2Threads, 1)
           }
           tc_commit(bar(kBarODone + 2 * i + hp));
           if (hp == 1) tc_commit(bar(kBarVEmpty + tp % kStagesV));
+          if (ONLINE && cp == *stop_word) {
+            // the tile stopped after chunk cp; Q K^T of chunk c (if any) is
+            // the last product in flight: wait for it before the CTA ends
+            if (c < nch) ok = mbar_wait_bounded(bar(kBarSFull + i), (uint32_t)(c & 1));
+            break;
+          }
         }
       }
       if (!ok) set_error(kErrTimeout);
@@ -418,6 +466,12 @@ __global__ void __launch_bounds__(kAttn2Threads, 1)
     float m_run = -INFINITY, ell = 0.f;
     bool ok = true;
     const int nch = 2 * ntiles;
+    // online stop: rows of the tile that exist (both heads)
+    const float nrows_valid = 2.f * (float)min(kLq, a.N - row0);
+    volatile float* gacc = reinterpret_cast<volatile float*>(sgen + kOff2Bar + 8 * kSlotGain);
+    int c_online = cmax;
+    bool stop_now = false;
+    int nch_done = nch;
     for (int c = 0; ok && c < nch; ++c) {
       // key k of the chunk is visible iff k <= lim
       int j0;
@@ -492,6 +546,27 @@ __global__ void __launch_bounds__(kAttn2Threads, 1)
         }
       }
       ell += rs;
+      if (ONLINE && kind == 2) {
+        // the block's gain for this row, relative to everything the row has
+        // processed (the block included; both sums share the reference m_run)
+        float gsum = row < a.N ? rs / ell : 0.f;
+#pragma unroll
+        for (int o = 16; o >= 1; o >>= 1) gsum += __shfl_xor_sync(0xffffffffu, gsum, o);
+        const int q = j0;  // candidate block index
+        if (lane == 0) {
+          atomicAdd(const_cast<float*>(gacc + q % 3), gsum);
+          mbar_arrive(bar(kBarGain));
+        }
+        if (!warp_wait(bar(kBarGain), (uint32_t)(q & 1))) { ok = false; break; }
+        const float tot = gacc[q % 3];
+        // the slot used at q - 1: every warp read it before arriving at q
+        if (warp == 0 && lane == 0) gacc[(q + 2) % 3] = 0.f;
+        stop_now = tot < a.tau * nrows_valid;
+        if (stop_now) {
+          c_online = q + 1;
+          if ((warp & 3) == 0 && lane == 0) *stop_word = c;  // read by the issuers after this chunk's P
+        }
+      }
       // P buffer c & 1 was last read by chunk c - 2's P V, which this head's
       // issuer committed before chunk c's Q K^T: the S-full barrier of chunk c
       // (waited above) already covers it
@@ -500,9 +575,16 @@ __global__ void __launch_bounds__(kAttn2Threads, 1)
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(bar(kBarPFull + 2 * qi + (c & 1)));
+      if (stop_now) {
+        nch_done = c + 1;
+        break;
+      }
     }
-    if (ok && nch > 0)
-      ok = warp_wait(bar(kBarODone + 2 * qi + ((nch - 1) & 1)), (uint32_t)(((nch - 1) >> 1) & 1));
+    if (ONLINE && tid == 0) {
+      for (int k = 0; k < 2; ++k) a.cout[((size_t)b * a.Hq + h0 + k) * a.S + s] = c_online;
+    }
+    if (ok && nch_done > 0)
+      ok = warp_wait(bar(kBarODone + 2 * qi + ((nch_done - 1) & 1)), (uint32_t)(((nch_done - 1) >> 1) & 1));
     if (!ok) {
       if (lane == 0) set_error(kErrTimeout);
     } else {

@@ -61,6 +61,12 @@ def test_null_and_alignment_rejected_before_any_launch(L):
     ws = s2o.plan_workspace_size(cfg)
     assert L.s2o_plan(ctypes.byref(cfg), good, good, good, good, good, None, P(1 << 20), ws - 1, None) == 3
     assert L.s2o_plan_contiguous(ctypes.byref(cfg), good, None, good, good, None) == 1
+    # the run-time stop: null output count, bad dtype, and an odd group size (its tile is a head pair)
+    assert L.s2o_attention_online(ctypes.byref(cfg), good, good, good, good, good, 0, None, None) == 1
+    assert L.s2o_attention_online(ctypes.byref(cfg), good, good, good, good, good, 7, good, None) == 1
+    odd = s2o.make_config(1, 3, 1, 1024)
+    assert L.s2o_attention_online(ctypes.byref(odd), good, good, good, good, good, 0, good, None) == 2
+    assert L.s2o_plan_filtered(ctypes.byref(cfg), None, good, good, good, good, None, good, 1 << 30, None) == 1
 
 
 def test_status_strings(L):

@@ -329,3 +329,90 @@ def test_filtered_plan_tau_sweep():
     for tau in synth.TAU_SWEEP:
         cfg = s2o.make_config(w.B, w.Hq, w.Hkv, w.N, tau=tau)
         filtered_matches_full(cfg, q, k, v)
+
+
+# ---------------------------------------------------------------------------
+# s2o_attention_online: the pages' run-time stop
+# ---------------------------------------------------------------------------
+
+def check_online(Q, K, V, cfg, perm_dev, out, cout, p, segments=None, kvheads=None, what=""):
+    """Per tile: the oracle's rule on the GPU's own order must stop where the
+    GPU stopped, except inside the band of tau; the output must match the
+    oracle over the GPU's kept set."""
+    G = cfg.Hq // cfg.Hkv
+    S = O.num_segments(cfg.N, p)
+    off = O.candidate_offsets(cfg.N, p)
+    T = int(off[-1])
+    perm = perm_dev[:cfg.B * cfg.Hkv * T].cpu().numpy().reshape(cfg.B, cfg.Hkv, T)
+    cg = cout.cpu().numpy().reshape(cfg.B, cfg.Hq, S)
+    got = out.float().cpu().numpy()
+    flips = 0
+    for b in range(cfg.B):
+        for kvh in (range(cfg.Hkv) if kvheads is None else kvheads):
+            for s in (range(S) if segments is None else segments):
+                perm_seg = perm[b, kvh, off[s]:off[s + 1]]
+                for pair in range(G // 2):
+                    heads = O.tile_heads(kvh, G, pair)
+                    c_gpu = int(cg[b, heads[0], s])
+                    assert c_gpu == int(cg[b, heads[1], s])
+                    st = O.online_stop_segment(Q, K, b, kvh, s, heads, perm_seg, p)
+                    if c_gpu != st.C:
+                        # the blocks where the two stopped must be near-ties of tau
+                        lo_c = min(c_gpu, st.C)
+                        assert lo_c - 1 in set(int(x) for x in st.near_ties), \
+                            f"{what} b={b} kvh={kvh} s={s} pair={pair}: C {c_gpu} != oracle {st.C}"
+                        flips += 1
+                    keep = O.keep_set(cfg.N, s, perm_seg, c_gpu, p)
+                    ref = O.attention_segment(Q, K, V, b, kvh, s, G, keep, p)
+                    r0, r1 = O.segment_rows(cfg.N, s, p)
+                    g = got[b, heads[0]:heads[-1] + 1, r0:r1]
+                    parity.assert_output_close(g, ref[heads[0] - kvh * G:heads[-1] - kvh * G + 1],
+                                               f"{what} online b={b} kvh={kvh} s={s} pair={pair}")
+    parity.log_near_ties({"case": what, "online": True, "tau": p.tau, "C_flips": flips})
+    return cg
+
+
+ONLINE_SMALL = [c for c in SMALL if (c[1] // c[2]) % 2 == 0]
+
+
+@pytest.mark.parametrize("B,Hq,Hkv,N,tau,planted,band", ONLINE_SMALL)
+def test_online_small_cases(B, Hq, Hkv, N, tau, planted, band):
+    Q, K, V = synth.generate(B, Hq, Hkv, N, 128, planted=planted, band=band, n_stripe=8, seed=N + 7)
+    cfg = s2o.make_config(B, Hq, Hkv, N, tau=tau)
+    q, k, v = dev(Q), dev(K), dev(V)
+    bufs = s2o.plan(cfg, q, k)
+    out, cout = s2o.attention_online(cfg, q, k, v, bufs["perm"])
+    assert s2o.last_launch_count() == 1
+    assert s2o.last_device_error() == 0
+    check_online(Q, K, V, cfg, bufs["perm"], out, cout, O.Params(tau=tau), what=f"online small N={N}")
+
+
+def test_online_tau_zero_equals_planned_kernel_with_every_block():
+    Q, K, V = synth.generate(1, 8, 2, 1280, 128, planted=True, band=True, n_stripe=8, seed=21)
+    cfg = s2o.make_config(1, 8, 2, 1280, tau=0.0)
+    q, k, v = dev(Q), dev(K), dev(V)
+    bufs = s2o.plan(cfg, q, k)
+    out, cout = s2o.attention_online(cfg, q, k, v, bufs["perm"])
+    S = s2o.num_segments(cfg)
+    cmax = torch.tensor([max(0, 128 * s - 192) // 64 for s in range(S)], dtype=torch.int32)
+    assert torch.equal(cout.cpu().view(8, S), cmax.repeat(8, 1))
+    ref = s2o.attention(cfg, q, k, v, bufs["perm"], bufs["nblocks"])  # tau = 0 plans every block too
+    assert torch.equal(bufs["nblocks"].cpu().view(2, S), cmax.repeat(2, 1))
+    assert torch.equal(out, ref)
+    assert s2o.last_device_error() == 0
+
+
+@pytest.mark.parametrize("name", ["llama_16k", "llama_128k"])
+def test_online_workloads(name):
+    w = synth.WORKLOADS[name]
+    Q, K, V = synth.generate_workload(w)
+    cfg = s2o.make_config(w.B, w.Hq, w.Hkv, w.N, tau=w.tau)
+    q, k, v = dev(Q), dev(K), dev(V)
+    bufs = s2o.plan(cfg, q, k)
+    out, cout = s2o.attention_online(cfg, q, k, v, bufs["perm"])
+    assert s2o.last_device_error() == 0
+    p = O.Params(tau=w.tau)
+    S = O.num_segments(w.N, p)
+    segs = sampled_segments(S)[::2] if w.N > 20000 else sampled_segments(S)
+    check_online(Q, K, V, cfg, bufs["perm"], out, cout, p, segments=segs, kvheads=[0, w.Hkv - 1],
+                 what=f"online {name}")
