@@ -63,7 +63,8 @@
  * Ownership: the caller allocates every buffer, including the plan workspace
  * (size from s2o_plan_workspace_size).  The library never allocates device
  * memory.  Its only global state per device is a 32-bit device error word
- * (see s2o_last_device_error) and the fixed scratch of s2o_plan_noalloc.
+ * (see s2o_last_device_error), the fixed scratch of s2o_plan_noalloc and the
+ * two copy streams of s2o_prefill_host (created on its first call).
  *
  * Execution: every call except s2o_prefill_host and s2o_last_device_error is
  * asynchronous on the given stream (NULL = the legacy default stream) and
@@ -242,7 +243,10 @@ s2o_status s2o_attention_online(const s2o_config* cfg, const uint16_t* Q, const 
  * s2o_prefill_host -- the whole path from HOST buffers: copies Q, K, V to
  * the device arena, plans (s2o_plan_filtered: it returns no perm, and O and
  * C(s) equal those of s2o_plan), runs the attention and copies O back to
- * host O.
+ * host O.  The work is split by (b, kvh), whose rows are contiguous in every
+ * buffer: the copies in run on one library stream, plan and attention on
+ * `stream`, the copies out on another library stream, so one group's copies
+ * overlap the kernels of the others (results equal a single whole call).
  * Host buffers should be page-locked for full copy speed.  The arena is
  * caller-allocated device memory of s2o_prefill_arena_size() bytes, 256-byte
  * aligned.  Synchronises the stream before returning and reports device

@@ -148,6 +148,29 @@ std::mutex g_scratch_mu;
 constexpr int kMaxDevices = 64;
 void* g_scratch_addr[kMaxDevices] = {};
 
+// Copy streams of s2o_prefill_host (host->device, device->host), created on
+// the first call on each device and kept for the life of the process.
+std::mutex g_copy_mu;
+cudaStream_t g_copy_in[kMaxDevices] = {}, g_copy_out[kMaxDevices] = {};
+bool copy_streams(cudaStream_t& in, cudaStream_t& out) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return false;
+  std::lock_guard<std::mutex> lock(g_copy_mu);
+  if (!g_copy_in[dev]) {
+    cudaStream_t a = nullptr, b = nullptr;
+    if (cudaStreamCreateWithFlags(&a, cudaStreamNonBlocking) != cudaSuccess) return false;
+    if (cudaStreamCreateWithFlags(&b, cudaStreamNonBlocking) != cudaSuccess) {
+      cudaStreamDestroy(a);
+      return false;
+    }
+    g_copy_in[dev] = a;
+    g_copy_out[dev] = b;
+  }
+  in = g_copy_in[dev];
+  out = g_copy_out[dev];
+  return true;
+}
+
 s2o_status launch_status() {
   return cudaGetLastError() == cudaSuccess ? S2O_OK : S2O_ERR_CUDA;
 }
@@ -335,8 +358,11 @@ s2o_status s2o_prefill_arena_size(const s2o_config* cfg, int32_t out_dtype, size
   const size_t T = (size_t)cfg->B * cfg->Hkv * ncand_total(cfg), S = (size_t)cfg->B * cfg->Hkv * nseg(cfg);
   size_t ws = 0;
   s2o_plan_workspace_size(cfg, &ws);
+  // nblocks: one 16-byte aligned slot of ceil(S/4)*4 entries per (b, kvh)
+  const size_t snb = (size_t)cfg->B * cfg->Hkv * (((size_t)nseg(cfg) + 3) & ~(size_t)3);
   *bytes = round256(q * 2) + 2 * round256(kv * 2) + round256(q * (out_dtype == S2O_OUT_F32 ? 4 : 2)) +
-           round256(T * 4 + 16) * 2 + round256(S * 4) + ws;
+           round256(T * 4 + 16) * 2 + round256(snb * 4) + ws;
+  (void)S;
   return S2O_OK;
 }
 
@@ -362,24 +388,76 @@ s2o_status s2o_prefill_host(const s2o_config* cfg, const uint16_t* Q_host, const
   void* dO = p; p += round256(obytes);
   float* dscores = reinterpret_cast<float*>(p); p += round256(T * 4 + 16);
   int32_t* dperm = reinterpret_cast<int32_t*>(p); p += round256(T * 4 + 16);
-  int32_t* dnb = reinterpret_cast<int32_t*>(p); p += round256(S * 4);
+  const size_t Sp = ((size_t)nseg(cfg) + 3) & ~(size_t)3;  // nblocks slot per (b, kvh), 16-byte aligned
+  int32_t* dnb = reinterpret_cast<int32_t*>(p); p += round256((size_t)cfg->B * cfg->Hkv * Sp * 4);
+  (void)S;
   void* ws = p;
   size_t wsb = 0;
   s2o_plan_workspace_size(cfg, &wsb);
 
-  if (cudaMemcpyAsync(dQ, Q_host, q * 2, cudaMemcpyHostToDevice, s) != cudaSuccess ||
-      cudaMemcpyAsync(dK, K_host, kv * 2, cudaMemcpyHostToDevice, s) != cudaSuccess ||
-      cudaMemcpyAsync(dV, V_host, kv * 2, cudaMemcpyHostToDevice, s) != cudaSuccess)
-    return S2O_ERR_CUDA;
-  st = run_plan(cfg, dQ, dK, dscores, dperm, dnb, nullptr, ws, wsb, stream, 1);
+  // One unit = one (b, kvh): its query heads, K and V rows are contiguous in
+  // every buffer and its plan and attention depend on nothing else.  Units
+  // are copied in on one stream, planned and attended on the caller's stream
+  // and copied out on a third, so the copies of one unit overlap the kernels
+  // of the others.  The kernels see exactly the inputs of a whole-problem
+  // call, so the results are the same.
+  cudaStream_t s_in = nullptr, s_out = nullptr;
+  if (!copy_streams(s_in, s_out)) return S2O_ERR_CUDA;
+  const int G = cfg->Hq / cfg->Hkv;
+  const int U = cfg->B * cfg->Hkv;
+  s2o_config sub = *cfg;
+  sub.B = 1;
+  sub.Hq = G;
+  sub.Hkv = 1;
+  const size_t qu = (size_t)G * cfg->N * kD, kvu = (size_t)cfg->N * kD;
+  const size_t Tu = (size_t)ncand_total(cfg), Su = (size_t)nseg(cfg);
+  const size_t oelt = out_dtype == S2O_OUT_F32 ? 4 : 2;
+  size_t wsu = 0;
+  s2o_plan_workspace_size(&sub, &wsu);
+  cudaEvent_t ev0 = nullptr;
+  cudaEvent_t* ev = new cudaEvent_t[2 * (size_t)U]();
+  bool cuda_ok = cudaEventCreateWithFlags(&ev0, cudaEventDisableTiming) == cudaSuccess;
+  for (int u = 0; cuda_ok && u < 2 * U; ++u)
+    cuda_ok = cudaEventCreateWithFlags(&ev[u], cudaEventDisableTiming) == cudaSuccess;
+  // the copies start after the caller's earlier work on its stream (the
+  // arena may still be in use there)
+  cuda_ok = cuda_ok && cudaEventRecord(ev0, s) == cudaSuccess && cudaStreamWaitEvent(s_in, ev0, 0) == cudaSuccess &&
+            cudaStreamWaitEvent(s_out, ev0, 0) == cudaSuccess;
+  for (int u = 0; cuda_ok && u < U; ++u) {
+    cuda_ok = cudaMemcpyAsync(dQ + u * qu, Q_host + u * qu, qu * 2, cudaMemcpyHostToDevice, s_in) == cudaSuccess &&
+              cudaMemcpyAsync(dK + u * kvu, K_host + u * kvu, kvu * 2, cudaMemcpyHostToDevice, s_in) == cudaSuccess &&
+              cudaMemcpyAsync(dV + u * kvu, V_host + u * kvu, kvu * 2, cudaMemcpyHostToDevice, s_in) == cudaSuccess &&
+              cudaEventRecord(ev[u], s_in) == cudaSuccess;
+  }
+  int32_t launches = 0;
+  for (int u = 0; cuda_ok && st == S2O_OK && u < U; ++u) {
+    cuda_ok = cudaStreamWaitEvent(s, ev[u], 0) == cudaSuccess;
+    if (!cuda_ok) break;
+    st = run_plan(&sub, dQ + u * qu, dK + u * kvu, dscores + u * Tu, dperm + u * Tu, dnb + u * Sp, nullptr, ws, wsu,
+                  stream, 1);
+    if (st != S2O_OK) break;
+    launches += t_launches;
+    void* dOu = static_cast<uint8_t*>(dO) + u * qu * oelt;
+    st = s2o_attention(&sub, dQ + u * qu, dK + u * kvu, dV + u * kvu, dperm + u * Tu, dnb + u * Sp, dOu, out_dtype,
+                       stream);
+    if (st != S2O_OK) break;
+    launches += t_launches;
+    cuda_ok = cudaEventRecord(ev[U + u], s) == cudaSuccess && cudaStreamWaitEvent(s_out, ev[U + u], 0) == cudaSuccess &&
+              cudaMemcpyAsync(static_cast<uint8_t*>(O_host) + u * qu * oelt, dOu, qu * oelt, cudaMemcpyDeviceToHost,
+                              s_out) == cudaSuccess &&
+              (!nblocks_host || cudaMemcpyAsync(nblocks_host + u * Su, dnb + u * Sp, Su * 4, cudaMemcpyDeviceToHost,
+                                                s_out) == cudaSuccess);
+  }
+  // every stream drains before the events go and the call returns
+  const bool sync_ok = cudaStreamSynchronize(s_in) == cudaSuccess && cudaStreamSynchronize(s_out) == cudaSuccess &&
+                       cudaStreamSynchronize(s) == cudaSuccess;
+  if (ev0) cudaEventDestroy(ev0);
+  for (int u = 0; u < 2 * U; ++u)
+    if (ev[u]) cudaEventDestroy(ev[u]);
+  delete[] ev;
+  t_launches = launches;
   if (st != S2O_OK) return st;
-  const int32_t n_plan = t_launches;
-  st = s2o_attention(cfg, dQ, dK, dV, dperm, dnb, dO, out_dtype, stream);
-  if (st != S2O_OK) return st;
-  t_launches += n_plan;
-  if (cudaMemcpyAsync(O_host, dO, obytes, cudaMemcpyDeviceToHost, s) != cudaSuccess) return S2O_ERR_CUDA;
-  if (nblocks_host && cudaMemcpyAsync(nblocks_host, dnb, S * 4, cudaMemcpyDeviceToHost, s) != cudaSuccess)
-    return S2O_ERR_CUDA;
+  if (!cuda_ok || !sync_ok) return S2O_ERR_CUDA;
   return s2o_last_device_error(stream);
 }
 

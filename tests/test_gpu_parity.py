@@ -176,15 +176,21 @@ def test_out_of_range_plan_is_clamped_and_reported():
     assert s2o.last_device_error() == 0
 
 
-def test_host_buffer_entry_matches_device_path():
-    Q, K, V = synth.generate(1, 8, 2, 1536, 128, planted=True, band=True, n_stripe=8, seed=12)
-    cfg, bufs, out = run_path(Q, K, V, 1e-3)
-    arena = torch.empty(s2o.prefill_arena_size(cfg), dtype=torch.uint8, device="cuda")
+@pytest.mark.parametrize("B,Hq,Hkv,N,out_dtype", [(1, 8, 2, 1536, s2o.OUT_BF16), (2, 4, 2, 1000, s2o.OUT_F32),
+                                                  (2, 4, 4, 640, s2o.OUT_BF16)])
+def test_host_buffer_entry_matches_device_path(B, Hq, Hkv, N, out_dtype):
+    # the host entry pipelines its work by (b, kvh) over three streams; the
+    # result must equal the device path bit for bit
+    Q, K, V = synth.generate(B, Hq, Hkv, N, 128, planted=True, band=True, n_stripe=8, seed=12)
+    cfg, bufs, out = run_path(Q, K, V, 1e-3, out_dtype)
+    arena = torch.empty(s2o.prefill_arena_size(cfg, out_dtype), dtype=torch.uint8, device="cuda")
     pin = lambda a: torch.from_numpy(a.view(np.int16)).pin_memory()
-    O_host = torch.empty(Q.shape, dtype=torch.int16).pin_memory()
+    odt = torch.int16 if out_dtype == s2o.OUT_BF16 else torch.float32
+    O_host = torch.empty(Q.shape, dtype=odt).pin_memory()
     nb_host = torch.empty(cfg.B * cfg.Hkv * s2o.num_segments(cfg), dtype=torch.int32)
-    s2o.prefill_host(cfg, pin(Q), pin(K), pin(V), O_host, arena, nblocks_host=nb_host)
-    assert torch.equal(O_host.view(torch.bfloat16), out.cpu())
+    s2o.prefill_host(cfg, pin(Q), pin(K), pin(V), O_host, arena, nblocks_host=nb_host, out_dtype=out_dtype)
+    got = O_host.view(torch.bfloat16) if out_dtype == s2o.OUT_BF16 else O_host
+    assert torch.equal(got, out.cpu())
     assert torch.equal(nb_host, bufs["nblocks"].cpu())
 
 
