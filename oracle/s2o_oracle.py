@@ -418,6 +418,54 @@ def tile_heads(kvh: int, G: int, pair: int) -> list:
 
 
 # ---------------------------------------------------------------------------
+# Ranking accuracy: the pooled order against the true attention mass
+# ---------------------------------------------------------------------------
+
+@dataclass
+class BlockTruth:
+    mass: np.ndarray     # [n_blocks] true mean mass of each block of the order
+    always: float        # true mean mass of the always-kept keys
+    kept: int            # blocks the plan keeps (C)
+    true: int            # blocks whose true mass is >= tau
+    both: int            # blocks in both sets
+    captured: float      # true mass of the kept blocks
+    total: float         # true mass of all candidate blocks
+
+
+def true_block_masses(Qf, Kf, b: int, kvh: int, s: int, G: int, perm_seg: np.ndarray, C: int,
+                      p: Params) -> BlockTruth:
+    """Checks the pooled estimate against exact attention (the referee
+    reports on the pith.science page note that ranking accuracy is not
+    measured).  For every row i of the segment and head of the group, the
+    exact causal softmax over all of [0, i] gives each candidate key its
+    probability; a block's true mass is the mean over those rows of the
+    probabilities of its keys.  The kept set is the plan's first C blocks,
+    the true set the blocks whose true mass is at least tau."""
+    N, d = Qf.shape[2], Qf.shape[3]
+    r0, r1 = segment_rows(N, s, p)
+    e = admissible_end(N, s, p)
+    rows = np.arange(r0, r1)
+    Ka = _f64(Kf[b, kvh, :e])
+    perm_seg = np.asarray(perm_seg, dtype=np.int64)
+    col = np.zeros(e)
+    for g in range(G):
+        Qs = _f64(Qf[b, kvh * G + g, r0:r1])
+        S = (Qs @ Ka.T) / math.sqrt(d)
+        S = np.where(np.arange(e)[None, :] <= rows[:, None], S, -np.inf)
+        P = np.exp(S - S.max(axis=1, keepdims=True))
+        P = P / P.sum(axis=1, keepdims=True)
+        col += P.sum(axis=0)
+    col /= G * (r1 - r0)
+    nb = num_blocks(len(perm_seg), p)
+    mass = np.array([col[perm_seg[k * p.Bk:(k + 1) * p.Bk]].sum() for k in range(nb)], dtype=np.float64)
+    always = float(col[always_kept(N, s, p)].sum())
+    kept = min(C, nb)
+    tset = mass >= p.tau
+    return BlockTruth(mass=mass, always=always, kept=kept, true=int(tset.sum()), both=int(tset[:kept].sum()),
+                      captured=float(mass[:kept].sum()), total=float(mass.sum()))
+
+
+# ---------------------------------------------------------------------------
 # Contiguous top-k comparator (block-sparse baseline at matched block count)
 # ---------------------------------------------------------------------------
 

@@ -530,3 +530,65 @@ def test_online_invariant_under_physical_permutation():
         b = O.online_stop_segment(Q, Kp, 0, 0, s, [0, 1], perm_seg, p, phys_of_logical=pi)
         assert a.C == b.C
         assert np.allclose(a.gains, b.gains, rtol=1e-12, atol=0)
+
+
+# ---------------------------------------------------------------------------
+# ranking accuracy: true block masses
+# ---------------------------------------------------------------------------
+
+def test_true_masses_sum_to_one_with_the_always_kept_keys():
+    # each row's softmax sums to 1, so the mean over rows does too
+    p = O.Params(tau=1e-3)
+    Q, K, V = _random_case(8, Hq=4, Hkv=1, N=1024, d=64)
+    N = Q.shape[2]
+    res = O.plan(Q, K, p)
+    off = res["offsets"]
+    for s in range(O.num_segments(N, p)):
+        bt = O.true_block_masses(Q, K, 0, 0, s, 4, res["perm"][0, 0, off[s]:off[s + 1]], int(res["nblocks"][0, 0, s]), p)
+        assert bt.total + bt.always == pytest.approx(1.0, abs=1e-12)
+        assert 0 <= bt.both <= min(bt.kept, bt.true)
+        assert bt.captured <= bt.total + 1e-15
+
+
+def test_true_masses_uniform_closed_form():
+    # Q = 0: row i attends uniformly to its i + 1 keys, so a candidate key
+    # (j < every row) gets mean_i 1/(i + 1) and a block 64 times that
+    N = 1024
+    p = O.Params(tau=1e-3)
+    rng = np.random.default_rng(2)
+    Q = np.zeros((1, 2, N, 64), dtype=np.uint16)
+    K = _bits(rng.standard_normal((1, 1, N, 64)))
+    for s in (2, 5, 7):
+        rows = np.arange(128 * s, 128 * s + 128)
+        per_key = float(np.mean(1.0 / (rows + 1)))
+        ncand = 128 * s - 192
+        perm_seg = np.arange(64, 64 + ncand)[::-1].copy()
+        bt = O.true_block_masses(Q, K, 0, 0, s, 2, perm_seg, 2, p)
+        assert np.allclose(bt.mass, 64 * per_key, rtol=1e-12, atol=0)
+        assert bt.true == (len(bt.mass) if 64 * per_key >= p.tau else 0)
+        kept = min(2, len(bt.mass))
+        assert bt.kept == kept and bt.both == (kept if 64 * per_key >= p.tau else 0)
+        assert bt.captured == pytest.approx(kept * 64 * per_key, rel=1e-12)
+
+
+def test_true_masses_brute_force_n16():
+    p = O.Params(Lq=4, Bk=2, n_sink=1, window_prev=4, tau=0.1)
+    rng = np.random.default_rng(4)
+    N, d, G = 16, 8, 2
+    Q = _bits(rng.standard_normal((1, G, N, d)) * 1.5)
+    K = _bits(rng.standard_normal((1, 1, N, d)) * 1.5)
+    Qv, Kv = O.widen_bf16(Q)[0].tolist(), O.widen_bf16(K)[0, 0].tolist()
+    res = O.plan(Q, K, p)
+    off = res["offsets"]
+    for s in range(2, O.num_segments(N, p)):
+        perm_seg = [int(x) for x in res["perm"][0, 0, off[s]:off[s + 1]]]
+        rows = range(4 * s, 4 * s + 4)
+        col = {j: 0.0 for j in range(N)}
+        for g in range(G):
+            for i in rows:
+                w = [math.exp(sum(Qv[g][i][c] * Kv[j][c] for c in range(d)) / math.sqrt(d)) for j in range(i + 1)]
+                for j in range(i + 1):
+                    col[j] += w[j] / sum(w) / (G * 4)
+        want = [sum(col[j] for j in perm_seg[k:k + 2]) for k in range(0, len(perm_seg), 2)]
+        bt = O.true_block_masses(Q, K, 0, 0, s, G, perm_seg, int(res["nblocks"][0, 0, s]), p)
+        assert np.allclose(bt.mass, want, rtol=1e-12, atol=1e-15)
