@@ -342,6 +342,31 @@ def main():
                   "rule": "stop after the first candidate block whose mean relative gain over the tile is < tau"}
         s2o.plan(cfg, Q, K, bufs, filtered=filtered)
 
+    # ranking accuracy of the pooled order on sampled segments (exact
+    # attention mass per candidate block against the plan's kept blocks)
+    ranking = None
+    if args.online_steps > 0:
+        s2o.plan(cfg, Q, K, bufs, filtered=False)
+        S = s2o.num_segments(cfg)
+        rng = np.random.default_rng(5)
+        segs = sorted(set([2, S // 4, S // 2, 3 * S // 4, S - 1] +
+                          [int(x) for x in rng.choice(np.arange(3, S - 1), min(27, max(0, S - 4)), replace=False)]))
+        segs = [x for x in segs if 2 <= x < S]
+        r0, r1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        r0.record(stream)
+        st, _ = s2o.block_truth(cfg, Q, K, bufs["perm"], bufs["nblocks"], segs, with_mass=False)
+        r1.record(stream)
+        torch.cuda.synchronize()
+        if s2o.last_device_error() != 0:
+            raise RuntimeError("device error in the ranking measurement")
+        a = st.cpu().numpy().astype(np.float64)
+        kept, true, both = a[..., 0].sum(), a[..., 1].sum(), a[..., 2].sum()
+        ranking = {"segments": len(segs), "precision": both / kept if kept else 1.0,
+                   "recall": both / true if true else 1.0,
+                   "captured_mass": float(a[..., 3].sum() / a[..., 4].sum()) if a[..., 4].sum() > 0 else 1.0,
+                   "ms": r0.elapsed_time(r1)}
+        s2o.plan(cfg, Q, K, bufs, filtered=filtered)
+
     # end to end through the host-buffer C ABI call (pinned host memory)
     e2e = None
     if args.e2e_steps > 0:
@@ -387,6 +412,7 @@ def main():
             "plan_ms": float(np.mean(plan_ms)), "attention_ms": attn_mean,
             "plan_other": {"kind": "full" if filtered else "filtered", "ms": other_ms},
             "online_stop": online,
+            "ranking": ranking,
             "attention_only_tflops": whole_job_tflops(world, dense, attn_mean),
             "kept_pair_fraction": density,
             "roofline": roofline, "cpu_baseline": cpu, "e2e": e2e, "gpu_launches": launches,

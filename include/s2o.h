@@ -240,6 +240,31 @@ s2o_status s2o_attention_online(const s2o_config* cfg, const uint16_t* Q, const 
                                 int32_t* nblocks_out, s2o_stream_t stream);
 
 /*
+ * s2o_block_truth -- ranking accuracy of the pooled order on sampled segments:
+ * each candidate block's true mass against the plan's choice (the referee
+ * report on the pith.science page: the ranking is never checked against
+ * exact attention).  For sampled segment k and (b, kvh), a block's true mass
+ * is the mean, over the segment's rows and the group's query heads, of the
+ * exact causal softmax probability (over all of [0, i]) of its keys.
+ *   Q, K          device bf16 inputs
+ *   perm, nblocks device, from s2o_plan (every block of the order is read,
+ *                 so a filtered plan's perm is not enough)
+ *   segments      HOST int32 [nsamp], each in [0, S); 1 <= nsamp <= 256
+ *   stats         out, device fp32 [nsamp, B, Hkv, 5]: C(s), blocks with true
+ *                 mass >= tau, blocks in both sets, true mass of the kept
+ *                 blocks, true mass of all candidate blocks
+ *   mass          out, device fp32 [nsamp, B, Hkv, nbmax] or NULL: the true
+ *                 mass of block b of the order; nbmax = |Cand(S-1)| / Bk
+ *   workspace     device scratch of s2o_block_truth_workspace_size() bytes,
+ *                 256-byte aligned (zeroed by the call itself)
+ *   fp32 arithmetic (a measurement).
+ */
+s2o_status s2o_block_truth_workspace_size(const s2o_config* cfg, int32_t nsamp, size_t* bytes);
+s2o_status s2o_block_truth(const s2o_config* cfg, const uint16_t* Q, const uint16_t* K, const int32_t* perm,
+                           const int32_t* nblocks, const int32_t* segments, int32_t nsamp, float* stats,
+                           float* mass, void* workspace, size_t workspace_bytes, s2o_stream_t stream);
+
+/*
  * s2o_prefill_host -- the whole path from HOST buffers: copies Q, K, V to
  * the device arena, plans (s2o_plan_filtered: it returns no perm, and O and
  * C(s) equal those of s2o_plan), runs the attention and copies O back to

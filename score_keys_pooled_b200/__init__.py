@@ -68,6 +68,8 @@ def lib() -> ctypes.CDLL:
         L.s2o_plan_contiguous.argtypes = [_CFG, _P, _P, _P, _P, _P]
         L.s2o_attention.argtypes = [_CFG, _P, _P, _P, _P, _P, _P, ctypes.c_int32, _P]
         L.s2o_attention_online.argtypes = [_CFG, _P, _P, _P, _P, _P, ctypes.c_int32, _P, _P]
+        L.s2o_block_truth_workspace_size.argtypes = [_CFG, ctypes.c_int32, ctypes.POINTER(ctypes.c_size_t)]
+        L.s2o_block_truth.argtypes = [_CFG, _P, _P, _P, _P, _P, ctypes.c_int32, _P, _P, _P, ctypes.c_size_t, _P]
         L.s2o_prefill_arena_size.argtypes = [_CFG, ctypes.c_int32, ctypes.POINTER(ctypes.c_size_t)]
         L.s2o_prefill_host.argtypes = [_CFG, _P, _P, _P, _P, ctypes.c_int32, _P, _P, ctypes.c_size_t, _P]
         L.s2o_status_string.argtypes = [ctypes.c_int]
@@ -75,6 +77,7 @@ def lib() -> ctypes.CDLL:
         L.s2o_last_device_error.argtypes = [_P]
         L.s2o_last_launch_count.restype = ctypes.c_int32
         for name in ("s2o_plan_workspace_size", "s2o_plan", "s2o_plan_filtered", "s2o_plan_noalloc", "s2o_plan_contiguous", "s2o_attention", "s2o_attention_online",
+                     "s2o_block_truth_workspace_size", "s2o_block_truth",
                      "s2o_prefill_arena_size", "s2o_prefill_host", "s2o_last_device_error"):
             getattr(L, name).restype = ctypes.c_int
         _lib = L
@@ -190,6 +193,27 @@ def attention_online(cfg: Config, Q, K, V, perm, O=None, nblocks_out=None, out_d
     _check(lib().s2o_attention_online(ctypes.byref(cfg), _ptr(Q), _ptr(K), _ptr(V), _ptr(perm), _ptr(O), out_dtype,
                                       _ptr(nblocks_out), _stream(stream)), "s2o_attention_online")
     return O, nblocks_out
+
+
+def block_truth(cfg: Config, Q, K, perm, nblocks, segments, with_mass: bool = True, stream=None):
+    """s2o_block_truth on the listed segments; returns (stats [n, B*Hkv, 5],
+    mass [n, B*Hkv, nbmax] or None) as device tensors."""
+    import numpy as np
+    import torch
+    segs = np.ascontiguousarray(np.asarray(segments, dtype=np.int32))
+    n = len(segs)
+    BH = cfg.B * cfg.Hkv
+    nbmax = max(0, 128 * (num_segments(cfg) - 1) - 192) // 64
+    stats = torch.empty(n * BH * 5, dtype=torch.float32, device=Q.device)
+    mass = torch.empty(max(1, n * BH * nbmax), dtype=torch.float32, device=Q.device) if with_mass else None
+    nbytes = ctypes.c_size_t(0)
+    _check(lib().s2o_block_truth_workspace_size(ctypes.byref(cfg), n, ctypes.byref(nbytes)),
+           "s2o_block_truth_workspace_size")
+    ws = torch.empty(nbytes.value, dtype=torch.uint8, device=Q.device)
+    _check(lib().s2o_block_truth(ctypes.byref(cfg), _ptr(Q), _ptr(K), _ptr(perm), _ptr(nblocks),
+                                 segs.ctypes.data, n, _ptr(stats), _ptr(mass), _ptr(ws), ws.numel(),
+                                 _stream(stream)), "s2o_block_truth")
+    return stats.view(n, BH, 5), (mass[:n * BH * nbmax].view(n, BH, nbmax) if with_mass else None)
 
 
 def prefill_host(cfg: Config, Q_host, K_host, V_host, O_host, arena, nblocks_host=None,

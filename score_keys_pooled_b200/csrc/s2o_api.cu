@@ -12,6 +12,7 @@
 #include "seg_sort2.cuh"
 #include "sparse_attn.cuh"
 #include "sparse_attn2.cuh"
+#include "block_truth.cuh"
 
 using namespace s2o;
 
@@ -103,6 +104,8 @@ cudaError_t set_kernel_attributes() {
       e = cudaFuncSetAttribute(k_sparse_attn2<true>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kAttn2Smem);
     if (e == cudaSuccess)
       e = cudaFuncSetAttribute(k_bucket_sort, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kBucketSmem);
+    if (e == cudaSuccess)
+      e = cudaFuncSetAttribute(k_truth_cols, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kTruthSmem);
     if (e == cudaSuccess)
       e = cudaFuncSetAttribute(k_contig_plan, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                (int)(kContigMaxBlocks * sizeof(unsigned long long)));
@@ -346,6 +349,48 @@ s2o_status s2o_attention_online(const s2o_config* cfg, const uint16_t* Q, const 
   if (!encode_rows_map(&tmQ, Q, (uint64_t)cfg->B * cfg->Hq * cfg->N, 128)) return S2O_ERR_CUDA;
   const int64_t ncta = (int64_t)cfg->B * cfg->Hkv * a.S * (G / 2);
   k_sparse_attn2<true><<<(unsigned)ncta, kAttn2Threads, kAttn2Smem, s>>>(a, tmQ);
+  ++t_launches;
+  return launch_status();
+}
+
+s2o_status s2o_block_truth_workspace_size(const s2o_config* cfg, int32_t nsamp, size_t* bytes) {
+  s2o_status st = check_cfg(cfg);
+  if (st != S2O_OK) return st;
+  if (!bytes || nsamp < 1 || nsamp > kTruthMaxSamples) return S2O_ERR_INVALID_ARG;
+  *bytes = round256((size_t)nsamp * cfg->B * cfg->Hkv * (size_t)num_cand(nseg(cfg) - 1) * sizeof(float) + 16);
+  return S2O_OK;
+}
+
+s2o_status s2o_block_truth(const s2o_config* cfg, const uint16_t* Q, const uint16_t* K, const int32_t* perm,
+                           const int32_t* nblocks, const int32_t* segments, int32_t nsamp, float* stats, float* mass,
+                           void* workspace, size_t workspace_bytes, s2o_stream_t stream) {
+  t_launches = 0;
+  s2o_status st = check_cfg(cfg);
+  if (st != S2O_OK) return st;
+  if (!Q || !K || !perm || !nblocks || !segments || !stats || !workspace) return S2O_ERR_INVALID_ARG;
+  if (!aligned16(Q) || !aligned16(K) || !aligned16(perm) || (reinterpret_cast<uintptr_t>(workspace) & 255u))
+    return S2O_ERR_INVALID_ARG;
+  size_t need = 0;
+  st = s2o_block_truth_workspace_size(cfg, nsamp, &need);
+  if (st != S2O_OK) return st;
+  if (workspace_bytes < need) return S2O_ERR_WORKSPACE_TOO_SMALL;
+  const int S = nseg(cfg);
+  TruthSegs segs;
+  for (int k = 0; k < nsamp; ++k) {
+    if (segments[k] < 0 || segments[k] >= S) return S2O_ERR_INVALID_ARG;
+    segs.s[k] = segments[k];
+  }
+  if (set_kernel_attributes() != cudaSuccess) return S2O_ERR_CUDA;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  const int64_t cmaxlen = num_cand(S - 1);
+  if (cudaMemsetAsync(workspace, 0, need, s) != cudaSuccess) return S2O_ERR_CUDA;
+  k_truth_cols<<<dim3(nsamp, cfg->B * cfg->Hq), kTruthThreads, kTruthSmem, s>>>(Q, K, segs,
+                                                                              static_cast<float*>(workspace),
+                                                                              cfg->Hq, cfg->Hkv, cfg->N, cmaxlen);
+  ++t_launches;
+  k_truth_stats<<<dim3(nsamp, cfg->B * cfg->Hkv), 256, 0, s>>>(perm, nblocks, segs, static_cast<float*>(workspace),
+                                                                stats, mass, cfg->B * cfg->Hkv, S, ncand_total(cfg),
+                                                                cmaxlen, (int)(cmaxlen / kBk), (float)cfg->tau);
   ++t_launches;
   return launch_status();
 }

@@ -422,3 +422,54 @@ def test_online_workloads(name):
     segs = sampled_segments(S)[::2] if w.N > 20000 else sampled_segments(S)
     check_online(Q, K, V, cfg, bufs["perm"], out, cout, p, segments=segs, kvheads=[0, w.Hkv - 1],
                  what=f"online {name}")
+
+
+# ---------------------------------------------------------------------------
+# s2o_block_truth: ranking accuracy of the pooled order
+# ---------------------------------------------------------------------------
+
+def check_truth(Q, K, q, k, cfg, bufs, segs, p, kvheads=None, what=""):
+    stats, mass = s2o.block_truth(cfg, q, k, bufs["perm"], bufs["nblocks"], segs)
+    assert s2o.last_launch_count() == 2
+    assert s2o.last_device_error() == 0
+    perm, nb, _, _ = host_plan(cfg, bufs)
+    G = cfg.Hq // cfg.Hkv
+    off = O.candidate_offsets(cfg.N, p)
+    st = stats.cpu().numpy()
+    ms = mass.cpu().numpy()
+    for k, s in enumerate(segs):
+        for b in range(cfg.B):
+            for kvh in (range(cfg.Hkv) if kvheads is None else kvheads):
+                bk = b * cfg.Hkv + kvh
+                bt = O.true_block_masses(Q, K, b, kvh, s, G, perm[b, kvh, off[s]:off[s + 1]], int(nb[b, kvh, s]), p)
+                n = len(bt.mass)
+                assert np.allclose(ms[k, bk, :n], bt.mass, rtol=2e-4, atol=1e-9), f"{what} s={s} bk={bk}"
+                assert int(st[k, bk, 0]) == bt.kept
+                # counts may differ only by blocks whose true mass is within 1e-3 of tau
+                close = int(np.sum(np.abs(bt.mass - p.tau) <= 1e-3 * p.tau))
+                assert abs(int(st[k, bk, 1]) - bt.true) <= close
+                assert abs(int(st[k, bk, 2]) - bt.both) <= close
+                assert st[k, bk, 3] == pytest.approx(bt.captured, rel=2e-4, abs=1e-9)
+                assert st[k, bk, 4] == pytest.approx(bt.total, rel=2e-4, abs=1e-9)
+
+
+@pytest.mark.parametrize("B,Hq,Hkv,N,tau,planted,band", [c for c in SMALL if c[3] >= 640][:4])
+def test_block_truth_small_cases(B, Hq, Hkv, N, tau, planted, band):
+    Q, K, V = synth.generate(B, Hq, Hkv, N, 128, planted=planted, band=band, n_stripe=8, seed=N + 3)
+    cfg = s2o.make_config(B, Hq, Hkv, N, tau=tau)
+    q, k = dev(Q), dev(K)
+    bufs = s2o.plan(cfg, q, k)
+    S = O.num_segments(N, O.Params(tau=tau))
+    check_truth(Q, K, q, k, cfg, bufs, list(range(S)), O.Params(tau=tau), what=f"truth N={N}")
+
+
+@pytest.mark.parametrize("name", ["llama_16k", "llama_128k"])
+def test_block_truth_workloads(name):
+    w = synth.WORKLOADS[name]
+    Q, K, V = synth.generate_workload(w)
+    cfg = s2o.make_config(w.B, w.Hq, w.Hkv, w.N, tau=w.tau)
+    q, k = dev(Q), dev(K)
+    bufs = s2o.plan(cfg, q, k)
+    S = s2o.num_segments(cfg)
+    segs = [2, S // 3, S - 1] if w.N > 20000 else [2, 5, S // 2, S - 1]
+    check_truth(Q, K, q, k, cfg, bufs, segs, O.Params(tau=w.tau), kvheads=[0, w.Hkv - 1], what=name)
