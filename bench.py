@@ -309,7 +309,7 @@ def main():
     achieved = 4.0 * w.d * pairs / (attn_mean * 1e-3) / 1e12
     peak = float(peaks.get("bf16_tflops_sustained", peaks["bf16_tflops"]))
     # DRAM bytes per launch of k_sparse_attn2 from an ncu capture of the 32K
-    # workload (765.5 MB), scaled by the rows processed to the 128K launch;
+    # workload (764.7 MB), scaled by the rows processed to the 128K launch;
     # None for other workloads
     traffic = 3.06e9 if w.name == "llama_128k" else None
     roofline = {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
