@@ -186,38 +186,7 @@ def key_scores(qbar: np.ndarray, Kf: np.ndarray, b: int, kvh: int, e: int) -> np
 
 
 def plan_segment(Qf, Kf, b: int, kvh: int, s: int, G: int, p: Params) -> SegmentPlan:
-    N = Kf.shape[2]
-    e = admissible_end(N, s, p)
-    qbar = pooled_query(Qf, b, kvh, s, G, p)
-    sc = key_scores(qbar, Kf, b, kvh, e)
-    if not np.all(np.isfinite(sc)):
-        raise ValueError("non-finite score")
-    M = float(np.max(sc))
-    Z = float(np.sum(np.exp(sc - M)))
-
-    lo, hi = candidate_range(N, s, p)
-    cand = np.arange(lo, hi, dtype=np.int64)
-    cs = sc[lo:hi]
-    # order by (-s_j, j): lexsort's last key is the primary one
-    order = cand[np.lexsort((cand, -cs))] if hi > lo else cand
-
-    w = np.exp(sc[order] - M) / Z
-    nb = num_blocks(hi - lo, p)
-    masses = np.array([w[k * p.Bk:(k + 1) * p.Bk].sum() for k in range(nb)], dtype=np.float64)
-    C = nb
-    for k in range(nb):
-        if masses[k] < p.tau:
-            C = k
-            break
-
-    tol = NEAR_TIE_REL * float(np.max(np.abs(sc)))
-    srt = sc[order]
-    score_ties = np.nonzero(np.abs(srt[:-1] - srt[1:]) <= tol)[0] if len(srt) > 1 else np.zeros(0, np.int64)
-    mass_ties = np.nonzero(np.abs(masses - p.tau) <= NEAR_TIE_REL * p.tau)[0]
-
-    keep = keep_set(N, s, order, C, p)
-    return SegmentPlan(s=s, qbar=qbar, scores=sc, M=M, Z=Z, order=order, masses=masses, C=C,
-                       score_ties=score_ties, mass_ties=mass_ties, tie_tol=tol, keep=keep)
+    return plan_segment_with_query(pooled_query(Qf, b, kvh, s, G, p), Kf, b, kvh, s, p)
 
 
 def plan(Qf, Kf, p: Params, segments=None):
@@ -415,6 +384,97 @@ def tile_heads(kvh: int, G: int, pair: int) -> list:
     if G % 2 == 0:
         return [kvh * G + 2 * pair, kvh * G + 2 * pair + 1]
     return [kvh * G + pair]
+
+
+# ---------------------------------------------------------------------------
+# Query permutation with finer sub-segments (Q_perm)
+# ---------------------------------------------------------------------------
+
+@dataclass
+class SubPlan:
+    rows: np.ndarray        # [rows] segment rows in Q_perm order (absolute indices)
+    sub_of_row: np.ndarray  # [rows] sub-segment (0 or 1) of each row, in row order
+    plans: list             # [SegmentPlan, SegmentPlan] of the two sub-segments
+
+
+def qperm_segment(Qf, Kf, b: int, kvh: int, s: int, G: int, p: Params) -> SubPlan:
+    """Q_perm (gist.science technical summary, section 1, "Classement par
+    Segment": queries reordered inside the segment by a coarse importance score
+    against a shared guide vector), with finer sub-segments whose kept sets
+    differ.  Guide vector: the segment's pooled query qbar.  Row importance:
+    the mean over the group's heads of q_{h,i} . qbar.  Rows are ordered by
+    importance descending, ties to the lower row; the first Lq/2 rows form
+    sub-segment 0, the others sub-segment 1.  Each sub-segment is planned like
+    a segment (same admissible keys, candidates and rule) with its own pooled
+    query: the mean over its rows and the group's heads.  An empty
+    sub-segment 1 (a segment of at most Lq/2 rows) reuses qbar."""
+    N = Qf.shape[2]
+    r0, r1 = segment_rows(N, s, p)
+    rows = np.arange(r0, r1)
+    qbar = pooled_query(Qf, b, kvh, s, G, p)
+    imp = np.zeros(r1 - r0)
+    for g in range(G):
+        imp += _f64(Qf[b, kvh * G + g, r0:r1]) @ qbar
+    imp /= G
+    order = rows[np.lexsort((rows, -imp))]
+    n0 = min(p.Lq // 2, r1 - r0)
+    groups = [np.sort(order[:n0]), np.sort(order[n0:])]
+    sub_of_row = np.zeros(r1 - r0, dtype=np.int64)
+    sub_of_row[groups[1] - r0] = 1
+    plans = []
+    for grp in groups:
+        if len(grp) == 0:
+            q = qbar
+        else:
+            acc = np.zeros(Qf.shape[3])
+            for g in range(G):
+                acc += _f64(Qf[b, kvh * G + g][grp]).sum(axis=0)
+            q = acc / (G * len(grp))
+        plans.append(plan_segment_with_query(q, Kf, b, kvh, s, p))
+    return SubPlan(rows=order, sub_of_row=sub_of_row, plans=plans)
+
+
+def plan_segment_with_query(qbar: np.ndarray, Kf, b: int, kvh: int, s: int, p: Params) -> SegmentPlan:
+    """plan_segment with a given pooled query (scores, order, masses, stop)."""
+    N = Kf.shape[2]
+    e = admissible_end(N, s, p)
+    sc = key_scores(qbar, Kf, b, kvh, e)
+    if not np.all(np.isfinite(sc)):
+        raise ValueError("non-finite score")
+    M = float(np.max(sc))
+    Z = float(np.sum(np.exp(sc - M)))
+    lo, hi = candidate_range(N, s, p)
+    cand = np.arange(lo, hi, dtype=np.int64)
+    cs = sc[lo:hi]
+    order = cand[np.lexsort((cand, -cs))] if hi > lo else cand
+    w = np.exp(sc[order] - M) / Z
+    nb = num_blocks(hi - lo, p)
+    masses = np.array([w[k * p.Bk:(k + 1) * p.Bk].sum() for k in range(nb)], dtype=np.float64)
+    C = nb
+    for k in range(nb):
+        if masses[k] < p.tau:
+            C = k
+            break
+    tol = NEAR_TIE_REL * float(np.max(np.abs(sc)))
+    srt = sc[order]
+    score_ties = np.nonzero(np.abs(srt[:-1] - srt[1:]) <= tol)[0] if len(srt) > 1 else np.zeros(0, np.int64)
+    mass_ties = np.nonzero(np.abs(masses - p.tau) <= NEAR_TIE_REL * p.tau)[0]
+    keep = keep_set(N, s, order, C, p)
+    return SegmentPlan(s=s, qbar=qbar, scores=sc, M=M, Z=Z, order=order, masses=masses, C=C,
+                       score_ties=score_ties, mass_ties=mass_ties, tie_tol=tol, keep=keep)
+
+
+def attention_qperm_segment(Qf, Kf, Vf, b: int, kvh: int, s: int, G: int, keeps, sub_of_row: np.ndarray,
+                            p: Params) -> np.ndarray:
+    """Each row attends over its own sub-segment's kept set (and [0, i])."""
+    r0, r1 = segment_rows(Qf.shape[2], s, p)
+    out = np.zeros((G, r1 - r0, Qf.shape[3]))
+    for sub in (0, 1):
+        if not np.any(sub_of_row == sub):
+            continue
+        full = attention_segment(Qf, Kf, Vf, b, kvh, s, G, keeps[sub], p)
+        out[:, sub_of_row == sub] = full[:, sub_of_row == sub]
+    return out
 
 
 # ---------------------------------------------------------------------------

@@ -592,3 +592,78 @@ def test_true_masses_brute_force_n16():
         want = [sum(col[j] for j in perm_seg[k:k + 2]) for k in range(0, len(perm_seg), 2)]
         bt = O.true_block_masses(Q, K, 0, 0, s, G, perm_seg, int(res["nblocks"][0, 0, s]), p)
         assert np.allclose(bt.mass, want, rtol=1e-12, atol=1e-15)
+
+
+# ---------------------------------------------------------------------------
+# Q_perm with finer sub-segments
+# ---------------------------------------------------------------------------
+
+def test_qperm_partition_follows_a_known_importance():
+    # rows q_i = c_i u with a shared unit u: qbar = mean(c) u and the importance
+    # of row i is c_i mean(c), so with mean(c) > 0 the rows order by c_i
+    # (ties to the lower row); some c repeat to exercise the tie-break
+    N, d = 512, 64
+    p = O.Params(tau=1e-3)
+    rng = np.random.default_rng(13)
+    u = np.zeros(d); u[3] = 1.0
+    c = rng.integers(1, 40, size=N).astype(np.float32) / 8.0
+    Q = _bits((c[None, None, :, None] * u[None, None, None, :]).repeat(2, axis=1))
+    K = _bits(rng.standard_normal((1, 1, N, d)))
+    for s in (2, 3):
+        r0 = 128 * s
+        rows = np.arange(r0, r0 + 128)
+        want_order = rows[np.lexsort((rows, -c[r0:r0 + 128]))]
+        sp = O.qperm_segment(Q, K, 0, 0, s, 2, p)
+        assert np.array_equal(sp.rows, want_order)
+        assert np.array_equal(np.nonzero(sp.sub_of_row == 0)[0] + r0, np.sort(want_order[:64]))
+        # each sub-segment's pooled query is the mean of its rows (both heads)
+        for sub in (0, 1):
+            grp = np.sort(want_order[64 * sub:64 * (sub + 1)])
+            want_q = float(np.mean(c[grp])) * u
+            assert np.allclose(sp.plans[sub].qbar, want_q, rtol=0, atol=1e-12)
+
+
+def test_qperm_identical_rows_reduce_to_the_segment_plan():
+    # every row of a segment equal: both sub-segments pool to qbar, so their
+    # plans and the outputs equal the unpermuted method
+    N, d = 768, 64
+    p = O.Params(tau=3e-3)
+    rng = np.random.default_rng(14)
+    base = rng.standard_normal((1, 2, N // 128, 1, d))
+    Q = _bits(np.repeat(base, 128, axis=3).reshape(1, 2, N, d))
+    K = _bits(rng.standard_normal((1, 1, N, d)))
+    V = _bits(rng.standard_normal((1, 1, N, d)))
+    for s in range(O.num_segments(N, p)):
+        sp = O.qperm_segment(Q, K, 0, 0, s, 2, p)
+        ref = O.plan_segment(Q, K, 0, 0, s, 2, p)
+        for sub in (0, 1):
+            assert np.array_equal(sp.plans[sub].order, ref.order)
+            assert sp.plans[sub].C == ref.C
+        keeps = [sp.plans[0].keep, sp.plans[1].keep]
+        got = O.attention_qperm_segment(Q, K, V, 0, 0, s, 2, keeps, sp.sub_of_row, p)
+        want = O.attention_segment(Q, K, V, 0, 0, s, 2, ref.keep, p)
+        assert np.max(np.abs(got - want)) <= 1e-12
+
+
+def test_qperm_each_row_uses_its_own_kept_set():
+    # brute force on N = 16 (Lq = 4: sub-segments of 2 rows): each row's
+    # output is plain softmax attention over its own sub-segment's kept keys
+    p = O.Params(Lq=4, Bk=2, n_sink=1, window_prev=4, tau=0.15)
+    rng = np.random.default_rng(15)
+    N, d = 16, 8
+    Q = _bits(rng.standard_normal((1, 1, N, d)) * 1.5)
+    K = _bits(rng.standard_normal((1, 1, N, d)) * 1.5)
+    V = _bits(rng.standard_normal((1, 1, N, d)))
+    Qv, Kv, Vv = O.widen_bf16(Q)[0, 0], O.widen_bf16(K)[0, 0], O.widen_bf16(V)[0, 0]
+    differ = 0
+    for s in range(O.num_segments(N, p)):
+        sp = O.qperm_segment(Q, K, 0, 0, s, 1, p)
+        keeps = [sp.plans[0].keep, sp.plans[1].keep]
+        differ += not np.array_equal(keeps[0], keeps[1])
+        got = O.attention_qperm_segment(Q, K, V, 0, 0, s, 1, keeps, sp.sub_of_row, p)
+        for r, i in enumerate(range(4 * s, 4 * s + 4)):
+            keys = [int(j) for j in keeps[int(sp.sub_of_row[r])] if j <= i]
+            w = [math.exp(float(Qv[i] @ Kv[j]) / math.sqrt(d)) for j in keys]
+            want = sum(wj * Vv[j] for wj, j in zip(w, keys)) / sum(w)
+            assert np.allclose(got[0, r], want, rtol=0, atol=1e-12)
+    assert differ >= 1  # some segment's two sub-segments keep different keys
