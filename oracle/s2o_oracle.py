@@ -44,7 +44,11 @@ the following readings (the GPU library takes the same ones):
     blocks in the plan's order; after each block every row's gain is the
     block's share of the exp-sum the row has processed so far (the block
     included); the tile stops after the first block whose mean gain over its
-    rows is below tau, keeping that block.
+    rows is below tau, keeping that block;
+  * Q_perm (optional): the segment's rows are ordered by the mean over the
+    group's heads of q_i . qbar (the shared guide vector), ties to the lower
+    row; the first Lq/2 rows and the rest form two sub-segments, each planned
+    with its own pooled query; a row attends over its sub-segment's kept set.
 
 All arithmetic is IEEE fp64 on inputs widened exactly from bf16.  Loops are
 plain; numpy's matmul, sort and sum are used as library steps only.  The
