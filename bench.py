@@ -61,6 +61,27 @@ def kept_pairs(nblocks: np.ndarray, N: int, G: int) -> int:
     return total
 
 
+def kept_pairs_qperm(nblocks2: np.ndarray, rowsub: np.ndarray, N: int, G: int) -> int:
+    """kept_pairs for Q_perm: nblocks2 [2, B, Hkv, S]; rowsub [B, Hkv, S, 128]
+    gives each row's sub-segment, whose C(s) counts for that row."""
+    _, B, Hkv, S = nblocks2.shape
+    total = 0
+    for s in range(S):
+        r0 = 128 * s
+        L = min(N, r0 + 128) - r0
+        diag = L * (L + 1) // 2
+        if s == 0:
+            per = np.full((B, Hkv), diag, dtype=np.int64)
+        elif s == 1:
+            per = np.full((B, Hkv), L * 128 + diag, dtype=np.int64)
+        else:
+            n1 = rowsub[:, :, s, :L].astype(np.int64).sum(axis=-1)
+            n0 = L - n1
+            per = L * (64 + 128) + diag + 64 * (n0 * nblocks2[0, :, :, s] + n1 * nblocks2[1, :, :, s])
+        total += int(per.sum()) * G
+    return total
+
+
 def reduce_max_ms(ms: float, dist=None, device="cpu") -> float:
     """Max over ranks of a per-rank time (the slowest rank bounds the job)."""
     if dist is None or not dist.is_initialized() or dist.get_world_size() == 1:
@@ -342,6 +363,31 @@ def main():
                   "rule": "stop after the first candidate block whose mean relative gain over the tile is < tau"}
         s2o.plan(cfg, Q, K, bufs, filtered=filtered)
 
+    # Q_perm: two query sub-segments per segment, each with its own plan
+    qperm = None
+    if args.online_steps > 0 and (w.Hq // w.Hkv) % 2 == 0:
+        for _ in range(2):
+            qp = s2o.plan_qperm(cfg, Q, K)
+            s2o.attention_qperm(cfg, Q, K, V, qp, O)
+        evq = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(args.online_steps)]
+        for e in evq:
+            e[0].record(stream)
+            qp = s2o.plan_qperm(cfg, Q, K)
+            e[1].record(stream)
+            s2o.attention_qperm(cfg, Q, K, V, qp, O)
+            e[2].record(stream)
+        torch.cuda.synchronize()
+        if s2o.last_device_error() != 0:
+            raise RuntimeError("device error in the Q_perm variant")
+        qpl = float(np.mean([e[0].elapsed_time(e[1]) for e in evq]))
+        qat = float(np.mean([e[1].elapsed_time(e[2]) for e in evq]))
+        nb2 = qp["nblocks"].cpu().numpy().reshape(2, w.B, w.Hkv, -1)
+        rsub = qp["rowsub"].cpu().numpy().reshape(w.B, w.Hkv, -1, 128)
+        qperm = {"plan_ms": qpl, "attention_ms": qat, "value": whole_job_tflops(world, dense, qpl + qat),
+                 "kept_pair_fraction": kept_pairs_qperm(nb2, rsub, w.N, w.Hq // w.Hkv) /
+                 (w.B * w.Hq * w.N * (w.N + 1) / 2.0)}
+        del qp
+
     # ranking accuracy of the pooled order on sampled segments (exact
     # attention mass per candidate block against the plan's kept blocks)
     ranking = None
@@ -413,6 +459,7 @@ def main():
             "plan_other": {"kind": "full" if filtered else "filtered", "ms": other_ms},
             "online_stop": online,
             "ranking": ranking,
+            "qperm": qperm,
             "attention_only_tflops": whole_job_tflops(world, dense, attn_mean),
             "kept_pair_fraction": density,
             "roofline": roofline, "cpu_baseline": cpu, "e2e": e2e, "gpu_launches": launches,

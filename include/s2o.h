@@ -240,6 +240,39 @@ s2o_status s2o_attention_online(const s2o_config* cfg, const uint16_t* Q, const 
                                 int32_t* nblocks_out, s2o_stream_t stream);
 
 /*
+ * Q_perm with two query sub-segments (gist.science technical summary,
+ * section 1, "Classement par Segment": the queries of a segment are reordered
+ * by a coarse importance score against a shared guide vector).  The guide is
+ * the segment's pooled query qbar; a row's importance is the mean over the
+ * group's query heads of q_i . qbar; rows are ordered by importance
+ * descending (ties to the lower row), the first 64 form sub-segment 0, the
+ * rest sub-segment 1.  Each sub-segment is planned like a segment (same
+ * admissible keys, candidates and stop rule) with its own pooled query, and a
+ * row attends over its own sub-segment's kept set.
+ *
+ * s2o_plan_qperm -- both sub-segment plans (filtered form: each order is
+ * exact on its first Bk * nblocks entries, the rest is unspecified).
+ *   scores   out, device fp32 [2, B, Hkv, T]   (sub-segment major)
+ *   perm     out, device int32 [2, B, Hkv, T]
+ *   nblocks  out, device int32 [2, B, Hkv, S]
+ *   rowsub   out, device uint8 [B, Hkv, S, 128]: sub-segment of each row of
+ *            each segment (rows past N: 1)
+ *   workspace  device scratch of s2o_plan_qperm_workspace_size() bytes,
+ *            256-byte aligned
+ * s2o_attention_qperm -- the sparse output with each row over its own
+ * sub-segment's kept set; perm, nblocks, rowsub as produced above; other
+ * arguments as s2o_attention.  Requires an even group size Hq/Hkv
+ * (S2O_ERR_UNSUPPORTED_SHAPE otherwise).
+ */
+s2o_status s2o_plan_qperm_workspace_size(const s2o_config* cfg, size_t* bytes);
+s2o_status s2o_plan_qperm(const s2o_config* cfg, const uint16_t* Q, const uint16_t* K, float* scores,
+                          int32_t* perm, int32_t* nblocks, uint8_t* rowsub, void* workspace,
+                          size_t workspace_bytes, s2o_stream_t stream);
+s2o_status s2o_attention_qperm(const s2o_config* cfg, const uint16_t* Q, const uint16_t* K,
+                               const uint16_t* V, const int32_t* perm, const int32_t* nblocks,
+                               const uint8_t* rowsub, void* O, int32_t out_dtype, s2o_stream_t stream);
+
+/*
  * s2o_block_truth -- ranking accuracy of the pooled order on sampled segments:
  * each candidate block's true mass against the plan's choice (the referee
  * report on the pith.science page: the ranking is never checked against

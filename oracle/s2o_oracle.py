@@ -399,6 +399,7 @@ class SubPlan:
     rows: np.ndarray        # [rows] segment rows in Q_perm order (absolute indices)
     sub_of_row: np.ndarray  # [rows] sub-segment (0 or 1) of each row, in row order
     plans: list             # [SegmentPlan, SegmentPlan] of the two sub-segments
+    imp: np.ndarray = field(default=None)  # [rows] importance of each row, in row order
 
 
 def qperm_segment(Qf, Kf, b: int, kvh: int, s: int, G: int, p: Params) -> SubPlan:
@@ -435,7 +436,7 @@ def qperm_segment(Qf, Kf, b: int, kvh: int, s: int, G: int, p: Params) -> SubPla
                 acc += _f64(Qf[b, kvh * G + g][grp]).sum(axis=0)
             q = acc / (G * len(grp))
         plans.append(plan_segment_with_query(q, Kf, b, kvh, s, p))
-    return SubPlan(rows=order, sub_of_row=sub_of_row, plans=plans)
+    return SubPlan(rows=order, sub_of_row=sub_of_row, plans=plans, imp=imp)
 
 
 def plan_segment_with_query(qbar: np.ndarray, Kf, b: int, kvh: int, s: int, p: Params) -> SegmentPlan:

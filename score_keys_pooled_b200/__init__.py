@@ -69,6 +69,9 @@ def lib() -> ctypes.CDLL:
         L.s2o_attention.argtypes = [_CFG, _P, _P, _P, _P, _P, _P, ctypes.c_int32, _P]
         L.s2o_attention_online.argtypes = [_CFG, _P, _P, _P, _P, _P, ctypes.c_int32, _P, _P]
         L.s2o_block_truth_workspace_size.argtypes = [_CFG, ctypes.c_int32, ctypes.POINTER(ctypes.c_size_t)]
+        L.s2o_plan_qperm_workspace_size.argtypes = [_CFG, ctypes.POINTER(ctypes.c_size_t)]
+        L.s2o_plan_qperm.argtypes = [_CFG, _P, _P, _P, _P, _P, _P, _P, ctypes.c_size_t, _P]
+        L.s2o_attention_qperm.argtypes = [_CFG, _P, _P, _P, _P, _P, _P, _P, ctypes.c_int32, _P]
         L.s2o_block_truth.argtypes = [_CFG, _P, _P, _P, _P, _P, ctypes.c_int32, _P, _P, _P, ctypes.c_size_t, _P]
         L.s2o_prefill_arena_size.argtypes = [_CFG, ctypes.c_int32, ctypes.POINTER(ctypes.c_size_t)]
         L.s2o_prefill_host.argtypes = [_CFG, _P, _P, _P, _P, ctypes.c_int32, _P, _P, ctypes.c_size_t, _P]
@@ -77,7 +80,8 @@ def lib() -> ctypes.CDLL:
         L.s2o_last_device_error.argtypes = [_P]
         L.s2o_last_launch_count.restype = ctypes.c_int32
         for name in ("s2o_plan_workspace_size", "s2o_plan", "s2o_plan_filtered", "s2o_plan_noalloc", "s2o_plan_contiguous", "s2o_attention", "s2o_attention_online",
-                     "s2o_block_truth_workspace_size", "s2o_block_truth",
+                     "s2o_block_truth_workspace_size", "s2o_block_truth", "s2o_plan_qperm_workspace_size",
+                     "s2o_plan_qperm", "s2o_attention_qperm",
                      "s2o_prefill_arena_size", "s2o_prefill_host", "s2o_last_device_error"):
             getattr(L, name).restype = ctypes.c_int
         _lib = L
@@ -193,6 +197,36 @@ def attention_online(cfg: Config, Q, K, V, perm, O=None, nblocks_out=None, out_d
     _check(lib().s2o_attention_online(ctypes.byref(cfg), _ptr(Q), _ptr(K), _ptr(V), _ptr(perm), _ptr(O), out_dtype,
                                       _ptr(nblocks_out), _stream(stream)), "s2o_attention_online")
     return O, nblocks_out
+
+
+def plan_qperm(cfg: Config, Q, K, stream=None):
+    """s2o_plan_qperm; returns dict(scores [2*B*Hkv*T], perm, nblocks [2*B*Hkv*S], rowsub [B*Hkv*S*128])."""
+    import torch
+    BH = cfg.B * cfg.Hkv
+    S, T = num_segments(cfg), num_candidates(cfg)
+    dev = Q.device
+    out = dict(scores=torch.empty(2 * BH * T + 4, dtype=torch.float32, device=dev),
+               perm=torch.empty(2 * BH * T + 4, dtype=torch.int32, device=dev),
+               nblocks=torch.empty(2 * BH * S, dtype=torch.int32, device=dev),
+               rowsub=torch.empty(BH * S * 128, dtype=torch.uint8, device=dev))
+    n = ctypes.c_size_t(0)
+    _check(lib().s2o_plan_qperm_workspace_size(ctypes.byref(cfg), ctypes.byref(n)), "s2o_plan_qperm_workspace_size")
+    ws = torch.empty(n.value, dtype=torch.uint8, device=dev)
+    _check(lib().s2o_plan_qperm(ctypes.byref(cfg), _ptr(Q), _ptr(K), _ptr(out["scores"]), _ptr(out["perm"]),
+                                _ptr(out["nblocks"]), _ptr(out["rowsub"]), _ptr(ws), ws.numel(), _stream(stream)),
+           "s2o_plan_qperm")
+    return out
+
+
+def attention_qperm(cfg: Config, Q, K, V, qp, O=None, out_dtype: int = OUT_BF16, stream=None):
+    import torch
+    if O is None:
+        O = torch.empty(Q.shape, dtype=torch.bfloat16 if out_dtype == OUT_BF16 else torch.float32,
+                        device=Q.device)
+    _check(lib().s2o_attention_qperm(ctypes.byref(cfg), _ptr(Q), _ptr(K), _ptr(V), _ptr(qp["perm"]),
+                                     _ptr(qp["nblocks"]), _ptr(qp["rowsub"]), _ptr(O), out_dtype, _stream(stream)),
+           "s2o_attention_qperm")
+    return O
 
 
 def block_truth(cfg: Config, Q, K, perm, nblocks, segments, with_mass: bool = True, stream=None):

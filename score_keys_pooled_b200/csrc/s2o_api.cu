@@ -13,6 +13,7 @@
 #include "sparse_attn.cuh"
 #include "sparse_attn2.cuh"
 #include "block_truth.cuh"
+#include "qperm.cuh"
 
 using namespace s2o;
 
@@ -102,6 +103,9 @@ cudaError_t set_kernel_attributes() {
       e = cudaFuncSetAttribute(k_sparse_attn2<false>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kAttn2Smem);
     if (e == cudaSuccess)
       e = cudaFuncSetAttribute(k_sparse_attn2<true>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kAttn2Smem);
+    if (e == cudaSuccess)
+      e = cudaFuncSetAttribute(k_sparse_attn2<false, true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                               (int)kAttn2Smem);
     if (e == cudaSuccess)
       e = cudaFuncSetAttribute(k_bucket_sort, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kBucketSmem);
     if (e == cudaSuccess)
@@ -205,6 +209,10 @@ s2o_status s2o_plan_workspace_size(const s2o_config* cfg, size_t* bytes) {
   return S2O_OK;
 }
 
+static void launch_plan_core(const s2o_config* cfg, const double* qbar, const uint16_t* K, float* scores,
+                             int32_t* perm, int32_t* nblocks, float* seg_stats, const PlanWs& w, cudaStream_t s,
+                             int filtered);
+
 // the plan's launches; `filtered` sorts only the prefix of each segment's
 // order that the stop rule can reach
 static s2o_status run_plan(const s2o_config* cfg, const uint16_t* Q, const uint16_t* K, float* scores, int32_t* perm,
@@ -223,13 +231,24 @@ static s2o_status run_plan(const s2o_config* cfg, const uint16_t* Q, const uint1
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
   const int S = nseg(cfg);
   const int BH = cfg->B * cfg->Hkv;
-  const int64_t T = ncand_total(cfg);
 
   k_pool<<<dim3(S, BH), 256, 0, s>>>(Q, w.qbar, cfg->Hq, cfg->Hkv, cfg->N, S);
   ++t_launches;
+  launch_plan_core(cfg, w.qbar, K, scores, perm, nblocks, seg_stats, w, s, filtered);
+  return launch_status();
+}
+
+// the plan's stages after the pooled query: scores and (max, sumexp)
+// partials, (M, Z), the order (bucketed sort, global fallback), the stop
+static void launch_plan_core(const s2o_config* cfg, const double* qbar, const uint16_t* K, float* scores,
+                             int32_t* perm, int32_t* nblocks, float* seg_stats, const PlanWs& w, cudaStream_t s,
+                             int filtered) {
+  const int S = nseg(cfg);
+  const int BH = cfg->B * cfg->Hkv;
+  const int64_t T = ncand_total(cfg);
   const int ntiles = (cfg->N + kScoreKeys - 1) / kScoreKeys;
   const int nchunks = (S + kScoreSegs - 1) / kScoreSegs;
-  k_score<<<dim3(ntiles, nchunks, BH), 256, kScoreSmem, s>>>(K, w.qbar, scores, w.part, cfg->Hkv, cfg->N, S, T);
+  k_score<<<dim3(ntiles, nchunks, BH), 256, kScoreSmem, s>>>(K, qbar, scores, w.part, cfg->Hkv, cfg->N, S, T);
   ++t_launches;
   const int nwarps = BH * S;
   k_seg_stats<<<(nwarps * 32 + 255) / 256, 256, 0, s>>>(w.part, w.segM, w.segZ, seg_stats, BH, S);
@@ -247,7 +266,6 @@ static s2o_status run_plan(const s2o_config* cfg, const uint16_t* Q, const uint1
   ++t_launches;
   k_mass_stop<<<BH * S, 256, 0, s>>>(w.sorted, w.segM, w.segZ, w.plen, nblocks, BH, S, T, cfg->tau);
   ++t_launches;
-  return launch_status();
 }
 
 s2o_status s2o_plan(const s2o_config* cfg, const uint16_t* Q, const uint16_t* K, float* scores, int32_t* perm,
@@ -260,6 +278,45 @@ s2o_status s2o_plan_filtered(const s2o_config* cfg, const uint16_t* Q, const uin
                              int32_t* perm, int32_t* nblocks, float* seg_stats, void* workspace,
                              size_t workspace_bytes, s2o_stream_t stream) {
   return run_plan(cfg, Q, K, scores, perm, nblocks, seg_stats, workspace, workspace_bytes, stream, 1);
+}
+
+s2o_status s2o_plan_qperm_workspace_size(const s2o_config* cfg, size_t* bytes) {
+  s2o_status st = check_cfg(cfg);
+  if (st != S2O_OK) return st;
+  if (!bytes) return S2O_ERR_INVALID_ARG;
+  *bytes = plan_layout(cfg, nullptr).bytes + round256((size_t)2 * cfg->B * cfg->Hkv * nseg(cfg) * kD * sizeof(double));
+  return S2O_OK;
+}
+
+s2o_status s2o_plan_qperm(const s2o_config* cfg, const uint16_t* Q, const uint16_t* K, float* scores, int32_t* perm,
+                          int32_t* nblocks, uint8_t* rowsub, void* workspace, size_t workspace_bytes,
+                          s2o_stream_t stream) {
+  t_launches = 0;
+  s2o_status st = check_cfg(cfg);
+  if (st != S2O_OK) return st;
+  if (!Q || !K || !scores || !perm || !nblocks || !rowsub || !workspace) return S2O_ERR_INVALID_ARG;
+  if (!aligned16(Q) || !aligned16(K) || !aligned16(scores) || !aligned16(perm) || !aligned16(nblocks) ||
+      (reinterpret_cast<uintptr_t>(workspace) & 255u))
+    return S2O_ERR_INVALID_ARG;
+  size_t need = 0;
+  s2o_plan_qperm_workspace_size(cfg, &need);
+  if (workspace_bytes < need) return S2O_ERR_WORKSPACE_TOO_SMALL;
+  if (set_kernel_attributes() != cudaSuccess) return S2O_ERR_CUDA;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  const PlanWs w = plan_layout(cfg, workspace);
+  const int S = nseg(cfg);
+  const int BH = cfg->B * cfg->Hkv;
+  const int64_t T = ncand_total(cfg);
+  double* qsub0 = reinterpret_cast<double*>(static_cast<uint8_t*>(workspace) + w.bytes);
+  double* qsub1 = qsub0 + (size_t)BH * S * kD;
+  k_pool<<<dim3(S, BH), 256, 0, s>>>(Q, w.qbar, cfg->Hq, cfg->Hkv, cfg->N, S);
+  ++t_launches;
+  k_qperm<<<dim3(S, BH), kLq, 0, s>>>(Q, w.qbar, qsub0, qsub1, rowsub, cfg->Hq, cfg->Hkv, cfg->N, S);
+  ++t_launches;
+  launch_plan_core(cfg, qsub0, K, scores, perm, nblocks, nullptr, w, s, 1);
+  launch_plan_core(cfg, qsub1, K, scores + (size_t)BH * T, perm + (size_t)BH * T, nblocks + (size_t)BH * S, nullptr,
+                   w, s, 1);
+  return launch_status();
 }
 
 s2o_status s2o_plan_contiguous(const s2o_config* cfg, const float* scores, const float* seg_stats,
@@ -304,7 +361,7 @@ s2o_status s2o_attention(const s2o_config* cfg, const uint16_t* Q, const uint16_
     a.B = cfg->B; a.Hq = cfg->Hq; a.Hkv = cfg->Hkv; a.N = cfg->N; a.S = nseg(cfg);
     a.T = ncand_total(cfg);
     a.out_f32 = out_dtype == S2O_OUT_F32;
-    a.tau = 0.f; a.cout = nullptr;
+    a.tau = 0.f; a.cout = nullptr; a.perm1 = nullptr; a.nblocks1 = nullptr; a.rowsub = nullptr;
     CUtensorMap tmQ;
     if (!encode_rows_map(&tmQ, Q, (uint64_t)cfg->B * cfg->Hq * cfg->N, 128))
       return S2O_ERR_CUDA;
@@ -344,7 +401,7 @@ s2o_status s2o_attention_online(const s2o_config* cfg, const uint16_t* Q, const 
   a.B = cfg->B; a.Hq = cfg->Hq; a.Hkv = cfg->Hkv; a.N = cfg->N; a.S = nseg(cfg);
   a.T = ncand_total(cfg);
   a.out_f32 = out_dtype == S2O_OUT_F32;
-  a.tau = (float)cfg->tau; a.cout = nblocks_out;
+  a.tau = (float)cfg->tau; a.cout = nblocks_out; a.perm1 = nullptr; a.nblocks1 = nullptr; a.rowsub = nullptr;
   CUtensorMap tmQ;
   if (!encode_rows_map(&tmQ, Q, (uint64_t)cfg->B * cfg->Hq * cfg->N, 128)) return S2O_ERR_CUDA;
   const int64_t ncta = (int64_t)cfg->B * cfg->Hkv * a.S * (G / 2);
@@ -391,6 +448,38 @@ s2o_status s2o_block_truth(const s2o_config* cfg, const uint16_t* Q, const uint1
   k_truth_stats<<<dim3(nsamp, cfg->B * cfg->Hkv), 256, 0, s>>>(perm, nblocks, segs, static_cast<float*>(workspace),
                                                                 stats, mass, cfg->B * cfg->Hkv, S, ncand_total(cfg),
                                                                 cmaxlen, (int)(cmaxlen / kBk), (float)cfg->tau);
+  ++t_launches;
+  return launch_status();
+}
+
+s2o_status s2o_attention_qperm(const s2o_config* cfg, const uint16_t* Q, const uint16_t* K, const uint16_t* V,
+                               const int32_t* perm, const int32_t* nblocks, const uint8_t* rowsub, void* O,
+                               int32_t out_dtype, s2o_stream_t stream) {
+  t_launches = 0;
+  s2o_status st = check_cfg(cfg);
+  if (st != S2O_OK) return st;
+  if (!Q || !K || !V || !perm || !nblocks || !rowsub || !O) return S2O_ERR_INVALID_ARG;
+  if (out_dtype != S2O_OUT_BF16 && out_dtype != S2O_OUT_F32) return S2O_ERR_INVALID_ARG;
+  if (!aligned16(Q) || !aligned16(K) || !aligned16(V) || !aligned16(O) || !aligned16(perm)) return S2O_ERR_INVALID_ARG;
+  const int G = cfg->Hq / cfg->Hkv;
+  if (G % 2 != 0 || (int64_t)cfg->B * cfg->Hq * cfg->N >= (int64_t)INT32_MAX) return S2O_ERR_UNSUPPORTED_SHAPE;
+  if (set_kernel_attributes() != cudaSuccess) return S2O_ERR_CUDA;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  const int64_t T = ncand_total(cfg);
+  const size_t BH = (size_t)cfg->B * cfg->Hkv;
+  Attn2Args a;
+  a.Q = Q; a.K = K; a.V = V; a.perm = perm; a.nblocks = nblocks; a.O = O;
+  a.B = cfg->B; a.Hq = cfg->Hq; a.Hkv = cfg->Hkv; a.N = cfg->N; a.S = nseg(cfg);
+  a.T = T;
+  a.out_f32 = out_dtype == S2O_OUT_F32;
+  a.tau = 0.f; a.cout = nullptr;
+  a.perm1 = perm + BH * T;
+  a.nblocks1 = nblocks + BH * a.S;
+  a.rowsub = rowsub;
+  CUtensorMap tmQ;
+  if (!encode_rows_map(&tmQ, Q, (uint64_t)cfg->B * cfg->Hq * cfg->N, 128)) return S2O_ERR_CUDA;
+  const int64_t ncta = (int64_t)cfg->B * cfg->Hkv * a.S * (G / 2);
+  k_sparse_attn2<false, true><<<(unsigned)ncta, kAttn2Threads, kAttn2Smem, s>>>(a, tmQ);
   ++t_launches;
   return launch_status();
 }

@@ -188,11 +188,18 @@ struct Attn2Args {
   // blocks processed per query head go to cout [B, Hq, S]
   float tau;
   int32_t* cout;
+  // Q_perm (k_sparse_attn2<false, true>): the segment's rows form two
+  // sub-segments (rowsub [B, Hkv, S, 128]) with their own orders and stops;
+  // the key walk covers sub-segment 0's kept blocks (perm, nblocks) then
+  // sub-segment 1's (perm1, nblocks1), each masked for the other's rows
+  const int32_t* perm1;
+  const int32_t* nblocks1;
+  const uint8_t* rowsub;
 };
 
-// ONLINE selects the run-time stop; the planned-stop kernel is compiled
-// without any of its code
-template <bool ONLINE>
+// ONLINE selects the run-time stop, QPERM the two query sub-segments; the
+// planned-stop kernel is compiled without any of their code
+template <bool ONLINE, bool QPERM = false>
 __global__ void __launch_bounds__(kAttn2Threads, 1)
     k_sparse_attn2(Attn2Args a, const __grid_constant__ CUtensorMap tmQ) {
   extern __shared__ uint8_t smem_raw[];
@@ -221,6 +228,15 @@ __global__ void __launch_bounds__(kAttn2Threads, 1)
   if (C < 0 || C > cmax) {
     if (tid == 0) set_error(kErrBadPlan);
     C = C < 0 ? 0 : cmax;
+  }
+  const int C0 = C;  // blocks of the first list (Q_perm: sub-segment 0)
+  if (QPERM) {
+    int C1 = a.nblocks1[(size_t)bk * a.S + s];
+    if (C1 < 0 || C1 > cmax) {
+      if (tid == 0) set_error(kErrBadPlan);
+      C1 = C1 < 0 ? 0 : cmax;
+    }
+    C = C0 + C1;
   }
   const Walk2 wk = make_walk2(s, a.N, C);
   const int ntiles = (wk.nb + 1) / 2;
@@ -279,7 +295,12 @@ __global__ void __launch_bounds__(kAttn2Threads, 1)
       const int kind = walk2_block(wk, s, 2 * t + (lane >> 4), j0);
       const int rr = (4 * lane) & 63;
       if (kind == 2) {
-        const int4 v = *reinterpret_cast<const int4*>(pseg + kBk * j0 + rr);
+        const int32_t* ps = pseg;
+        if (QPERM && j0 >= C0) {
+          ps = a.perm1 + (size_t)bk * a.T + cand_offset(s);
+          j0 -= C0;
+        }
+        const int4 v = *reinterpret_cast<const int4*>(ps + kBk * j0 + rr);
         y[0] = v.x; y[1] = v.y; y[2] = v.z; y[3] = v.w;
       } else {
 #pragma unroll
@@ -460,6 +481,7 @@ __global__ void __launch_bounds__(kAttn2Threads, 1)
     const int r = tid & 127;                // row in the segment
     const int row = row0 + r;
     const uint32_t lane_base = (uint32_t)((warp & 3) * 32) << 16;
+    const int my_sub = QPERM ? (int)a.rowsub[((size_t)bk * a.S + s) * kLq + r] : 0;
     const uint32_t tS = tmem + col_s(qi) + lane_base;
     const uint32_t tO = tmem + col_o(qi) + lane_base;
     const float sl2 = 1.4426950408889634f * 0.08838834764831845f;  // log2(e) / sqrt(d)
@@ -476,7 +498,8 @@ __global__ void __launch_bounds__(kAttn2Threads, 1)
       // key k of the chunk is visible iff k <= lim
       int j0;
       const int kind = walk2_block(wk, s, c, j0);
-      const int lim = kind == 3 ? -1 : (kind == 0 ? row - j0 : kBk);
+      int lim = kind == 3 ? -1 : (kind == 0 ? row - j0 : kBk);
+      if (QPERM && kind == 2 && (j0 >= C0 ? 1 : 0) != my_sub) lim = -1;  // the other sub-segment's block
       if (!warp_wait(bar(kBarSFull + qi), (uint32_t)(c & 1))) { ok = false; break; }
       tc_fence_after();
       float x[kBk];

@@ -473,3 +473,93 @@ def test_block_truth_workloads(name):
     S = s2o.num_segments(cfg)
     segs = [2, S // 3, S - 1] if w.N > 20000 else [2, 5, S // 2, S - 1]
     check_truth(Q, K, q, k, cfg, bufs, segs, O.Params(tau=w.tau), kvheads=[0, w.Hkv - 1], what=name)
+
+
+# ---------------------------------------------------------------------------
+# Q_perm: two query sub-segments per segment
+# ---------------------------------------------------------------------------
+
+def check_qperm(Q, K, V, cfg, qp, out, segments=None, kvheads=None, what=""):
+    p = O.Params(tau=cfg.tau)
+    G = cfg.Hq // cfg.Hkv
+    BH = cfg.B * cfg.Hkv
+    S, T = s2o.num_segments(cfg), s2o.num_candidates(cfg)
+    off = O.candidate_offsets(cfg.N, p)
+    perm = qp["perm"][:2 * BH * T].cpu().numpy().reshape(2, cfg.B, cfg.Hkv, T)
+    nb = qp["nblocks"].cpu().numpy().reshape(2, cfg.B, cfg.Hkv, S)
+    rs = qp["rowsub"].cpu().numpy().reshape(cfg.B, cfg.Hkv, S, 128)
+    got = out.float().cpu().numpy()
+    swaps = flips = moved = 0
+    for b in range(cfg.B):
+        for kvh in (range(cfg.Hkv) if kvheads is None else kvheads):
+            for s in (range(S) if segments is None else segments):
+                sp = O.qperm_segment(Q, K, b, kvh, s, G, p)
+                r0, r1 = O.segment_rows(cfg.N, s, p)
+                gsub = rs[b, kvh, s, :r1 - r0].astype(np.int64)
+                if not np.array_equal(gsub, sp.sub_of_row):
+                    # only rows tied in importance with the boundary may move
+                    order = np.sort(sp.imp)[::-1]
+                    cut = order[min(64, r1 - r0) - 1]
+                    diff = np.nonzero(gsub != sp.sub_of_row)[0]
+                    assert np.all(np.abs(sp.imp[diff] - cut) <= 1e-12 * np.max(np.abs(sp.imp))), f"{what} s={s}"
+                    moved += len(diff)
+                    continue  # the sub-segment plans then differ legitimately
+                for sub in (0, 1):
+                    sw, fl = parity.compare_segment_plan(perm[sub, b, kvh, off[s]:off[s + 1]], int(nb[sub, b, kvh, s]),
+                                                         sp.plans[sub], p, prefix_only=True)
+                    swaps += sw
+                    flips += fl
+                keeps = [O.keep_set(cfg.N, s, perm[sub, b, kvh, off[s]:off[s + 1]], int(nb[sub, b, kvh, s]), p)
+                         for sub in (0, 1)]
+                ref = O.attention_qperm_segment(Q, K, V, b, kvh, s, G, keeps, gsub, p)
+                parity.assert_output_close(got[b, kvh * G:(kvh + 1) * G, r0:r1], ref, f"{what} b={b} kvh={kvh} s={s}")
+    parity.log_near_ties({"case": what, "qperm": True, "swapped_positions": swaps, "C_flips": flips,
+                          "rows_moved": moved})
+
+
+@pytest.mark.parametrize("B,Hq,Hkv,N,tau,planted,band", ONLINE_SMALL)
+def test_qperm_small_cases(B, Hq, Hkv, N, tau, planted, band):
+    Q, K, V = synth.generate(B, Hq, Hkv, N, 128, planted=planted, band=band, n_stripe=8, seed=N + 11)
+    cfg = s2o.make_config(B, Hq, Hkv, N, tau=tau)
+    q, k, v = dev(Q), dev(K), dev(V)
+    qp = s2o.plan_qperm(cfg, q, k)
+    assert s2o.last_launch_count() >= 12
+    out = s2o.attention_qperm(cfg, q, k, v, qp)
+    assert s2o.last_launch_count() == 1
+    assert s2o.last_device_error() == 0
+    check_qperm(Q, K, V, cfg, qp, out, what=f"qperm small N={N}")
+
+
+def test_qperm_identical_rows_equal_the_plain_path():
+    # every row of a segment equal in every head: both sub-segments pool to
+    # the segment's query, so plans and output equal the plain method's
+    rng = np.random.default_rng(31)
+    B, Hq, Hkv, N = 1, 4, 2, 1024
+    base = rng.standard_normal((B, Hq, N // 128, 1, 128)).astype(np.float32)
+    Q = synth.to_bf16_bits(np.repeat(base, 128, axis=3).reshape(B, Hq, N, 128))
+    _, K, V = synth.generate(B, Hq, Hkv, N, 128, planted=True, band=True, n_stripe=8, seed=31)
+    cfg = s2o.make_config(B, Hq, Hkv, N, tau=3e-3)
+    q, k, v = dev(Q), dev(K), dev(V)
+    qp = s2o.plan_qperm(cfg, q, k)
+    out = s2o.attention_qperm(cfg, q, k, v, qp)
+    bufs = s2o.plan(cfg, q, k)
+    ref = s2o.attention(cfg, q, k, v, bufs["perm"], bufs["nblocks"])
+    assert s2o.last_device_error() == 0
+    S = s2o.num_segments(cfg)
+    nb = qp["nblocks"].view(2, -1)
+    assert torch.equal(nb[0], bufs["nblocks"]) and torch.equal(nb[1], bufs["nblocks"])
+    assert torch.equal(out, ref)
+
+
+@pytest.mark.parametrize("name", ["llama_16k", "llama_128k"])
+def test_qperm_workloads(name):
+    w = synth.WORKLOADS[name]
+    Q, K, V = synth.generate_workload(w)
+    cfg = s2o.make_config(w.B, w.Hq, w.Hkv, w.N, tau=w.tau)
+    q, k, v = dev(Q), dev(K), dev(V)
+    qp = s2o.plan_qperm(cfg, q, k)
+    out = s2o.attention_qperm(cfg, q, k, v, qp)
+    assert s2o.last_device_error() == 0
+    S = s2o.num_segments(cfg)
+    segs = sampled_segments(S)[::2] if w.N > 20000 else sampled_segments(S)
+    check_qperm(Q, K, V, cfg, qp, out, segments=segs, kvheads=[0, w.Hkv - 1], what=f"qperm {name}")
