@@ -67,9 +67,15 @@ __global__ void __launch_bounds__(256) k_pool(const uint16_t* __restrict__ Q, do
 // rounded once to fp32.  (fp32 accumulation of these 128-term dots errs by
 // ~1e-6 relative when the terms share a sign, the width of the near-tie band
 // the importance order is checked against.)
-// The d = 128 reduction runs in two halves of 64 so that the transposed key
-// tile (fp64) and pooled queries (fp64) fit twice per SM.  Thread (tk, ts)
-// accumulates keys 2 tk + 32 a + {0, 1} (a < 4) x segments ts + 16 b (b < 4).
+// The products run on the fp64 tensor path (mma.sync m8n8k4): each warp owns
+// 16 segments x 64 keys (2 x 8 accumulator tiles), and its operand fragments
+// are reused across 256 multiply-adds per instruction, where scalar fp64 FMAs
+// were bound by shared-memory reads.  The d = 128 reduction runs in two
+// halves of 64 so that the key tile and the pooled queries (fp64, rows padded
+// to 68 doubles: the fragment pattern is then conflict-free) fit twice per
+// SM.  The sums are then staged in shared memory for the epilogue, where
+// thread (tk, ts) takes keys 2 tk + 32 a + {0, 1} (a < 4) x segments
+// ts + 16 b (b < 4).
 // Outputs:
 //   scores[bk][off(s) + j - 64] for candidate keys j of segment s
 //   part[bk][s][t] = (max over the tile's admissible keys,
@@ -77,9 +83,18 @@ __global__ void __launch_bounds__(256) k_pool(const uint16_t* __restrict__ Q, do
 // ---------------------------------------------------------------------------
 constexpr int kScoreKeys = 128;
 constexpr int kScoreSegs = 64;
-constexpr int kScoreHalf = 64;  // d per pass
-constexpr int kQtStride = kScoreSegs + 2;  // padded rows: the transposed fill is conflict-free
-constexpr size_t kScoreSmem = sizeof(double) * (kScoreHalf * kScoreKeys + kScoreHalf * kQtStride);
+constexpr int kScoreHalf = 64;       // d per pass
+constexpr int kScoreStride = 68;     // padded rows of the fp64 operand tiles
+constexpr int kStageStride = kScoreKeys + 2;  // epilogue staging [64 segs][128 keys], padded
+constexpr size_t kScoreSmem = sizeof(double) * (kScoreKeys * kScoreStride + kScoreSegs * kScoreStride);
+static_assert(kScoreSegs * kStageStride <= kScoreKeys * kScoreStride + kScoreSegs * kScoreStride,
+              "staging must fit in the operand tiles");
+
+__device__ __forceinline__ void dmma_8x8x4(double& c0, double& c1, double a, double b) {
+  asm volatile("mma.sync.aligned.m8n8k4.row.col.f64.f64.f64.f64 {%0, %1}, {%2}, {%3}, {%0, %1};\n"
+               : "+d"(c0), "+d"(c1)
+               : "d"(a), "d"(b));
+}
 
 __global__ void __launch_bounds__(256, 2) k_score(const uint16_t* __restrict__ K, const double* __restrict__ qbar,
                                                  float* __restrict__ scores, float2* __restrict__ part,
@@ -92,59 +107,77 @@ __global__ void __launch_bounds__(256, 2) k_score(const uint16_t* __restrict__ K
   if (s_hi - 1 < t) return;
 
   extern __shared__ double smd[];
-  double* Kt = smd;                               // [64 d][128 keys]
-  double* Qt = smd + kScoreHalf * kScoreKeys;     // [64 d][64 segs], rows padded to kQtStride
+  double* Ks = smd;                                // [128 keys][64 d], rows of kScoreStride
+  double* Qs = smd + kScoreKeys * kScoreStride;    // [64 segs][64 d], rows of kScoreStride
   const int tid = threadIdx.x;
-  const int tk = tid & 15;
-  const int ts = tid >> 4;
+  const int lane = tid & 31, warp = tid >> 5;
   const uint16_t* Kb = K + (size_t)bk * N * kD;
   const double* qb = qbar + (size_t)bk * S * kD;
+  // this warp's block: segments m0 .. m0+15, keys n0 .. n0+63
+  const int m0 = 16 * (warp & 3), n0 = 64 * (warp >> 2);
+  const int fr = lane >> 2, fc = lane & 3;  // fragment row / column of this lane
 
-  double acc[8][4];
+  double c[2][8][2];
 #pragma unroll
-  for (int a = 0; a < 8; ++a)
+  for (int mt = 0; mt < 2; ++mt)
 #pragma unroll
-    for (int q = 0; q < 4; ++q) acc[a][q] = 0.0;
+    for (int nt = 0; nt < 8; ++nt) c[mt][nt][0] = c[mt][nt][1] = 0.0;
 
   for (int half = 0; half < 2; ++half) {
     if (half) __syncthreads();
-    // key tile half -> fp64, transposed; keys >= N are zero (never admissible)
+    // key tile half -> fp64, row-major; keys >= N are zero (never admissible)
     for (int q = tid; q < kScoreKeys * 8; q += 256) {
-      const int key = q & (kScoreKeys - 1), c = q >> 7;  // c: 16-byte chunk 0..7 of this half
+      const int key = q >> 3, cch = q & 7;  // cch: 16-byte chunk 0..7 of this half
       const int j = t * kScoreKeys + key;
       uint4 w = make_uint4(0, 0, 0, 0);
-      if (j < N) w = *reinterpret_cast<const uint4*>(Kb + (size_t)j * kD + half * kScoreHalf + 8 * c);
+      if (j < N) w = *reinterpret_cast<const uint4*>(Kb + (size_t)j * kD + half * kScoreHalf + 8 * cch);
       if (bf16x2_nonfinite(w.x) | bf16x2_nonfinite(w.y) | bf16x2_nonfinite(w.z) | bf16x2_nonfinite(w.w))
         set_error(kErrNonFinite);
-      double* col = Kt + (8 * c) * kScoreKeys + key;
-      col[0 * kScoreKeys] = bf16_lo(w.x); col[1 * kScoreKeys] = bf16_hi(w.x);
-      col[2 * kScoreKeys] = bf16_lo(w.y); col[3 * kScoreKeys] = bf16_hi(w.y);
-      col[4 * kScoreKeys] = bf16_lo(w.z); col[5 * kScoreKeys] = bf16_hi(w.z);
-      col[6 * kScoreKeys] = bf16_lo(w.w); col[7 * kScoreKeys] = bf16_hi(w.w);
+      double* row = Ks + key * kScoreStride + 8 * cch;
+      row[0] = bf16_lo(w.x); row[1] = bf16_hi(w.x);
+      row[2] = bf16_lo(w.y); row[3] = bf16_hi(w.y);
+      row[4] = bf16_lo(w.z); row[5] = bf16_hi(w.z);
+      row[6] = bf16_lo(w.w); row[7] = bf16_hi(w.w);
     }
     for (int q = tid; q < kScoreSegs * kScoreHalf; q += 256) {
       const int seg = q / kScoreHalf, dd = q % kScoreHalf;
       const int s = s_lo + seg;
-      Qt[dd * kQtStride + seg] = (s < S) ? qb[(size_t)s * kD + half * kScoreHalf + dd] : 0.0;
+      Qs[seg * kScoreStride + dd] = (s < S) ? qb[(size_t)s * kD + half * kScoreHalf + dd] : 0.0;
     }
     __syncthreads();
 #pragma unroll 2
-    for (int dd = 0; dd < kScoreHalf; ++dd) {
-      double kk[8], qq[4];
+    for (int k0 = 0; k0 < kScoreHalf; k0 += 4) {
+      double a[2], bb[8];
 #pragma unroll
-      for (int a = 0; a < 4; ++a) {  // keys 2 tk + 32 a and 2 tk + 32 a + 1, one 16-byte load
-        const double2 k2 = *reinterpret_cast<const double2*>(Kt + dd * kScoreKeys + 2 * tk + 32 * a);
-        kk[2 * a] = k2.x;
-        kk[2 * a + 1] = k2.y;
-      }
+      for (int mt = 0; mt < 2; ++mt) a[mt] = Qs[(m0 + 8 * mt + fr) * kScoreStride + k0 + fc];
 #pragma unroll
-      for (int q = 0; q < 4; ++q) qq[q] = Qt[dd * kQtStride + ts + 16 * q];
+      for (int nt = 0; nt < 8; ++nt) bb[nt] = Ks[(n0 + 8 * nt + fr) * kScoreStride + k0 + fc];
 #pragma unroll
-      for (int a = 0; a < 8; ++a)
+      for (int mt = 0; mt < 2; ++mt)
 #pragma unroll
-        for (int q = 0; q < 4; ++q) acc[a][q] = fma(kk[a], qq[q], acc[a][q]);
+        for (int nt = 0; nt < 8; ++nt) dmma_8x8x4(c[mt][nt][0], c[mt][nt][1], a[mt], bb[nt]);
     }
   }
+  // stage the sums: stg[seg][key] (accumulator element i of tile (mt, nt) is
+  // segment m0 + 8 mt + fr, key n0 + 8 nt + 2 fc + i)
+  __syncthreads();
+  double* stg = smd;
+#pragma unroll
+  for (int mt = 0; mt < 2; ++mt)
+#pragma unroll
+    for (int nt = 0; nt < 8; ++nt) {
+      double* dst = stg + (m0 + 8 * mt + fr) * kStageStride + n0 + 8 * nt + 2 * fc;
+      dst[0] = c[mt][nt][0];
+      dst[1] = c[mt][nt][1];
+    }
+  __syncthreads();
+  const int tk = tid & 15;
+  const int ts = tid >> 4;
+  double acc[8][4];
+#pragma unroll
+  for (int aa = 0; aa < 8; ++aa)
+#pragma unroll
+    for (int q = 0; q < 4; ++q) acc[aa][q] = stg[(ts + 16 * q) * kStageStride + 2 * tk + 32 * (aa >> 1) + (aa & 1)];
 
   float* sc_bk = scores + (size_t)bk * T;
   float2* part_bk = part + (size_t)bk * S * S;

@@ -111,7 +111,7 @@ __global__ void __launch_bounds__(kBucketThreads) k_bucket_plan(const float* __r
   __shared__ float red[64];
   __shared__ int flag;
   __shared__ uint8_t bin2bkt[kNumBins];  // bucket id of each bin (< kMaxBuckets = 256)
-  __shared__ uint16_t wcnt[kSortWarps][kMaxBuckets];
+  __shared__ uint32_t wcnt[kMaxBuckets][kSortWarps + 1];  // [bucket][warp] counts, then ranks (padded rows)
   __shared__ int cursor[kMaxBuckets];
   __shared__ int bin_cut;  // first bin left out of the order (filtered form)
   const int q = blockIdx.x;
@@ -246,6 +246,7 @@ __global__ void __launch_bounds__(kBucketThreads) k_bucket_plan(const float* __r
   for (int e = 0; e < 2; ++e)
     if (end_id[e] >= 0) myslot[end_id[e]].count = end_rank[e] - myslot[end_id[e]].base;
   // stable multisplit into the buckets, 1024 elements per step in index order
+  // (two block barriers per step)
   bin2bkt[2 * tid] = (uint8_t)(st0 / kBucketHalf);
   bin2bkt[2 * tid + 1] = (uint8_t)(st1 / kBucketHalf);
   __syncthreads();
@@ -260,38 +261,40 @@ __global__ void __launch_bounds__(kBucketThreads) k_bucket_plan(const float* __r
   const uint32_t lt_mask = (1u << lane) - 1u;
   uint32_t* skey = stage_key + base;
   uint32_t* sval = stage_val + base;
+  const int nbk = min(kMaxBuckets, my_slots);  // bucket ids in use are below this
   for (int t0 = 0; t0 < n; t0 += kBucketThreads) {
     const int i = t0 + tid;
     const float x = i < n ? sc[i] : 0.f;
     const int bin = score_bin(x, hi, scale);
     const bool valid = i < n && bin < bcut;
     const uint32_t d = valid ? bin2bkt[bin] : 0u;
-    for (int k = lane; k < kMaxBuckets; k += 32) wcnt[warp][k] = 0;
+    __syncwarp();
+    for (int k = lane; k < nbk; k += 32) wcnt[k][warp] = 0;
     __syncwarp();
     const uint32_t peers = __match_any_sync(0xffffffffu, valid ? d : 1024u + lane);
     const uint32_t rank = __popc(peers & lt_mask);
-    if (valid && (__ffs(peers) - 1) == lane) wcnt[warp][d] = (uint16_t)__popc(peers);
+    if (valid && (__ffs(peers) - 1) == lane) wcnt[d][warp] = __popc(peers);
     __syncthreads();
-    if (tid < kMaxBuckets) {
-      int run = cursor[tid];
-      for (int w2 = 0; w2 < kSortWarps; ++w2) {
-        const int c = wcnt[w2][tid];
-        wcnt[w2][tid] = (uint16_t)(run - cursor[tid]);
-        run += c;
+    // per bucket, one warp scans the 32 warps' counts across its lanes: the
+    // counts become absolute ranks and the bucket's cursor advances
+    for (int db = warp; db < nbk; db += kSortWarps) {
+      const uint32_t v = wcnt[db][lane];
+      uint32_t incl = v;
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        const uint32_t y = __shfl_up_sync(0xffffffffu, incl, o);
+        if (lane >= o) incl += y;
       }
-      // offsets within this step are relative to the bucket cursor; the
-      // cursor itself advances after everyone has read it
-      hist[tid] = run;
+      const uint32_t cur = (uint32_t)cursor[db];
+      wcnt[db][lane] = cur + incl - v;
+      if (lane == 31) cursor[db] = (int)(cur + incl);
     }
     __syncthreads();
     if (valid) {
-      const int pos = cursor[d] + wcnt[warp][d] + (int)rank;
+      const uint32_t pos = wcnt[d][warp] + rank;
       skey[pos] = desc_key(x);
       sval[pos] = (uint32_t)i;
     }
-    __syncthreads();
-    if (tid < kMaxBuckets) cursor[tid] = hist[tid];
-    __syncthreads();
   }
   if (tid == 0) mode[(size_t)bk * S + s] = kModeBuckets;
 }
