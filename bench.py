@@ -189,6 +189,14 @@ def cpu_oracle_sample(Q, K, V, tau, seconds=15.0):
     return flops / dt / 1e12, sample, dt
 
 
+def bench_config(w, world: int, plan: str) -> dict:
+    """The workload description both arms print."""
+    return {"workload": w.name, "B": w.B, "Hq": w.Hq, "Hkv": w.Hkv, "N": w.N, "d": w.d, "tau": w.tau,
+            "global_batch": w.B * world, "seq_len": w.N, "parallelism": f"independent x{world}",
+            "l2": "inputs larger than L2 (Q alone is 1 GiB)" if w.N >= 131072 else "inputs per step exceed L2",
+            "plan": plan}
+
+
 def reference_arm(args, w, world, rank):
     """The CPU oracle as the reference implementation, rank 0 only."""
     if rank != 0:
@@ -208,7 +216,7 @@ def reference_arm(args, w, world, rank):
         "impl": "reference", "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1000.0 * total / max(1, args.steps),
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-        "config": {"workload": w.name, "B": w.B, "Hq": w.Hq, "Hkv": w.Hkv, "N": w.N, "d": w.d, "tau": w.tau},
+        "config": bench_config(w, world, args.plan),
         "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": 1, "kind": "oracle", "sample": sample},
         "e2e": {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }
@@ -452,9 +460,7 @@ def main():
             "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak",
             "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
-            "config": {"workload": w.name, "B": w.B, "Hq": w.Hq, "Hkv": w.Hkv, "N": w.N, "d": w.d, "tau": w.tau,
-                       "global_batch": w.B * world, "seq_len": w.N, "parallelism": f"independent x{world}",
-                       "l2": "inputs larger than L2 (Q alone is 1 GiB)", "plan": args.plan},
+            "config": bench_config(w, world, args.plan),
             "plan_ms": float(np.mean(plan_ms)), "attention_ms": attn_mean,
             "plan_other": {"kind": "full" if filtered else "filtered", "ms": other_ms},
             "online_stop": online,
