@@ -46,6 +46,8 @@ constexpr int kBucketThreads = 1024;          // planner CTA
 constexpr int kSorterThreads = 512;           // bucket-sorter CTA (two per SM)
 constexpr int kSorterWarps = kSorterThreads / 32;
 constexpr int kMaxBuckets = 256;              // bucket ids per segment (N <= 2^19)
+constexpr int kPlanRounds = 4;                // elements per planner thread and multisplit step
+constexpr int kPlanRow = kPlanRounds * 32 + 4;  // words per bucket row of the planner's counts (16-byte rows, padded)
 
 enum SegMode : int { kModeDone = 0, kModeBuckets = 1, kModeFallback = 2 };
 
@@ -96,7 +98,7 @@ __device__ __forceinline__ int block_excl_scan(int v, int* warp_tot, int& total)
 // ---------------------------------------------------------------------------
 // planner: one 1024-thread CTA per (b, kvh, s), largest segments first
 // ---------------------------------------------------------------------------
-__global__ void __launch_bounds__(kBucketThreads) k_bucket_plan(const float* __restrict__ scores,
+__global__ void __launch_bounds__(kBucketThreads, 2) k_bucket_plan(const float* __restrict__ scores,
                                                               float* __restrict__ sorted, int32_t* __restrict__ perm,
                                                               BucketSlot* __restrict__ slots, int* __restrict__ mode,
                                                               float2* __restrict__ range,
@@ -111,7 +113,9 @@ __global__ void __launch_bounds__(kBucketThreads) k_bucket_plan(const float* __r
   __shared__ float red[64];
   __shared__ int flag;
   __shared__ uint8_t bin2bkt[kNumBins];  // bucket id of each bin (< kMaxBuckets = 256)
-  __shared__ uint32_t wcnt[kMaxBuckets][kSortWarps + 1];  // [bucket][warp] counts, then ranks (padded rows)
+  // [bucket][round * 32 + warp] counts, then ranks: rows of kPlanRow words
+  // (dynamic shared memory, one row per bucket id in use)
+  extern __shared__ uint32_t wcnt[];
   __shared__ int cursor[kMaxBuckets];
   __shared__ int bin_cut;  // first bin left out of the order (filtered form)
   const int q = blockIdx.x;
@@ -245,7 +249,7 @@ __global__ void __launch_bounds__(kBucketThreads) k_bucket_plan(const float* __r
 #pragma unroll
   for (int e = 0; e < 2; ++e)
     if (end_id[e] >= 0) myslot[end_id[e]].count = end_rank[e] - myslot[end_id[e]].base;
-  // stable multisplit into the buckets, 1024 elements per step in index order
+  // stable multisplit into the buckets, 4096 elements per step in index order
   // (two block barriers per step)
   bin2bkt[2 * tid] = (uint8_t)(st0 / kBucketHalf);
   bin2bkt[2 * tid + 1] = (uint8_t)(st1 / kBucketHalf);
@@ -262,38 +266,53 @@ __global__ void __launch_bounds__(kBucketThreads) k_bucket_plan(const float* __r
   uint32_t* skey = stage_key + base;
   uint32_t* sval = stage_val + base;
   const int nbk = min(kMaxBuckets, my_slots);  // bucket ids in use are below this
-  for (int t0 = 0; t0 < n; t0 += kBucketThreads) {
-    const int i = t0 + tid;
-    const float x = i < n ? sc[i] : 0.f;
-    const int bin = score_bin(x, hi, scale);
-    const bool valid = i < n && bin < bcut;
-    const uint32_t d = valid ? bin2bkt[bin] : 0u;
+  // a step takes 4 rounds of 1024 elements: element i = t0 + 1024 k + tid, so
+  // index order is (round, warp, lane) and each bucket's row of 128 (round,
+  // warp) counts is scanned in that order
+  for (int t0 = 0; t0 < n; t0 += kPlanRounds * kBucketThreads) {
+    float x[kPlanRounds];
+    uint32_t d[kPlanRounds], rank[kPlanRounds];
+    bool valid[kPlanRounds];
     __syncwarp();
-    for (int k = lane; k < nbk; k += 32) wcnt[k][warp] = 0;
+    for (int q = lane; q < kPlanRounds * nbk; q += 32) wcnt[(q >> 2) * kPlanRow + (q & 3) * kSortWarps + warp] = 0;
     __syncwarp();
-    const uint32_t peers = __match_any_sync(0xffffffffu, valid ? d : 1024u + lane);
-    const uint32_t rank = __popc(peers & lt_mask);
-    if (valid && (__ffs(peers) - 1) == lane) wcnt[d][warp] = __popc(peers);
+#pragma unroll
+    for (int k = 0; k < kPlanRounds; ++k) {
+      const int i = t0 + k * kBucketThreads + tid;
+      x[k] = i < n ? sc[i] : 0.f;
+      const int bin = score_bin(x[k], hi, scale);
+      valid[k] = i < n && bin < bcut;
+      d[k] = valid[k] ? bin2bkt[bin] : 0u;
+      const uint32_t peers = __match_any_sync(0xffffffffu, valid[k] ? d[k] : 1024u + lane);
+      rank[k] = __popc(peers & lt_mask);
+      if (valid[k] && (__ffs(peers) - 1) == lane) wcnt[d[k] * kPlanRow + k * kSortWarps + warp] = __popc(peers);
+    }
     __syncthreads();
-    // per bucket, one warp scans the 32 warps' counts across its lanes: the
-    // counts become absolute ranks and the bucket's cursor advances
+    // per bucket, one warp scans its 128 counts (4 per lane): they become
+    // absolute ranks and the bucket's cursor advances
     for (int db = warp; db < nbk; db += kSortWarps) {
-      const uint32_t v = wcnt[db][lane];
-      uint32_t incl = v;
+      uint4 v = *reinterpret_cast<const uint4*>(wcnt + db * kPlanRow + 4 * lane);
+      const uint32_t tot = v.x + v.y + v.z + v.w;
+      uint32_t incl = tot;
 #pragma unroll
       for (int o = 1; o < 32; o <<= 1) {
         const uint32_t y = __shfl_up_sync(0xffffffffu, incl, o);
         if (lane >= o) incl += y;
       }
       const uint32_t cur = (uint32_t)cursor[db];
-      wcnt[db][lane] = cur + incl - v;
+      const uint32_t b0 = cur + incl - tot;
+      *reinterpret_cast<uint4*>(wcnt + db * kPlanRow + 4 * lane) =
+          make_uint4(b0, b0 + v.x, b0 + v.x + v.y, b0 + v.x + v.y + v.z);
       if (lane == 31) cursor[db] = (int)(cur + incl);
     }
     __syncthreads();
-    if (valid) {
-      const uint32_t pos = wcnt[d][warp] + rank;
-      skey[pos] = desc_key(x);
-      sval[pos] = (uint32_t)i;
+#pragma unroll
+    for (int k = 0; k < kPlanRounds; ++k) {
+      if (valid[k]) {
+        const uint32_t pos = wcnt[d[k] * kPlanRow + k * kSortWarps + warp] + rank[k];
+        skey[pos] = desc_key(x[k]);
+        sval[pos] = (uint32_t)(t0 + k * kBucketThreads + tid);
+      }
     }
   }
   if (tid == 0) mode[(size_t)bk * S + s] = kModeBuckets;
