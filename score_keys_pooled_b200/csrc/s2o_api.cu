@@ -261,8 +261,8 @@ static void launch_plan_core(const s2o_config* cfg, const double* qbar, const ui
                                                    w.segM, w.segZ, w.plen, cfg->tau, filtered, BH, S, T);
   ++t_launches;
   if (w.nslots > 0) {
-    k_bucket_sort<<<(unsigned)w.nslots, kSorterThreads, kBucketSmem, s>>>(w.keyB, w.valB, w.slots, w.sorted, perm,
-                                                                          T);
+    k_bucket_sort<<<(unsigned)((w.nslots + kSortGroup - 1) / kSortGroup), kSorterThreads, kBucketSmem, s>>>(
+        w.keyB, w.valB, w.slots, w.sorted, perm, w.nslots, T);
     ++t_launches;
   }
   k_sort<<<BH * S, kSortThreads, 0, s>>>(scores, w.segM, w.segZ, w.keyA, w.keyB, w.valA, w.valB, perm, w.sorted,

@@ -12,7 +12,9 @@
 //                  most kBucketHalf + one bin <= kBucketCap elements); then a
 //                  stable multisplit of the segment into its buckets: (key,
 //                  index) pairs land at the bucket's rank range, in index order;
-//   k_bucket_sort  one CTA per bucket: loads its range into shared memory and
+//   k_bucket_sort  one CTA per group of kSortGroup consecutive bucket slots
+//                  (the empty ones, buckets a segment did not need, are
+//                  skipped); per bucket: loads its range into shared memory and
 //                  sorts it there: a counting sort into 4096 fine bins linear
 //                  in the score, then each fine bin (a few elements) by
 //                  (key, index); a bucket with a crowded fine bin is sorted by
@@ -340,15 +342,11 @@ struct BucketSmem {
 };
 constexpr size_t kBucketSmem = sizeof(BucketSmem);
 
-__global__ void __launch_bounds__(kSorterThreads, 2) k_bucket_sort(const uint32_t* __restrict__ stage_key,
-                                                                  const uint32_t* __restrict__ stage_val,
-                                                                  const BucketSlot* __restrict__ slots,
-                                                                  float* __restrict__ sorted,
-                                                                  int32_t* __restrict__ perm, int64_t T) {
-  extern __shared__ uint8_t bsm_raw[];
-  BucketSmem& sm = *reinterpret_cast<BucketSmem*>(bsm_raw);
-  const BucketSlot slot = slots[blockIdx.x];
-  if (slot.count == 0) return;
+// one bucket: its pairs in shared memory, sorted, written back at its ranks
+__device__ __forceinline__ void sort_bucket(const BucketSlot& slot, BucketSmem& sm,
+                                            const uint32_t* __restrict__ stage_key,
+                                            const uint32_t* __restrict__ stage_val, float* __restrict__ sorted,
+                                            int32_t* __restrict__ perm, int64_t T) {
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const size_t base = (size_t)slot.bk * T + cand_offset(slot.s);
   if (tid == 0) { sm.kmin = 0xFFFFFFFFu; sm.kmax = 0u; }
@@ -508,6 +506,34 @@ write_out:
   for (int i = tid; i < m; i += kSorterThreads) {
     sorted[base + slot.base + i] = key_score(sm.key[cur][i]);
     perm[base + slot.base + i] = kSink + (int32_t)sm.val[cur][i];
+  }
+}
+
+// CTA = a group of kSortGroup consecutive slots; empty slots (the buckets a
+// segment did not need) cost one read of the group's records
+constexpr int kSortGroup = 8;
+__global__ void __launch_bounds__(kSorterThreads, 2) k_bucket_sort(const uint32_t* __restrict__ stage_key,
+                                                                  const uint32_t* __restrict__ stage_val,
+                                                                  const BucketSlot* __restrict__ slots,
+                                                                  float* __restrict__ sorted,
+                                                                  int32_t* __restrict__ perm, int64_t nslots,
+                                                                  int64_t T) {
+  extern __shared__ uint8_t bsm_raw[];
+  BucketSmem& sm = *reinterpret_cast<BucketSmem*>(bsm_raw);
+  __shared__ BucketSlot group[kSortGroup];
+  const int64_t g0 = (int64_t)blockIdx.x * kSortGroup;
+  if (threadIdx.x < kSortGroup) {
+    const int64_t k = g0 + threadIdx.x;
+    BucketSlot sl{};
+    if (k < nslots) sl = slots[k];
+    group[threadIdx.x] = sl;
+  }
+  __syncthreads();
+  for (int gi = 0; gi < kSortGroup; ++gi) {
+    const BucketSlot slot = group[gi];
+    if (slot.count == 0) continue;
+    sort_bucket(slot, sm, stage_key, stage_val, sorted, perm, T);
+    __syncthreads();  // the next bucket reuses the shared arrays
   }
 }
 
