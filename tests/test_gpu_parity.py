@@ -328,6 +328,51 @@ def test_filtered_plan_workloads(name):
                prefix_only=True)
 
 
+def test_clustered_scores_take_every_sort_path():
+    """Keys drawn from three distinct vectors: each segment's candidate scores
+    take three values, each shared by about a third of the candidates.  The
+    order is then fixed by the tie rule alone (equal scores, lower index
+    first) and both plans must reproduce the oracle's exactly.  The shapes
+    reach the sorter's less common paths: where the first tie group holds
+    fewer candidates than a bucket's window of 2816 ranks, two distinct values
+    share a bucket and crowd its fine bins (the bucket's radix sort); where a
+    tie group exceeds a bucket's room of 2816, the segment goes to the
+    global-memory sort."""
+    N, tau = 16384, 5e-3
+    Q, _, V = synth.generate(1, 2, 1, N, 128, planted=False, band=False, n_stripe=8, seed=5)
+    rng = np.random.default_rng(11)
+    # spread wide enough that the stop rule cuts most segments inside a group
+    vecs = synth.to_bf16_bits((32.0 * rng.standard_normal((3, 128))).astype(np.float32))
+    K = vecs[rng.integers(0, 3, N)][None, None].copy()
+    cfg = s2o.make_config(1, 2, 1, N, tau=tau)
+    filt, _ = filtered_matches_full(cfg, dev(Q), dev(K), dev(V))
+    full = s2o.plan(cfg, dev(Q), dev(K))
+    assert s2o.last_device_error() == 0
+    p = O.Params(tau=tau)
+    off = O.candidate_offsets(N, p)
+    perm_f, nb_f, _, _ = host_plan(cfg, full)
+    perm_p, nb_p, _, _ = host_plan(cfg, filt)
+    radix = fallback = cut = 0
+    for s in range(O.num_segments(N, p)):
+        sp = O.plan_segment(Q, K, 0, 0, s, 2, p)
+        n = len(sp.order)
+        cut += sp.C < len(sp.masses)
+        assert np.array_equal(perm_f[0, 0, off[s]:off[s + 1]], sp.order)
+        if sp.mass_ties.size == 0:
+            assert nb_f[0, 0, s] == sp.C
+        head = p.Bk * int(nb_p[0, 0, s])
+        assert np.array_equal(perm_p[0, 0, off[s]:off[s] + min(n, head)], sp.order[:head])
+        if n:
+            lo, hi = O.candidate_range(N, s, p)
+            vals, counts = np.unique(-sp.scores[lo:hi], return_counts=True)  # descending score
+            assert len(vals) <= 3
+            if counts.max() > 2816:
+                fallback += 1
+            elif len(counts) > 1 and counts[0] < 2816 and min(counts[0], counts[1]) > 64:
+                radix += 1
+    assert radix >= 20 and fallback >= 20 and cut >= 20, (radix, fallback, cut)
+
+
 def test_filtered_plan_tau_sweep():
     w = synth.WORKLOADS["sweep_64k"]
     Q, K, V = synth.generate_workload(w)
