@@ -45,7 +45,7 @@ constexpr int kNumBins = 2048;
 constexpr int kBucketCap = 5632;              // elements a bucket CTA sorts in shared memory
 constexpr int kBucketHalf = kBucketCap / 2;   // rank window of a bucket
 constexpr int kBucketThreads = 1024;          // planner CTA
-constexpr int kSorterThreads = 512;           // bucket-sorter CTA (two per SM)
+constexpr int kSorterThreads = 512;           // bucket-sorter CTA (three per SM)
 constexpr int kSorterWarps = kSorterThreads / 32;
 constexpr int kMaxBuckets = 256;              // bucket ids per segment (N <= 2^19)
 constexpr int kPlanRounds = 4;                // elements per planner thread and multisplit step
@@ -321,10 +321,16 @@ __global__ void __launch_bounds__(kBucketThreads, 2) k_bucket_plan(const float* 
 }
 
 // ---------------------------------------------------------------------------
-// bucket sorter: one 1024-thread CTA per slot
+// bucket sorter: one 512-thread CTA per group of slots, three CTAs per SM.
+// A bucket's pairs live in registers while they are counted and scattered
+// (pair k of thread tid is element tid + 512 k, so index order is (k, warp,
+// lane)); shared memory holds one key/value array, the scatter target.
 // ---------------------------------------------------------------------------
 constexpr int kFine = 4096;     // fine bins of a bucket (= kSorterWarps * 256 counters)
 constexpr int kFineMax = 64;    // larger fine bins send the bucket to the radix path
+constexpr int kSortPer = kBucketCap / kSorterThreads;  // pairs per thread
+static_assert(kSortPer * kSorterThreads == kBucketCap, "a bucket fills the sorter's registers exactly");
+static_assert(kFine == kSorterWarps * 256, "fine counters reuse the radix count rows");
 
 __device__ __forceinline__ int fine_bin(float x, float hi, float scale) {
   const int b = (int)((hi - x) * scale);
@@ -332,8 +338,8 @@ __device__ __forceinline__ int fine_bin(float x, float hi, float scale) {
 }
 
 struct BucketSmem {
-  uint32_t key[2][kBucketCap];
-  uint32_t val[2][kBucketCap];
+  uint32_t key[kBucketCap];
+  uint32_t val[kBucketCap];
   uint32_t cnt[kSorterWarps][256];  // radix digit counts, or the kFine fine-bin counters
   uint32_t dbase[256];
   int wtot[33];
@@ -342,108 +348,149 @@ struct BucketSmem {
 };
 constexpr size_t kBucketSmem = sizeof(BucketSmem);
 
-// one bucket: its pairs in shared memory, sorted, written back at its ranks
+// one bucket: sorted by (key, index) and written back at its global ranks
 __device__ __forceinline__ void sort_bucket(const BucketSlot& slot, BucketSmem& sm,
                                             const uint32_t* __restrict__ stage_key,
                                             const uint32_t* __restrict__ stage_val, float* __restrict__ sorted,
                                             int32_t* __restrict__ perm, int64_t T) {
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-  const size_t base = (size_t)slot.bk * T + cand_offset(slot.s);
+  const size_t base = (size_t)slot.bk * T + cand_offset(slot.s) + slot.base;
+  const int m = slot.count;
   if (tid == 0) { sm.kmin = 0xFFFFFFFFu; sm.kmax = 0u; }
 
   // the bucket's pairs, already in index order at its rank range
-  const int m = slot.count;
+  uint32_t rk[kSortPer], rv[kSortPer];
   uint32_t kmin = 0xFFFFFFFFu, kmax = 0u;
-  for (int i = tid; i < m; i += kSorterThreads) {
-    const uint32_t key = stage_key[base + slot.base + i];
-    kmin = min(kmin, key);
-    kmax = max(kmax, key);
-    sm.key[0][i] = key;
-    sm.val[0][i] = stage_val[base + slot.base + i];
+#pragma unroll
+  for (int k = 0; k < kSortPer; ++k) {
+    const int i = tid + kSorterThreads * k;
+    rk[k] = 0u;
+    rv[k] = 0u;
+    if (i < m) {
+      rk[k] = stage_key[base + i];
+      rv[k] = stage_val[base + i];
+      kmin = min(kmin, rk[k]);
+      kmax = max(kmax, rk[k]);
+    }
   }
+  kmin = __reduce_min_sync(0xffffffffu, kmin);
+  kmax = __reduce_max_sync(0xffffffffu, kmax);
   __syncthreads();
-  atomicMin(&sm.kmin, kmin);
-  atomicMax(&sm.kmax, kmax);
+  if (lane == 0) {
+    atomicMin(&sm.kmin, kmin);
+    atomicMax(&sm.kmax, kmax);
+  }
   __syncthreads();
   const uint32_t k0 = sm.kmin;
   const uint32_t span = sm.kmax - k0;
   const uint32_t lt_mask = (1u << lane) - 1u;
-  int cur = 0;
-  if (span == 0) goto write_out;  // one key: the index order is the order
+  if (span == 0) {
+    // one key: the index order is the order
+#pragma unroll
+    for (int k = 0; k < kSortPer; ++k) {
+      const int i = tid + kSorterThreads * k;
+      if (i < m) {
+        sorted[base + i] = key_score(rk[k]);
+        perm[base + i] = kSink + (int32_t)rv[k];
+      }
+    }
+    return;
+  }
 
   // Fine counting sort: kFine bins linear in the score between the bucket's
-  // extremes (monotone, ties share a bin), a stable-free scatter, then each
+  // extremes (monotone, ties share a bin), a scatter in any order, then each
   // bin sorted by (key, index) -- a total order, so the result is unique.
   {
     const float xhi = key_score(k0), xlo = key_score(sm.kmax);
     uint32_t* fcnt = &sm.cnt[0][0];  // kFine counters, then cursors
     const float fscale = (float)kFine / (xhi - xlo);
+    constexpr int kPerT = kFine / kSorterThreads;  // counters per thread
     for (int k = tid; k < kFine; k += kSorterThreads) fcnt[k] = 0;
     if (tid == 0) sm.big = 0;
     __syncthreads();
-    for (int i = tid; i < m; i += kSorterThreads)
-      atomicAdd(&fcnt[fine_bin(key_score(sm.key[0][i]), xhi, fscale)], 1u);
+#pragma unroll
+    for (int k = 0; k < kSortPer; ++k)
+      if (tid + kSorterThreads * k < m) atomicAdd(&fcnt[fine_bin(key_score(rk[k]), xhi, fscale)], 1u);
     __syncthreads();
-    uint32_t c[kFine / kSorterThreads];
     int mine = 0, big = 0;
 #pragma unroll
-    for (int e = 0; e < kFine / kSorterThreads; ++e) {
-      c[e] = fcnt[tid * (kFine / kSorterThreads) + e];
-      mine += (int)c[e];
-      big |= c[e] > kFineMax;
+    for (int e = 0; e < kPerT; ++e) {
+      const uint32_t c = fcnt[tid * kPerT + e];
+      mine += (int)c;
+      big |= c > kFineMax;
     }
     if (big) atomicOr(&sm.big, 1);
     int total;
     int run = block_excl_scan<kSorterWarps>(mine, sm.wtot, total);
     if (!sm.big) {
-      // counters become cursors (start ranks) and the bins are scattered
+      // counters become cursors (start ranks) and the pairs are scattered
 #pragma unroll
-      for (int e = 0; e < kFine / kSorterThreads; ++e) {
-        fcnt[tid * (kFine / kSorterThreads) + e] = (uint32_t)run;
-        run += (int)c[e];
+      for (int e = 0; e < kPerT; ++e) {
+        const uint32_t c = fcnt[tid * kPerT + e];
+        fcnt[tid * kPerT + e] = (uint32_t)run;
+        run += (int)c;
       }
       __syncthreads();
-      for (int i = tid; i < m; i += kSorterThreads) {
-        const uint32_t key = sm.key[0][i];
-        const uint32_t pos = atomicAdd(&fcnt[fine_bin(key_score(key), xhi, fscale)], 1u);
-        sm.key[1][pos] = key;
-        sm.val[1][pos] = sm.val[0][i];
-      }
-      __syncthreads();
-      // insertion sort of every fine bin (typically 1-3 elements)
 #pragma unroll
-      for (int e = 0; e < kFine / kSorterThreads; ++e) {
-        const int end = (int)fcnt[tid * (kFine / kSorterThreads) + e];
-        const int beg = end - (int)c[e];
-        for (int a2 = beg + 1; a2 < end; ++a2) {
-          const uint32_t kk = sm.key[1][a2], vv = sm.val[1][a2];
-          int b2 = a2 - 1;
-          while (b2 >= beg && (sm.key[1][b2] > kk || (sm.key[1][b2] == kk && sm.val[1][b2] > vv))) {
-            sm.key[1][b2 + 1] = sm.key[1][b2];
-            sm.val[1][b2 + 1] = sm.val[1][b2];
-            --b2;
-          }
-          sm.key[1][b2 + 1] = kk;
-          sm.val[1][b2 + 1] = vv;
+      for (int k = 0; k < kSortPer; ++k) {
+        if (tid + kSorterThreads * k < m) {
+          const uint32_t pos = atomicAdd(&fcnt[fine_bin(key_score(rk[k]), xhi, fscale)], 1u);
+          sm.key[pos] = rk[k];
+          sm.val[pos] = rv[k];
         }
       }
       __syncthreads();
-      cur = 1;
-      goto write_out;
+      // insertion sort of every fine bin (typically 1-3 elements); the
+      // cursors now hold each bin's end, so a bin starts where the last ended
+#pragma unroll
+      for (int e = 0; e < kPerT; ++e) {
+        const int b = tid * kPerT + e;
+        const int end = (int)fcnt[b];
+        const int beg = b ? (int)fcnt[b - 1] : 0;
+        for (int a2 = beg + 1; a2 < end; ++a2) {
+          const uint32_t kk = sm.key[a2], vv = sm.val[a2];
+          int b2 = a2 - 1;
+          while (b2 >= beg && (sm.key[b2] > kk || (sm.key[b2] == kk && sm.val[b2] > vv))) {
+            sm.key[b2 + 1] = sm.key[b2];
+            sm.val[b2 + 1] = sm.val[b2];
+            --b2;
+          }
+          sm.key[b2 + 1] = kk;
+          sm.val[b2 + 1] = vv;
+        }
+      }
+      __syncthreads();
+      for (int i = tid; i < m; i += kSorterThreads) {
+        sorted[base + i] = key_score(sm.key[i]);
+        perm[base + i] = kSink + (int32_t)sm.val[i];
+      }
+      return;
     }
-    __syncthreads();
   }
 
-  // a heavy fine bin: stable LSD radix sort over the bucket-relative key
-  {
+  // a crowded fine bin: stable LSD radix sort over the bucket-relative key,
+  // each pass scattering from the registers into the shared array
   const int nbits = 32 - __clz(span);
   const int passes = (nbits + 7) / 8;
   for (int pass = 0; pass < passes; ++pass) {
     const int shift = 8 * pass;
+    if (pass) {
+      // the previous pass's order, back into the registers
+#pragma unroll
+      for (int k = 0; k < kSortPer; ++k) {
+        const int i = tid + kSorterThreads * k;
+        if (i < m) {
+          rk[k] = sm.key[i];
+          rv[k] = sm.val[i];
+        }
+      }
+    }
     // digit totals
     for (int k = tid; k < kSorterWarps * 256; k += kSorterThreads) (&sm.cnt[0][0])[k] = 0;
     __syncthreads();
-    for (int i = tid; i < m; i += kSorterThreads) atomicAdd(&sm.cnt[warp][((sm.key[cur][i] - k0) >> shift) & 255u], 1u);
+#pragma unroll
+    for (int k = 0; k < kSortPer; ++k)
+      if (tid + kSorterThreads * k < m) atomicAdd(&sm.cnt[warp][((rk[k] - k0) >> shift) & 255u], 1u);
     __syncthreads();
     if (tid < 256) {
       uint32_t t = 0;
@@ -467,16 +514,13 @@ __device__ __forceinline__ void sort_bucket(const BucketSlot& slot, BucketSmem& 
       for (int k = 0; k < 8; ++k) sm.dbase[lane * 8 + k] = excl + v[k];
     }
     __syncthreads();
-    // stable scatter, one element per thread per step
-    const int out = cur ^ 1;
-    for (int t0 = 0; t0 < m; t0 += kSorterThreads) {
-      const int i = t0 + tid;
-      const bool valid = i < m;
-      const uint32_t key = valid ? sm.key[cur][i] : 0u;
-      const uint32_t val = valid ? sm.val[cur][i] : 0u;
-      const uint32_t dg = ((key - k0) >> shift) & 255u;
+    // stable scatter, 512 pairs (one per thread) per step, in index order
 #pragma unroll
-      for (int k = 0; k < 8; ++k) sm.cnt[warp][lane * 8 + k] = 0;
+    for (int k = 0; k < kSortPer; ++k) {
+      const bool valid = tid + kSorterThreads * k < m;
+      const uint32_t dg = ((rk[k] - k0) >> shift) & 255u;
+#pragma unroll
+      for (int q = 0; q < 8; ++q) sm.cnt[warp][lane * 8 + q] = 0;
       __syncwarp();
       const uint32_t peers = __match_any_sync(0xffffffffu, valid ? dg : 256u + lane);
       const uint32_t rank = __popc(peers & lt_mask);
@@ -494,25 +538,22 @@ __device__ __forceinline__ void sort_bucket(const BucketSlot& slot, BucketSmem& 
       __syncthreads();
       if (valid) {
         const uint32_t pos = sm.cnt[warp][dg] + rank;
-        sm.key[out][pos] = key;
-        sm.val[out][pos] = val;
+        sm.key[pos] = rk[k];
+        sm.val[pos] = rv[k];
       }
       __syncthreads();
     }
-    cur = out;
   }
-  }
-write_out:
   for (int i = tid; i < m; i += kSorterThreads) {
-    sorted[base + slot.base + i] = key_score(sm.key[cur][i]);
-    perm[base + slot.base + i] = kSink + (int32_t)sm.val[cur][i];
+    sorted[base + i] = key_score(sm.key[i]);
+    perm[base + i] = kSink + (int32_t)sm.val[i];
   }
 }
 
 // CTA = a group of kSortGroup consecutive slots; empty slots (the buckets a
 // segment did not need) cost one read of the group's records
 constexpr int kSortGroup = 8;
-__global__ void __launch_bounds__(kSorterThreads, 2) k_bucket_sort(const uint32_t* __restrict__ stage_key,
+__global__ void __launch_bounds__(kSorterThreads, 3) k_bucket_sort(const uint32_t* __restrict__ stage_key,
                                                                   const uint32_t* __restrict__ stage_val,
                                                                   const BucketSlot* __restrict__ slots,
                                                                   float* __restrict__ sorted,
