@@ -267,7 +267,12 @@ __global__ void __launch_bounds__(kBucketThreads, 2) k_bucket_plan(const float* 
   const uint32_t lt_mask = (1u << lane) - 1u;
   uint32_t* skey = stage_key + base;
   uint32_t* sval = stage_val + base;
-  const int nbk = min(kMaxBuckets, my_slots);  // bucket ids in use are below this
+  // bucket ids in use: those of the bins below bin_cut
+  const int nbk = bcut > 0 ? (int)bin2bkt[bcut - 1] + 1 : 0;
+  if (nbk == 0) {
+    if (tid == 0) mode[(size_t)bk * S + s] = kModeBuckets;
+    return;
+  }
   // a step takes 4 rounds of 1024 elements: element i = t0 + 1024 k + tid, so
   // index order is (round, warp, lane) and each bucket's row of 128 (round,
   // warp) counts is scanned in that order
@@ -285,7 +290,9 @@ __global__ void __launch_bounds__(kBucketThreads, 2) k_bucket_plan(const float* 
       const int bin = score_bin(x[k], hi, scale);
       valid[k] = i < n && bin < bcut;
       d[k] = valid[k] ? bin2bkt[bin] : 0u;
-      const uint32_t peers = __match_any_sync(0xffffffffu, valid[k] ? d[k] : 1024u + lane);
+      // lanes holding the same bucket id (the lanes left out share one value:
+      // a match costs more the more distinct values a warp holds)
+      const uint32_t peers = __match_any_sync(0xffffffffu, valid[k] ? d[k] : 0xFFFFFFFFu);
       rank[k] = __popc(peers & lt_mask);
       if (valid[k] && (__ffs(peers) - 1) == lane) wcnt[d[k] * kPlanRow + k * kSortWarps + warp] = __popc(peers);
     }
