@@ -141,7 +141,7 @@ __global__ void __launch_bounds__(kSortThreads, 2)
 #pragma unroll
       for (int k = 0; k < 8; ++k) sm.cnt[warp][lane * 8 + k] = 0;
       __syncwarp();
-      const uint32_t peers = __match_any_sync(0xffffffffu, valid ? dg : 256u + lane);
+      const uint32_t peers = __match_any_sync(0xffffffffu, valid ? dg : 0xFFFFFFFFu);
       const uint32_t rank = __popc(peers & lt_mask);
       if (valid && (__ffs(peers) - 1) == lane) sm.cnt[warp][dg] = __popc(peers);
       __syncthreads();

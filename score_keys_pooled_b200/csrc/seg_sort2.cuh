@@ -529,7 +529,7 @@ __device__ __forceinline__ void sort_bucket(const BucketSlot& slot, BucketSmem& 
 #pragma unroll
       for (int q = 0; q < 8; ++q) sm.cnt[warp][lane * 8 + q] = 0;
       __syncwarp();
-      const uint32_t peers = __match_any_sync(0xffffffffu, valid ? dg : 256u + lane);
+      const uint32_t peers = __match_any_sync(0xffffffffu, valid ? dg : 0xFFFFFFFFu);
       const uint32_t rank = __popc(peers & lt_mask);
       if (valid && (__ffs(peers) - 1) == lane) sm.cnt[warp][dg] = __popc(peers);
       __syncthreads();
