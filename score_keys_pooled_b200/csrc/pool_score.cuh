@@ -60,8 +60,8 @@ __global__ void __launch_bounds__(256) k_pool(const uint16_t* __restrict__ Q, do
 
 // ---------------------------------------------------------------------------
 // score: CTA = (key tile t of 128 keys, chunk of 64 segments, b*Hkv).
-// Only segments s >= t see tile t (e(s) = 128 s + 128 > 128 t), so CTAs whose
-// chunk ends before t exit at once.  Dot products are accumulated in fp64:
+// Only segments s >= t see tile t (e(s) = 128 s + 128 > 128 t), so the grid
+// holds only the pairs whose chunk reaches t.  Dot products are accumulated in fp64:
 // qbar is the exact fp64 mean of bf16 values and k_j is bf16, so every
 // product is exact and the sum carries ~1e-15 relative error; each score is
 // rounded once to fp32.  (fp32 accumulation of these 128-term dots errs by
@@ -99,9 +99,17 @@ __device__ __forceinline__ void dmma_8x8x4(double& c0, double& c1, double a, dou
 __global__ void __launch_bounds__(256, 2) k_score(const uint16_t* __restrict__ K, const double* __restrict__ qbar,
                                                  float* __restrict__ scores, float2* __restrict__ part,
                                                  int Hkv, int N, int S, int64_t T) {
-  const int t = blockIdx.x;           // key tile
-  const int chunk = blockIdx.y;       // segment chunk
-  const int bk = blockIdx.z;          // b * Hkv + kvh
+  // blockIdx.x enumerates the (chunk, tile) pairs on or below the causal
+  // diagonal, chunk-major: chunk c holds the tiles t < min(S, 64 (c + 1))
+  const int nchunks = (S + kScoreSegs - 1) / kScoreSegs;
+  int t = blockIdx.x;                 // key tile, once the chunks before are skipped
+  int chunk = 0;                      // segment chunk
+  while (chunk < nchunks && t >= min(S, kScoreSegs * (chunk + 1))) {
+    t -= min(S, kScoreSegs * (chunk + 1));
+    ++chunk;
+  }
+  if (chunk >= nchunks) return;
+  const int bk = blockIdx.y;          // b * Hkv + kvh
   const int s_lo = chunk * kScoreSegs;
   const int s_hi = min(S, s_lo + kScoreSegs);
   if (s_hi - 1 < t) return;

@@ -249,9 +249,11 @@ static void launch_plan_core(const s2o_config* cfg, const double* qbar, const ui
   const int S = nseg(cfg);
   const int BH = cfg->B * cfg->Hkv;
   const int64_t T = ncand_total(cfg);
-  const int ntiles = (cfg->N + kScoreKeys - 1) / kScoreKeys;
+  // (chunk, tile) pairs on or below the causal diagonal: chunk c reaches tiles t < min(S, 64 (c + 1))
   const int nchunks = (S + kScoreSegs - 1) / kScoreSegs;
-  k_score<<<dim3(ntiles, nchunks, BH), 256, kScoreSmem, s>>>(K, qbar, scores, w.part, cfg->Hkv, cfg->N, S, T);
+  int pairs = 0;
+  for (int c = 0; c < nchunks; ++c) pairs += min(S, kScoreSegs * (c + 1));
+  k_score<<<dim3(pairs, BH), 256, kScoreSmem, s>>>(K, qbar, scores, w.part, cfg->Hkv, cfg->N, S, T);
   ++t_launches;
   const int nwarps = BH * S;
   k_seg_stats<<<(nwarps * 32 + 255) / 256, 256, 0, s>>>(w.part, w.segM, w.segZ, seg_stats, BH, S);
