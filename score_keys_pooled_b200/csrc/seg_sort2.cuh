@@ -48,8 +48,11 @@ constexpr int kBucketThreads = 1024;          // planner CTA
 constexpr int kSorterThreads = 512;           // bucket-sorter CTA (three per SM)
 constexpr int kSorterWarps = kSorterThreads / 32;
 constexpr int kMaxBuckets = 256;              // bucket ids per segment (N <= 2^19)
+constexpr int kPlanWarps = kBucketThreads / 32;
 constexpr int kPlanRounds = 4;                // elements per planner thread and multisplit step
-constexpr int kPlanRow = kPlanRounds * 32 + 4;  // words per bucket row of the planner's counts (16-byte rows, padded)
+constexpr int kPlanRow = kPlanRounds * kPlanWarps + 4;  // words per bucket row of the planner's counts (16-byte rows, padded)
+static_assert(kPlanRounds * kPlanWarps == 128, "a bucket's counts are scanned by one warp, 4 per lane");
+static_assert(kPlanRounds == 4, "count rows are cleared as (bucket, round) = (q / 4, q % 4)");
 
 enum SegMode : int { kModeDone = 0, kModeBuckets = 1, kModeFallback = 2 };
 
@@ -281,7 +284,7 @@ __global__ void __launch_bounds__(kBucketThreads, 2) k_bucket_plan(const float* 
     uint32_t d[kPlanRounds], rank[kPlanRounds];
     bool valid[kPlanRounds];
     __syncwarp();
-    for (int q = lane; q < kPlanRounds * nbk; q += 32) wcnt[(q >> 2) * kPlanRow + (q & 3) * kSortWarps + warp] = 0;
+    for (int q = lane; q < kPlanRounds * nbk; q += 32) wcnt[(q >> 2) * kPlanRow + (q & 3) * kPlanWarps + warp] = 0;
     __syncwarp();
 #pragma unroll
     for (int k = 0; k < kPlanRounds; ++k) {
@@ -294,12 +297,12 @@ __global__ void __launch_bounds__(kBucketThreads, 2) k_bucket_plan(const float* 
       // a match costs more the more distinct values a warp holds)
       const uint32_t peers = __match_any_sync(0xffffffffu, valid[k] ? d[k] : 0xFFFFFFFFu);
       rank[k] = __popc(peers & lt_mask);
-      if (valid[k] && (__ffs(peers) - 1) == lane) wcnt[d[k] * kPlanRow + k * kSortWarps + warp] = __popc(peers);
+      if (valid[k] && (__ffs(peers) - 1) == lane) wcnt[d[k] * kPlanRow + k * kPlanWarps + warp] = __popc(peers);
     }
     __syncthreads();
     // per bucket, one warp scans its 128 counts (4 per lane): they become
     // absolute ranks and the bucket's cursor advances
-    for (int db = warp; db < nbk; db += kSortWarps) {
+    for (int db = warp; db < nbk; db += kPlanWarps) {
       uint4 v = *reinterpret_cast<const uint4*>(wcnt + db * kPlanRow + 4 * lane);
       const uint32_t tot = v.x + v.y + v.z + v.w;
       uint32_t incl = tot;
@@ -318,7 +321,7 @@ __global__ void __launch_bounds__(kBucketThreads, 2) k_bucket_plan(const float* 
 #pragma unroll
     for (int k = 0; k < kPlanRounds; ++k) {
       if (valid[k]) {
-        const uint32_t pos = wcnt[d[k] * kPlanRow + k * kSortWarps + warp] + rank[k];
+        const uint32_t pos = wcnt[d[k] * kPlanRow + k * kPlanWarps + warp] + rank[k];
         skey[pos] = desc_key(x[k]);
         sval[pos] = (uint32_t)(t0 + k * kBucketThreads + tid);
       }
