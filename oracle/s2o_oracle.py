@@ -48,7 +48,11 @@ the following readings (the GPU library takes the same ones):
   * Q_perm (optional): the segment's rows are ordered by the mean over the
     group's heads of q_i . qbar (the shared guide vector), ties to the lower
     row; the first Lq/2 rows and the rest form two sub-segments, each planned
-    with its own pooled query; a row attends over its sub-segment's kept set.
+    with its own pooled query; a row attends over its sub-segment's kept set;
+  * MSE against dense attention: the mean over every output element of the
+    squared difference between the sparse and the dense causal output;
+  * contiguous comparator: original-order blocks of Bk candidates ranked by
+    the sum of their pooled-softmax masses, ties to the lower block.
 
 All arithmetic is IEEE fp64 on inputs widened exactly from bf16.  Loops are
 plain; numpy's matmul, sort and sum are used as library steps only.  The
@@ -564,3 +568,40 @@ def kept_pairs_segment(N: int, s: int, keep: np.ndarray, p: Params) -> int:
     for i in range(r0, r1):
         total += int(np.searchsorted(keep, i, side="right"))
     return total
+
+
+def mse_segment(Qf, Kf, Vf, b: int, kvh: int, s: int, G: int, keep: np.ndarray, p: Params) -> tuple[float, int]:
+    """Squared error of the sparse output against dense causal attention for
+    one segment (all heads of the group, all rows, all channels).
+
+    The pages quote a "single-operator MSE" of S2O against full attention
+    (pith.science page, "read the original abstract") without defining it;
+    the reading taken here is the mean over every output element (b, h, i, c)
+    of (O_sparse - O_dense)^2, both exact fp64 evaluations on the same bf16
+    inputs.  Returns (sum of squared differences, number of elements) so that
+    sums over segments give the mean over any set of segments.
+    """
+    sparse = attention_segment(Qf, Kf, Vf, b, kvh, s, G, keep, p)
+    dense = dense_segment(Qf, Kf, Vf, b, kvh, s, G, p)
+    diff = sparse - dense
+    return float(np.sum(diff * diff)), int(diff.size)
+
+
+def mse(Qf, Kf, Vf, perm, nblocks, p: Params, segments=None, offsets=None) -> float:
+    """Mean over the listed segments' output elements (every (b, kvh) and
+    head) of the squared difference between the plan's sparse output and
+    dense causal attention; all segments when `segments` is None."""
+    B, Hq, N, d = Qf.shape
+    Hkv = Kf.shape[1]
+    G = Hq // Hkv
+    off = candidate_offsets(N, p) if offsets is None else offsets
+    segs = range(num_segments(N, p)) if segments is None else segments
+    sse, n = 0.0, 0
+    for b in range(B):
+        for kvh in range(Hkv):
+            for s in segs:
+                keep = keep_set(N, s, perm[b, kvh, off[s]:off[s + 1]], int(nblocks[b, kvh, s]), p)
+                e, m = mse_segment(Qf, Kf, Vf, b, kvh, s, G, keep, p)
+                sse += e
+                n += m
+    return sse / n if n else 0.0

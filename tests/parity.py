@@ -1,12 +1,19 @@
 """Comparison helpers: GPU plan / output against the fp64 oracle.
 
-Index lists and block counts must match the oracle exactly, except inside
-near-tie sets the oracle reports: runs of the oracle order whose adjacent
-scores differ by at most 1e-6 x max|s| (their relative order is not decided
-by the inputs at the precision the GPU computes in), and blocks whose mass
-lies within 1e-6 x tau of tau.  Every such allowance is counted and logged.
-Outputs must be within max-abs 1.5e-2 and relative RMS 4e-3 of the oracle
-evaluated on the same bf16 inputs and the same kept set.
+Index lists and block counts must match the oracle exactly, except where the
+inputs do not decide the answer at the precision the GPU computes in:
+
+  * a position p of the order may hold a different key than the oracle's
+    only if the two keys' oracle (fp64) scores differ by at most
+    1e-6 x max|s| over the segment's admissible keys (a score near-tie);
+  * C(s) may differ from the oracle's only if every block between the two
+    stop points has a mass within 1e-6 x tau of tau (a mass near-tie).
+
+Every allowance used is counted.  The totals are printed in pytest's
+terminal summary (see tests/conftest.py) and, when S2O_NEAR_TIE_LOG names a
+file, appended to it per case.  Outputs must be within max-abs 1.5e-2 and
+relative RMS 4e-3 of the oracle evaluated on the same bf16 inputs and the
+same kept set.
 """
 from __future__ import annotations
 
@@ -20,8 +27,14 @@ from oracle import s2o_oracle as O
 MAX_ABS = 1.5e-2
 REL_RMS = 4e-3
 
+# allowances used in this process: segments compared, positions holding a
+# different (near-tied) key, and blocks between differing stop points
+TOTALS = {"segments": 0, "swapped_positions": 0, "C_flips": 0, "online_C_flips": 0, "cases": 0}
+
 
 def log_near_ties(record: dict):
+    TOTALS["cases"] += 1
+    TOTALS["online_C_flips"] += int(record.get("C_flips", 0)) if record.get("online") else 0
     path = os.environ.get("S2O_NEAR_TIE_LOG")
     if path:
         with open(path, "a") as f:
@@ -46,25 +59,22 @@ def compare_segment_plan(gpu_perm: np.ndarray, gpu_C: int, sp: O.SegmentPlan, p:
             assert len(np.unique(head)) == len(head), "perm prefix repeats a key"
         else:
             assert np.array_equal(np.sort(gpu_perm), np.arange(lo, lo + n)), "perm is not a permutation of Cand(s)"
-    # near-tie runs of the oracle order
-    run = np.zeros(n, dtype=np.int64)
-    if n > 1:
-        brk = np.ones(n - 1, dtype=bool)
-        brk[sp.score_ties] = False
-        run[1:] = np.cumsum(brk)
     if prefix_only:
         span = min(n, p.Bk * gpu_C)
     else:
         span = n if full_list else min(n, p.Bk * max(gpu_C, sp.C) + p.Bk)
     swapped = 0
-    if n:
-        pos = np.empty(n, dtype=np.int64)
-        pos[sp.order - lo] = np.arange(n)
-        gpos = pos[gpu_perm[:span] - lo]
-        mism = gpu_perm[:span] != sp.order[:span]
-        bad = np.nonzero(mism & (run[gpos] != run[:span]))[0]
-        assert bad.size == 0, f"position {bad[:5]}: keys outside the oracle's near-tie runs"
-        swapped = int(mism.sum())
+    if span:
+        mism = np.nonzero(gpu_perm[:span] != sp.order[:span])[0]
+        if mism.size:
+            # the scores of the two keys at each differing position, both fp64 oracle values
+            s_gpu = sp.scores[gpu_perm[mism]]
+            s_ora = sp.scores[sp.order[mism]]
+            gap = np.abs(s_gpu - s_ora)
+            bad = mism[gap > sp.tie_tol]
+            assert bad.size == 0, (f"positions {bad[:5]}: keys {gpu_perm[bad[:5]]} for {sp.order[bad[:5]]}, "
+                                   f"score gaps {gap[gap > sp.tie_tol][:5]} > {sp.tie_tol:.3g}")
+        swapped = int(mism.size)
     flip = 0
     if gpu_C != sp.C:
         lo_b, hi_b = min(gpu_C, sp.C), max(gpu_C, sp.C)
@@ -72,6 +82,9 @@ def compare_segment_plan(gpu_perm: np.ndarray, gpu_C: int, sp: O.SegmentPlan, p:
         assert all(b in ties for b in range(lo_b, hi_b)), \
             f"C(s) {gpu_C} != oracle {sp.C} and the blocks between are not mass near-ties"
         flip = hi_b - lo_b
+    TOTALS["segments"] += 1
+    TOTALS["swapped_positions"] += swapped
+    TOTALS["C_flips"] += flip
     return swapped, flip
 
 

@@ -172,6 +172,64 @@ def test_hand_worked_contiguous_comparator():
     assert full[:spec["C_match"] * p.Bk].tolist() == spec["expected_prefix"]
 
 
+def _contig_case(spec, a):
+    sh = spec["shape"]
+    N, d = sh["N"], sh["d"]
+    Q = np.zeros((1, 1, N, d), dtype=np.float32)
+    Q[0, 0, 8:12, 0] = 2.0
+    K = np.zeros((1, 1, N, d), dtype=np.float32)
+    K[0, 0, 1:8, 0] = a
+    return _bits(Q), _bits(K)
+
+
+@pytest.mark.parametrize("ci", [0, 1])
+def test_contiguous_comparator_hand_cases(ci):
+    # tests/golden/hand_contiguous.json: the highest-mass block is not the one
+    # with the highest score, nor the one with the highest sum of raw scores
+    # or of mean mass per key; and an exact mass tie goes to the lower block
+    with open(os.path.join(GOLDEN, "hand_contiguous.json")) as f:
+        spec = json.load(f)
+    case = spec["cases"][ci]
+    Q, K = _contig_case(spec, case["a_candidates"])
+    p = O.Params(tau=0.0, **spec["params"])
+    sp = O.plan_segment(Q, K, 0, 0, 2, 1, p)
+    assert np.array_equal(sp.scores[1:8], np.asarray(case["a_candidates"], dtype=np.float64))
+    full = O.contiguous_plan_segment(sp, spec["shape"]["N"], case["C_match"], p)
+    assert full.tolist() == case["expected_full"]
+    assert full[:case["C_match"] * p.Bk].tolist() == case["expected_prefix"]
+
+
+# ---------------------------------------------------------------------------
+# MSE against dense attention
+# ---------------------------------------------------------------------------
+
+def test_mse_hand_worked_closed_form():
+    with open(os.path.join(GOLDEN, "hand_mse.json")) as f:
+        spec = json.load(f)
+    g = _load_golden()
+    case = [c for c in g["cases"] if c["name"] == spec["case"]][0]
+    Q, K, V = _golden_case(case)
+    p = O.Params(tau=spec["tau"], **case["params"])
+    res = O.plan(Q, K, p)
+    got = O.mse(Q, K, V, res["perm"], res["nblocks"], p)
+    want = sum((_ev(sx) - _ev(dx)) ** 2 for sx, dx in spec["rows"].values()) / spec["elements"]
+    assert want > 1e-4
+    assert got == pytest.approx(want, rel=1e-12, abs=0)
+    # segment 0 has nothing to drop
+    sse0, n0 = O.mse_segment(Q, K, V, 0, 0, 0, 1, res["plans"][(0, 0, 0)].keep, p)
+    assert sse0 == 0.0 and n0 == 16
+
+
+def test_mse_is_zero_at_tau_zero():
+    # tau = 0 keeps every admissible key, so the sparse output is the dense one
+    Q, K, V = _random_case(7, Hq=2, Hkv=1, N=640, d=32)
+    for tau, zero in ((0.0, True), (5e-2, False)):
+        p = O.Params(tau=tau)
+        res = O.plan(Q, K, p)
+        m = O.mse(Q, K, V, res["perm"], res["nblocks"], p)
+        assert (m == 0.0) == zero
+
+
 # ---------------------------------------------------------------------------
 # all-ties closed form: Q = 0 makes every score exactly 0
 # ---------------------------------------------------------------------------
