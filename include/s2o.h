@@ -169,9 +169,15 @@ s2o_status s2o_plan_filtered(const s2o_config* cfg, const uint16_t* Q, const uin
  *   process exits).  Configs whose plan workspace (s2o_plan_workspace_size)
  *   exceeds 32 MiB -- e.g. B=1, 8 KV heads, N above ~7K -- are rejected with
  *   S2O_ERR_WORKSPACE_TOO_SMALL before anything is launched.
- *   The first call on a device looks up the buffer's device address for that
- *   device (make that first call before any stream capture).  Nothing in the
- *   buffer has to start at zero: every word the kernels read is written
+ *   The 32 MiB are committed by the driver when the library's device code is
+ *   loaded into a context: with lazy loading (the default since CUDA 12.2)
+ *   that happens on the first call into the library on a device, which may be
+ *   this one, and that load can synchronise the device.  The first call on a
+ *   device (and again after cudaDeviceReset or in another context) also looks
+ *   up the buffer's device address with that device current.  So make one
+ *   warm-up call -- e.g. s2o_plan_noalloc on a small config -- at engine
+ *   start-up, before any stream capture; later calls do neither.  Nothing in
+ *   the buffer has to start at zero: every word the kernels read is written
  *   earlier in the same call.  All calls share the one buffer, so calls whose
  *   work overlaps on the GPU (other streams, other host threads) race and
  *   corrupt each other's results; serialise them.
@@ -215,6 +221,24 @@ s2o_status s2o_attention(const s2o_config* cfg, const uint16_t* Q, const uint16_
 
 /* Device bytes s2o_prefill_host needs in its arena. */
 s2o_status s2o_prefill_arena_size(const s2o_config* cfg, int32_t out_dtype, size_t* bytes);
+
+/*
+ * s2o_attention_bounded -- s2o_attention with every wait of its pipeline
+ * (mbarrier polls between the loader, tensor-core and softmax roles of a
+ * CTA) limited to max_polls polls instead of the default 2^24, for testing
+ * the timeout path (the pages have no counterpart; the library's failure
+ * handling is its own).  A wait that runs out sets the device error word
+ * (s2o_last_device_error then returns S2O_ERR_DEVICE_TIMEOUT) and the CTA
+ * winds down: it waits, with the default limit, for the tensor-core products
+ * and Q tiles it already started, frees its tensor memory and ends.  Outputs
+ * are unspecified after a timeout.  max_polls = 0 makes every wait give up
+ * at once.  Only the even-group-size kernel (Hq/Hkv even) takes the limit;
+ * other shapes return S2O_ERR_UNSUPPORTED_SHAPE, max_polls above 2^24
+ * S2O_ERR_INVALID_ARG.  Arguments otherwise as s2o_attention.
+ */
+s2o_status s2o_attention_bounded(const s2o_config* cfg, const uint16_t* Q, const uint16_t* K,
+                                 const uint16_t* V, const int32_t* perm, const int32_t* nblocks, void* O,
+                                 int32_t out_dtype, uint32_t max_polls, s2o_stream_t stream);
 
 /*
  * s2o_attention_online -- the pages' run-time stop in place of the planned one
@@ -329,6 +353,30 @@ s2o_status s2o_last_device_error(s2o_stream_t stream);
 /* Number of kernels the last s2o_plan / s2o_attention / s2o_plan_contiguous
  * call on this thread launched (the library's own kernels only). */
 int32_t s2o_last_launch_count(void);
+
+/*
+ * Per-kernel timing of the plan calls, for measurement (the pages report no
+ * per-stage times; they name the ranking step as the main preprocessing
+ * cost: gist.science technical summary, "Resultats Experimentaux").
+ * s2o_stage_timing(1) creates this host thread's timing events on the
+ * current device; from then on every plan call on this thread (s2o_plan,
+ * s2o_plan_filtered, s2o_plan_noalloc, s2o_plan_qperm) records one event on
+ * its stream before its first kernel and one after each kernel.
+ * s2o_stage_timing(0) destroys the events and stops the recording.  Returns
+ * S2O_ERR_CUDA if the events cannot be created.  Recording costs a few
+ * microseconds per kernel; leave it off outside measurements.
+ */
+s2o_status s2o_stage_timing(int32_t enable);
+
+/*
+ * Elapsed device time of each kernel of the last plan call on this thread
+ * (between consecutive events on its stream).  Waits for that call's last
+ * event.  ms[i] (and names[i], a static kernel name, when names is not NULL)
+ * are written for i < min(count, cap).  Returns the number of kernels
+ * recorded (at most 16), or -1 when timing is off, ms is NULL with cap > 0,
+ * or a CUDA event call fails.
+ */
+int32_t s2o_last_stage_times(float* ms, const char** names, int32_t cap);
 
 #ifdef __cplusplus
 }

@@ -67,6 +67,7 @@ def lib() -> ctypes.CDLL:
         L.s2o_plan_noalloc.argtypes = [_CFG, _P, _P, _P, _P, _P, _P, _P]
         L.s2o_plan_contiguous.argtypes = [_CFG, _P, _P, _P, _P, _P]
         L.s2o_attention.argtypes = [_CFG, _P, _P, _P, _P, _P, _P, ctypes.c_int32, _P]
+        L.s2o_attention_bounded.argtypes = [_CFG, _P, _P, _P, _P, _P, _P, ctypes.c_int32, ctypes.c_uint32, _P]
         L.s2o_attention_online.argtypes = [_CFG, _P, _P, _P, _P, _P, ctypes.c_int32, _P, _P]
         L.s2o_block_truth_workspace_size.argtypes = [_CFG, ctypes.c_int32, ctypes.POINTER(ctypes.c_size_t)]
         L.s2o_plan_qperm_workspace_size.argtypes = [_CFG, ctypes.POINTER(ctypes.c_size_t)]
@@ -79,7 +80,12 @@ def lib() -> ctypes.CDLL:
         L.s2o_status_string.restype = ctypes.c_char_p
         L.s2o_last_device_error.argtypes = [_P]
         L.s2o_last_launch_count.restype = ctypes.c_int32
-        for name in ("s2o_plan_workspace_size", "s2o_plan", "s2o_plan_filtered", "s2o_plan_noalloc", "s2o_plan_contiguous", "s2o_attention", "s2o_attention_online",
+        L.s2o_stage_timing.argtypes = [ctypes.c_int32]
+        L.s2o_stage_timing.restype = ctypes.c_int
+        L.s2o_last_stage_times.argtypes = [ctypes.POINTER(ctypes.c_float), ctypes.POINTER(ctypes.c_char_p),
+                                           ctypes.c_int32]
+        L.s2o_last_stage_times.restype = ctypes.c_int32
+        for name in ("s2o_plan_workspace_size", "s2o_plan", "s2o_plan_filtered", "s2o_plan_noalloc", "s2o_plan_contiguous", "s2o_attention", "s2o_attention_bounded", "s2o_attention_online",
                      "s2o_block_truth_workspace_size", "s2o_block_truth", "s2o_plan_qperm_workspace_size",
                      "s2o_plan_qperm", "s2o_attention_qperm",
                      "s2o_prefill_arena_size", "s2o_prefill_host", "s2o_last_device_error"):
@@ -186,6 +192,18 @@ def attention(cfg: Config, Q, K, V, perm, nblocks, O=None, out_dtype: int = OUT_
     return O
 
 
+def attention_bounded(cfg: Config, Q, K, V, perm, nblocks, max_polls: int, O=None, out_dtype: int = OUT_BF16,
+                      stream=None):
+    """s2o_attention with every pipeline wait limited to max_polls polls (tests of the timeout path)."""
+    import torch
+    if O is None:
+        O = torch.empty(Q.shape, dtype=torch.bfloat16 if out_dtype == OUT_BF16 else torch.float32,
+                        device=Q.device)
+    _check(lib().s2o_attention_bounded(ctypes.byref(cfg), _ptr(Q), _ptr(K), _ptr(V), _ptr(perm), _ptr(nblocks),
+                                       _ptr(O), out_dtype, max_polls, _stream(stream)), "s2o_attention_bounded")
+    return O
+
+
 def attention_online(cfg: Config, Q, K, V, perm, O=None, nblocks_out=None, out_dtype: int = OUT_BF16, stream=None):
     """s2o_attention_online: the run-time stop; returns (O, nblocks_out [B*Hq*S])."""
     import torch
@@ -265,6 +283,21 @@ def last_device_error(stream=None) -> int:
 
 def last_launch_count() -> int:
     return lib().s2o_last_launch_count()
+
+
+def stage_timing(enable: bool):
+    """Turn per-kernel event timing of the plan calls on or off (this thread)."""
+    _check(lib().s2o_stage_timing(1 if enable else 0), "s2o_stage_timing")
+
+
+def last_stage_times() -> list[tuple[str, float]]:
+    """(kernel name, device ms) of each kernel of the last plan call on this thread."""
+    ms = (ctypes.c_float * 16)()
+    names = (ctypes.c_char_p * 16)()
+    n = lib().s2o_last_stage_times(ms, names, 16)
+    if n < 0:
+        raise S2OError(4, "s2o_last_stage_times")
+    return [(names[i].decode(), float(ms[i])) for i in range(n)]
 
 
 def status_string(code: int) -> str:

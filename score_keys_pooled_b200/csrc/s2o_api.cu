@@ -153,20 +153,48 @@ bool encode_rows_map(CUtensorMap* map, const void* base, uint64_t rows, uint32_t
              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-// Device address of g_s2o_plan_scratch, looked up once per device.
+// The context current on the calling thread (driver entry point fetched
+// through the runtime once).  Per-device state below is tied to the context
+// it was made in: after cudaDeviceReset, or with another context current on
+// the same device, the module is loaded again at new addresses and old
+// streams are gone, so each cache entry remembers its context and is made
+// again when the context changes.
+using CtxGetCurrentFn = CUresult (*)(CUcontext*);
+std::once_flag g_ctx_once;
+CtxGetCurrentFn g_ctx_get = nullptr;
+
+CUcontext current_context() {
+  std::call_once(g_ctx_once, [] {
+    void* fn = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuCtxGetCurrent", &fn, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      g_ctx_get = reinterpret_cast<CtxGetCurrentFn>(fn);
+  });
+  CUcontext c = nullptr;
+  if (!g_ctx_get || g_ctx_get(&c) != CUDA_SUCCESS) return nullptr;
+  return c;
+}
+
+// Device address of g_s2o_plan_scratch, looked up once per device and context.
 std::mutex g_scratch_mu;
 constexpr int kMaxDevices = 64;
 void* g_scratch_addr[kMaxDevices] = {};
+CUcontext g_scratch_ctx[kMaxDevices] = {};
 
 // Copy streams of s2o_prefill_host (host->device, device->host), created on
-// the first call on each device and kept for the life of the process.
+// the first call on each device (and context) and kept for the life of that
+// context.
 std::mutex g_copy_mu;
 cudaStream_t g_copy_in[kMaxDevices] = {}, g_copy_out[kMaxDevices] = {};
+CUcontext g_copy_ctx[kMaxDevices] = {};
 bool copy_streams(cudaStream_t& in, cudaStream_t& out) {
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return false;
   std::lock_guard<std::mutex> lock(g_copy_mu);
-  if (!g_copy_in[dev]) {
+  const CUcontext ctx = current_context();
+  if (!g_copy_in[dev] || !ctx || ctx != g_copy_ctx[dev]) {
+    // streams of an earlier context died with it: make new ones, drop the old handles
     cudaStream_t a = nullptr, b = nullptr;
     if (cudaStreamCreateWithFlags(&a, cudaStreamNonBlocking) != cudaSuccess) return false;
     if (cudaStreamCreateWithFlags(&b, cudaStreamNonBlocking) != cudaSuccess) {
@@ -175,6 +203,7 @@ bool copy_streams(cudaStream_t& in, cudaStream_t& out) {
     }
     g_copy_in[dev] = a;
     g_copy_out[dev] = b;
+    g_copy_ctx[dev] = current_context();
   }
   in = g_copy_in[dev];
   out = g_copy_out[dev];
@@ -183,6 +212,30 @@ bool copy_streams(cudaStream_t& in, cudaStream_t& out) {
 
 s2o_status launch_status() {
   return cudaGetLastError() == cudaSuccess ? S2O_OK : S2O_ERR_CUDA;
+}
+
+// Optional per-stage timing (s2o_stage_timing): an event on the caller's
+// stream before the first kernel of a call and after each kernel, per host
+// thread; s2o_last_stage_times reads the gaps.
+constexpr int kMaxStages = 16;
+struct StageClock {
+  bool on = false;
+  cudaEvent_t ev[kMaxStages + 1] = {};
+  const char* name[kMaxStages] = {};
+  int n = 0;
+};
+thread_local StageClock t_clock;
+
+void stage_begin(cudaStream_t s) {
+  if (!t_clock.on) return;
+  t_clock.n = 0;
+  cudaEventRecord(t_clock.ev[0], s);
+}
+
+void stage_mark(cudaStream_t s, const char* name) {
+  if (!t_clock.on || t_clock.n >= kMaxStages) return;
+  t_clock.name[t_clock.n] = name;
+  cudaEventRecord(t_clock.ev[++t_clock.n], s);
 }
 
 }  // namespace
@@ -235,8 +288,10 @@ static s2o_status run_plan(const s2o_config* cfg, const uint16_t* Q, const uint1
   const int S = nseg(cfg);
   const int BH = cfg->B * cfg->Hkv;
 
+  stage_begin(s);
   k_pool<<<dim3(S, BH), 256, 0, s>>>(Q, w.qbar, cfg->Hq, cfg->Hkv, cfg->N, S);
   ++t_launches;
+  stage_mark(s, "k_pool");
   launch_plan_core(cfg, w.qbar, K, scores, perm, nblocks, seg_stats, w, s, filtered);
   return launch_status();
 }
@@ -255,23 +310,29 @@ static void launch_plan_core(const s2o_config* cfg, const double* qbar, const ui
   for (int c = 0; c < nchunks; ++c) pairs += min(S, kScoreSegs * (c + 1));
   k_score<<<dim3(pairs, BH), 256, kScoreSmem, s>>>(K, qbar, scores, w.part, cfg->Hkv, cfg->N, S, T);
   ++t_launches;
+  stage_mark(s, "k_score");
   const int nwarps = BH * S;
   k_seg_stats<<<(nwarps * 32 + 255) / 256, 256, 0, s>>>(w.part, w.segM, w.segZ, seg_stats, BH, S);
   ++t_launches;
+  stage_mark(s, "k_seg_stats");
   const size_t plan_smem = (size_t)min(kMaxBuckets, bucket_slots(num_cand(S - 1))) * kPlanRow * sizeof(uint32_t);
   k_bucket_plan<<<BH * S, kBucketThreads, plan_smem, s>>>(scores, w.sorted, perm, w.slots, w.mode, w.range, w.keyB, w.valB,
                                                    w.segM, w.segZ, w.plen, cfg->tau, filtered, BH, S, T);
   ++t_launches;
+  stage_mark(s, "k_bucket_plan");
   if (w.nslots > 0) {
     k_bucket_sort<<<(unsigned)((w.nslots + kSortGroup - 1) / kSortGroup), kSorterThreads, kBucketSmem, s>>>(
         w.keyB, w.valB, w.slots, w.sorted, perm, w.nslots, T);
     ++t_launches;
+    stage_mark(s, "k_bucket_sort");
   }
   k_sort<<<BH * S, kSortThreads, 0, s>>>(scores, w.segM, w.segZ, w.keyA, w.keyB, w.valA, w.valB, perm, w.sorted,
                                          w.mode, kModeFallback, BH, S, T);
   ++t_launches;
+  stage_mark(s, "k_sort");
   k_mass_stop<<<BH * S, 256, 0, s>>>(w.sorted, w.segM, w.segZ, w.plen, nblocks, BH, S, T, cfg->tau);
   ++t_launches;
+  stage_mark(s, "k_mass_stop");
 }
 
 s2o_status s2o_plan(const s2o_config* cfg, const uint16_t* Q, const uint16_t* K, float* scores, int32_t* perm,
@@ -345,9 +406,26 @@ s2o_status s2o_plan_contiguous(const s2o_config* cfg, const float* scores, const
   return launch_status();
 }
 
+static s2o_status run_attention(const s2o_config* cfg, const uint16_t* Q, const uint16_t* K, const uint16_t* V,
+                                const int32_t* perm, const int32_t* nblocks, void* O, int32_t out_dtype,
+                                s2o_stream_t stream, uint32_t spin);
+
 s2o_status s2o_attention(const s2o_config* cfg, const uint16_t* Q, const uint16_t* K, const uint16_t* V,
                          const int32_t* perm, const int32_t* nblocks, void* O, int32_t out_dtype,
                          s2o_stream_t stream) {
+  return run_attention(cfg, Q, K, V, perm, nblocks, O, out_dtype, stream, kSpinLimit);
+}
+
+s2o_status s2o_attention_bounded(const s2o_config* cfg, const uint16_t* Q, const uint16_t* K, const uint16_t* V,
+                                 const int32_t* perm, const int32_t* nblocks, void* O, int32_t out_dtype,
+                                 uint32_t max_polls, s2o_stream_t stream) {
+  if (max_polls > kSpinLimit) return S2O_ERR_INVALID_ARG;
+  return run_attention(cfg, Q, K, V, perm, nblocks, O, out_dtype, stream, max_polls);
+}
+
+static s2o_status run_attention(const s2o_config* cfg, const uint16_t* Q, const uint16_t* K, const uint16_t* V,
+                                const int32_t* perm, const int32_t* nblocks, void* O, int32_t out_dtype,
+                                s2o_stream_t stream, uint32_t spin) {
   t_launches = 0;
   s2o_status st = check_cfg(cfg);
   if (st != S2O_OK) return st;
@@ -368,12 +446,15 @@ s2o_status s2o_attention(const s2o_config* cfg, const uint16_t* Q, const uint16_
     a.T = ncand_total(cfg);
     a.out_f32 = out_dtype == S2O_OUT_F32;
     a.tau = 0.f; a.cout = nullptr; a.perm1 = nullptr; a.nblocks1 = nullptr; a.rowsub = nullptr;
+    a.spin = spin;
     CUtensorMap tmQ;
     if (!encode_rows_map(&tmQ, Q, (uint64_t)cfg->B * cfg->Hq * cfg->N, 128))
       return S2O_ERR_CUDA;
     const int64_t ncta = (int64_t)cfg->B * cfg->Hkv * a.S * (G / 2);
     k_sparse_attn2<false><<<(unsigned)ncta, kAttn2Threads, kAttn2Smem, s>>>(a, tmQ);
   } else {
+    // this kernel's waits always take the default limit
+    if (spin != kSpinLimit) return S2O_ERR_UNSUPPORTED_SHAPE;
     AttnArgs a;
     a.Q = Q; a.K = K; a.V = V; a.perm = perm; a.nblocks = nblocks; a.O = O;
     a.B = cfg->B; a.Hq = cfg->Hq; a.Hkv = cfg->Hkv; a.N = cfg->N; a.S = nseg(cfg);
@@ -408,6 +489,7 @@ s2o_status s2o_attention_online(const s2o_config* cfg, const uint16_t* Q, const 
   a.T = ncand_total(cfg);
   a.out_f32 = out_dtype == S2O_OUT_F32;
   a.tau = (float)cfg->tau; a.cout = nblocks_out; a.perm1 = nullptr; a.nblocks1 = nullptr; a.rowsub = nullptr;
+  a.spin = kSpinLimit;
   CUtensorMap tmQ;
   if (!encode_rows_map(&tmQ, Q, (uint64_t)cfg->B * cfg->Hq * cfg->N, 128)) return S2O_ERR_CUDA;
   const int64_t ncta = (int64_t)cfg->B * cfg->Hkv * a.S * (G / 2);
@@ -482,6 +564,7 @@ s2o_status s2o_attention_qperm(const s2o_config* cfg, const uint16_t* Q, const u
   a.perm1 = perm + BH * T;
   a.nblocks1 = nblocks + BH * a.S;
   a.rowsub = rowsub;
+  a.spin = kSpinLimit;
   CUtensorMap tmQ;
   if (!encode_rows_map(&tmQ, Q, (uint64_t)cfg->B * cfg->Hq * cfg->N, 128)) return S2O_ERR_CUDA;
   const int64_t ncta = (int64_t)cfg->B * cfg->Hkv * a.S * (G / 2);
@@ -613,12 +696,15 @@ s2o_status s2o_plan_noalloc(const s2o_config* cfg, const uint16_t* Q, const uint
   void* scratch = nullptr;
   {
     std::lock_guard<std::mutex> lock(g_scratch_mu);
-    if (!g_scratch_addr[dev]) {
+    const CUcontext ctx = current_context();
+    if (!g_scratch_addr[dev] || !ctx || ctx != g_scratch_ctx[dev]) {
       // In host code the array's name is only a host-side handle; the device
-      // address comes from the runtime, with this device current.
+      // address comes from the runtime, with this device current.  The
+      // lookup loads the module into the context if it is not loaded yet.
       void* p = nullptr;
       if (cudaGetSymbolAddress(&p, g_s2o_plan_scratch) != cudaSuccess || !p) return S2O_ERR_CUDA;
       g_scratch_addr[dev] = p;
+      g_scratch_ctx[dev] = current_context();
     }
     scratch = g_scratch_addr[dev];
   }
@@ -652,5 +738,34 @@ s2o_status s2o_last_device_error(s2o_stream_t stream) {
 }
 
 int32_t s2o_last_launch_count(void) { return t_launches; }
+
+s2o_status s2o_stage_timing(int32_t enable) {
+  if (enable && !t_clock.on) {
+    for (int i = 0; i <= kMaxStages; ++i) {
+      if (cudaEventCreate(&t_clock.ev[i]) != cudaSuccess) {
+        for (int j = 0; j < i; ++j) cudaEventDestroy(t_clock.ev[j]);
+        return S2O_ERR_CUDA;
+      }
+    }
+    t_clock.on = true;
+    t_clock.n = 0;
+  } else if (!enable && t_clock.on) {
+    for (int i = 0; i <= kMaxStages; ++i) cudaEventDestroy(t_clock.ev[i]);
+    t_clock.on = false;
+    t_clock.n = 0;
+  }
+  return S2O_OK;
+}
+
+int32_t s2o_last_stage_times(float* ms, const char** names, int32_t cap) {
+  if (!t_clock.on || cap < 0 || (cap > 0 && !ms)) return -1;
+  const int n = t_clock.n;
+  if (n > 0 && cudaEventSynchronize(t_clock.ev[n]) != cudaSuccess) return -1;
+  for (int i = 0; i < n && i < cap; ++i) {
+    if (cudaEventElapsedTime(&ms[i], t_clock.ev[i], t_clock.ev[i + 1]) != cudaSuccess) return -1;
+    if (names) names[i] = t_clock.name[i];
+  }
+  return n;
+}
 
 }  // extern "C"

@@ -79,6 +79,7 @@ constexpr int kBarGain = 23;    //      online stop: the 8 softmax warps (count 
 constexpr int kSlotTmem = 24;
 constexpr int kSlotGain = 25;   //      online stop: 3 fp32 gain accumulators (slots 25, 26)
 constexpr int kSlotStop = 27;   //      online stop: index of the chunk after which the tile stops
+constexpr int kBarDrain = 28;   // [2]  issuer i's final commit: every tensor-core op it issued is done
 constexpr int kNoStop = 0x7fffffff;
 // tensor-memory columns
 __device__ __forceinline__ uint32_t col_o(int i) { return 128u * i; }
@@ -127,6 +128,43 @@ __device__ __forceinline__ float fmax3(float a, float b, float c) {
 }
 __device__ __forceinline__ float f2_lo(uint64_t v) { return __uint_as_float((uint32_t)v); }
 __device__ __forceinline__ float f2_hi(uint64_t v) { return __uint_as_float((uint32_t)(v >> 32)); }
+__device__ __forceinline__ uint64_t f2_sub(uint64_t a, uint64_t b) {
+  uint64_t d;
+  asm("sub.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+  return d;
+}
+
+// 2^x for a pair of fp32 values on the FMA pipe, leaving the special-function
+// unit (ex2.approx) to the other pairs of a row.  x = n + f with n = round(x)
+// and f in [-1/2, 1/2] (exact in fp32; n comes from adding 1.5 * 2^23, which
+// leaves round(x) in the low mantissa bits); 2^f is the degree-4 polynomial
+// of least maximum relative error on [-1/2, 1/2] (Remez exchange; the
+// coefficients and the generator are in exp2_poly.py), evaluated by Horner's
+// rule with packed fused multiply-adds; n is added to the exponent field.
+// Relative error below 3e-6 (the P values are then rounded to bf16).
+// Arguments are clamped to >= -125 so that the exponent stays normal.
+constexpr float kExp2C0 = 0.9999992847442627f;
+constexpr float kExp2C1 = 0.6931217908859253f;
+constexpr float kExp2C2 = 0.240247443318367f;
+constexpr float kExp2C3 = 0.05591785907745361f;
+constexpr float kExp2C4 = 0.009570102207362652f;
+__device__ __forceinline__ uint64_t exp2_poly_x2(uint64_t v) {
+  const float a = fmaxf(f2_lo(v), -125.f), b = fmaxf(f2_hi(v), -125.f);
+  const uint64_t x = f2_pack(a, b);
+  const uint64_t magic = f2_pack(12582912.f, 12582912.f);
+  const uint64_t t = f2_add(x, magic);
+  const uint64_t f = f2_sub(x, f2_sub(t, magic));
+  uint64_t p = f2_fma(f2_pack(kExp2C4, kExp2C4), f, f2_pack(kExp2C3, kExp2C3));
+  p = f2_fma(p, f, f2_pack(kExp2C2, kExp2C2));
+  p = f2_fma(p, f, f2_pack(kExp2C1, kExp2C1));
+  p = f2_fma(p, f, f2_pack(kExp2C0, kExp2C0));
+  const uint32_t lo = (uint32_t)p + ((uint32_t)t << 23);
+  const uint32_t hi = (uint32_t)(p >> 32) + ((uint32_t)(t >> 32) << 23);
+  return ((uint64_t)hi << 32) | lo;
+}
+// of every 8 pairs of a row's 64 scores in an unmasked chunk, this many take
+// exp2_poly_x2 and the rest ex2.approx
+constexpr int kPolyOf8 = 0;
 
 __device__ __forceinline__ void mbar_arrive(uint32_t bar) {
   asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];\n" ::"r"(bar) : "memory");
@@ -142,8 +180,8 @@ __device__ __forceinline__ void tma_load_2d(uint32_t dst, const CUtensorMap* map
       : "memory");
 }
 // warp-uniform bounded wait: every lane polls, all agree on the outcome
-__device__ __forceinline__ bool warp_wait(uint32_t bar, uint32_t parity) {
-  const bool ok = mbar_wait_bounded(bar, parity);
+__device__ __forceinline__ bool warp_wait(uint32_t bar, uint32_t parity, uint32_t limit) {
+  const bool ok = mbar_wait_bounded(bar, parity, limit);
   return __all_sync(0xffffffffu, ok);
 }
 
@@ -195,6 +233,9 @@ struct Attn2Args {
   const int32_t* perm1;
   const int32_t* nblocks1;
   const uint8_t* rowsub;
+  // polls of every pipeline wait before it gives up (kSpinLimit; smaller only
+  // to exercise the timeout path).  The final drains always use kSpinLimit.
+  uint32_t spin;
 };
 
 // ONLINE selects the run-time stop, QPERM the two query sub-segments; the
@@ -250,6 +291,8 @@ __global__ void __launch_bounds__(kAttn2Threads, 1)
       if (k == kBarGain) count = 8;
       mbar_init(bar(k), count);
     }
+    mbar_init(bar(kBarDrain), 1);
+    mbar_init(bar(kBarDrain + 1), 1);
     float* gacc = reinterpret_cast<float*>(sgen + kOff2Bar + 8 * kSlotGain);
     gacc[0] = gacc[1] = gacc[2] = 0.f;
     *reinterpret_cast<volatile int*>(sgen + kOff2Bar + 8 * kSlotStop) = kNoStop;
@@ -360,20 +403,20 @@ __global__ void __launch_bounds__(kAttn2Threads, 1)
       if (t + 1 < ntiles) fetch_keys(t + 1, y);  // in flight while this stage fills
       bool okw;
       if (!ONLINE) {
-        okw = warp_wait(bar(bar_empty + st), (uint32_t)((round & 1) ^ 1));
+        okw = warp_wait(bar(bar_empty + st), (uint32_t)((round & 1) ^ 1), a.spin);
       } else {
         // lane 0 waits for the stage or for a stop that makes it unneeded;
         // after a free stage every lane acquires the barrier itself
         int r = 0;
         if (lane == 0) {
-          for (uint32_t it = 0; it < kSpinLimit && r == 0; ++it) {
+          for (uint32_t it = 0; it < a.spin && r == 0; ++it) {
             if (mbar_try_wait(bar(bar_empty + st), (uint32_t)((round & 1) ^ 1))) r = 1;
             else if (not_needed(t)) r = 2;
           }
         }
         r = __shfl_sync(0xffffffffu, r, 0);
         if (r == 2) break;
-        okw = r == 1 && warp_wait(bar(bar_empty + st), (uint32_t)((round & 1) ^ 1));
+        okw = r == 1 && warp_wait(bar(bar_empty + st), (uint32_t)((round & 1) ^ 1), a.spin);
       }
       if (!okw) {
         if (lane == 0) set_error(kErrTimeout);
@@ -410,6 +453,9 @@ __global__ void __launch_bounds__(kAttn2Threads, 1)
       __syncwarp();
       if (lane == 0) mbar_arrive(bar(bar_full + st));
     }
+    // Q's TMA tiles may still be landing if the issuers gave up waiting for
+    // them: shared memory must not change after the CTA ends
+    if (is_k && lane == 0 && !mbar_wait_bounded(bar(kBarQFull), 0)) set_error(kErrTimeout);
   } else if (warp == kMmaWarp || warp == kMmaWarp1) {
     // ------------------------------------------------------------------ MMA issuers
     // head i's products, in order: its P V of tile t-1 and half h precedes its
@@ -420,7 +466,7 @@ __global__ void __launch_bounds__(kAttn2Threads, 1)
     if (lane == 0) {
       const uint32_t idesc_qk = idesc_bf16_f32(128, kBk, false);   // one 64-key half
       const uint32_t idesc_pv = idesc_bf16_f32(128, 128, true);
-      bool ok = mbar_wait_bounded(bar(kBarQFull), 0);
+      bool ok = mbar_wait_bounded(bar(kBarQFull), 0, a.spin);
       // chunk c = half c & 1 of tile c >> 1: S of chunk c as soon as the
       // softmax has read S of chunk c - 1, then P V of chunk c - 1
       const int nch = 2 * ntiles;
@@ -428,11 +474,11 @@ __global__ void __launch_bounds__(kAttn2Threads, 1)
         if (c < nch) {
           const int t = c >> 1, h = c & 1;
           if (h == 0) {
-            ok = mbar_wait_bounded(bar(kBarKFull + t % kStagesK), (uint32_t)((t / kStagesK) & 1));
+            ok = mbar_wait_bounded(bar(kBarKFull + t % kStagesK), (uint32_t)((t / kStagesK) & 1), a.spin);
             if (!ok) break;
           }
           if (c > 0) {
-            ok = mbar_wait_bounded(bar(kBarSEmpty + i), (uint32_t)((c - 1) & 1));
+            ok = mbar_wait_bounded(bar(kBarSEmpty + i), (uint32_t)((c - 1) & 1), a.spin);
             if (!ok) break;
             tc_fence_after();
           }
@@ -450,10 +496,10 @@ __global__ void __launch_bounds__(kAttn2Threads, 1)
         if (c > 0) {
           const int cp = c - 1, tp = cp >> 1, hp = cp & 1;
           if (hp == 0) {
-            ok = mbar_wait_bounded(bar(kBarVFull + tp % kStagesV), (uint32_t)((tp / kStagesV) & 1));
+            ok = mbar_wait_bounded(bar(kBarVFull + tp % kStagesV), (uint32_t)((tp / kStagesV) & 1), a.spin);
             if (!ok) break;
           }
-          ok = mbar_wait_bounded(bar(kBarPFull + 2 * i + hp), (uint32_t)((cp >> 1) & 1));
+          ok = mbar_wait_bounded(bar(kBarPFull + 2 * i + hp), (uint32_t)((cp >> 1) & 1), a.spin);
           if (!ok) break;
           tc_fence_after();
           const uint32_t sV = sbase + kOff2V + (tp % kStagesV) * kTile2Bytes;
@@ -467,12 +513,16 @@ __global__ void __launch_bounds__(kAttn2Threads, 1)
           if (ONLINE && cp == *stop_word) {
             // the tile stopped after chunk cp; Q K^T of chunk c (if any) is
             // the last product in flight: wait for it before the CTA ends
-            if (c < nch) ok = mbar_wait_bounded(bar(kBarSFull + i), (uint32_t)(c & 1));
+            if (c < nch) ok = mbar_wait_bounded(bar(kBarSFull + i), (uint32_t)(c & 1), a.spin);
             break;
           }
         }
       }
       if (!ok) set_error(kErrTimeout);
+      // every product this thread issued must be done before the tensor
+      // memory is freed (a given-up wait may leave some in flight)
+      tc_commit(bar(kBarDrain + i));
+      if (!mbar_wait_bounded(bar(kBarDrain + i), 0)) set_error(kErrTimeout);
     }
   } else {
     // ------------------------------------------------------------------ softmax
@@ -500,7 +550,7 @@ __global__ void __launch_bounds__(kAttn2Threads, 1)
       const int kind = walk2_block(wk, s, c, j0);
       int lim = kind == 3 ? -1 : (kind == 0 ? row - j0 : kBk);
       if (QPERM && kind == 2 && (j0 >= C0 ? 1 : 0) != my_sub) lim = -1;  // the other sub-segment's block
-      if (!warp_wait(bar(kBarSFull + qi), (uint32_t)(c & 1))) { ok = false; break; }
+      if (!warp_wait(bar(kBarSFull + qi), (uint32_t)(c & 1), a.spin)) { ok = false; break; }
       tc_fence_after();
       float x[kBk];
       tmem_ld32(tS, x);
@@ -533,7 +583,10 @@ __global__ void __launch_bounds__(kAttn2Threads, 1)
       // a moved reference rescales O once every P V issued so far (the last
       // one is chunk c - 1's) is done
       if (c > 0 && __any_sync(0xffffffffu, move)) {
-        if (!warp_wait(bar(kBarODone + 2 * qi + ((c - 1) & 1)), (uint32_t)(((c - 1) >> 1) & 1))) { ok = false; break; }
+        if (!warp_wait(bar(kBarODone + 2 * qi + ((c - 1) & 1)), (uint32_t)(((c - 1) >> 1) & 1), a.spin)) {
+          ok = false;
+          break;
+        }
         tc_fence_after();
 #pragma unroll
         for (int cc = 0; cc < 128; cc += 32) {
@@ -553,7 +606,15 @@ __global__ void __launch_bounds__(kAttn2Threads, 1)
 #pragma unroll
         for (int k = 0; k < kBk; k += 2) {
           const uint64_t v = f2_fma(f2_pack(x[k], x[k + 1]), s2, nm2);
-          const float p0 = ex2_approx(f2_lo(v)), p1 = ex2_approx(f2_hi(v));
+          float p0, p1;
+          if (((k >> 1) & 7) < kPolyOf8) {
+            const uint64_t pp = exp2_poly_x2(v);
+            p0 = f2_lo(pp);
+            p1 = f2_hi(pp);
+          } else {
+            p0 = ex2_approx(f2_lo(v));
+            p1 = ex2_approx(f2_hi(v));
+          }
           rs2 = f2_add(rs2, f2_pack(p0, p1));
           x[k / 2] = __uint_as_float(pack_bf16x2(p0, p1));
         }
@@ -580,7 +641,7 @@ __global__ void __launch_bounds__(kAttn2Threads, 1)
           atomicAdd(const_cast<float*>(gacc + q % 3), gsum);
           mbar_arrive(bar(kBarGain));
         }
-        if (!warp_wait(bar(kBarGain), (uint32_t)(q & 1))) { ok = false; break; }
+        if (!warp_wait(bar(kBarGain), (uint32_t)(q & 1), a.spin)) { ok = false; break; }
         const float tot = gacc[q % 3];
         // the slot used at q - 1: every warp read it before arriving at q
         if (warp == 0 && lane == 0) gacc[(q + 2) % 3] = 0.f;
@@ -607,7 +668,7 @@ __global__ void __launch_bounds__(kAttn2Threads, 1)
       for (int k = 0; k < 2; ++k) a.cout[((size_t)b * a.Hq + h0 + k) * a.S + s] = c_online;
     }
     if (ok && nch_done > 0)
-      ok = warp_wait(bar(kBarODone + 2 * qi + ((nch_done - 1) & 1)), (uint32_t)(((nch_done - 1) >> 1) & 1));
+      ok = warp_wait(bar(kBarODone + 2 * qi + ((nch_done - 1) & 1)), (uint32_t)(((nch_done - 1) >> 1) & 1), a.spin);
     if (!ok) {
       if (lane == 0) set_error(kErrTimeout);
     } else {

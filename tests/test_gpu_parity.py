@@ -270,6 +270,85 @@ def test_sweep_64k_tau_and_contiguous():
             check_output(Q, K, V, cfg, pch, nb, outc, p, segments=segs, kvheads=[5], what=f"contig tau={tau}")
 
 
+def test_contiguous_comparator_hand_case():
+    """Keys one-hot along dim 0 (s_j = 0.99989 a_j for the pooled query
+    (11.3125, 0, ...)); original-order candidate blocks B0..B4 of 64 keys:
+    B0 = 32 keys at 2 and 32 at -10, B1 = B3 = 64 keys at 1.1875, B2 = one key
+    at 2.5 and 63 at -10, B4 = 64 keys at -10.  Block masses go B0 > B1 = B3 >
+    B2 > B4, while the largest score is in B2 and the largest raw-score sum in
+    B1; B1 and B3 hold the same values in the same places, so their masses tie
+    exactly and the lower block ranks first."""
+    N = 640
+    a = np.zeros(N, dtype=np.float32)
+    a[64:96], a[96:128] = 2.0, -10.0
+    a[128:192] = 1.1875
+    a[192], a[193:256] = 2.5, -10.0
+    a[256:320] = 1.1875
+    a[320:384] = -10.0
+    Kf = np.zeros((1, 1, N, 128), dtype=np.float32)
+    Kf[0, 0, :, 0] = a
+    Qf = np.zeros((1, 2, N, 128), dtype=np.float32)
+    Qf[..., 0] = 11.3125
+    Q, K = synth.to_bf16_bits(Qf), synth.to_bf16_bits(Kf)
+    p = O.Params(tau=1e-3)
+    cfg = s2o.make_config(1, 2, 1, N, tau=1e-3)
+    bufs = s2o.plan(cfg, dev(Q), dev(K))
+    pc = torch.full_like(bufs["perm"], -1)
+    s2o.plan_contiguous(cfg, bufs["scores"], bufs["seg_stats"], bufs["nblocks"], pc)
+    assert s2o.last_device_error() == 0
+    off = O.candidate_offsets(N, p)
+    got = pc.cpu().numpy()
+    blk = lambda *bs: [j for b in bs for j in range(64 + 64 * b, 128 + 64 * b)]
+    want = {3: blk(0, 1, 2), 4: blk(0, 1, 3, 2, 4)}
+    for s, w in want.items():
+        sp = O.plan_segment(Q, K, 0, 0, s, 2, p)
+        assert O.contiguous_plan_segment(sp, N, 1, p).tolist() == w
+        assert got[off[s]:off[s + 1]].tolist() == w
+
+
+def test_mse_measurement_matches_oracle():
+    """The benchmark's MSE against dense attention (the plan's fp32 output
+    against the tau = 0 output, averaged on the device) against the oracle's
+    fp64 MSE on the same kept sets, on sampled segments of llama_16k.  Each
+    GPU output is within relative RMS 4e-3 of its oracle value, so by the
+    triangle inequality in L2 the two root-mean-square differences agree to
+    within 2 x 4e-3 x RMS(dense output).  tau = 3e-3, where these segments
+    drop a measurable share of their mass (at 1e-3 llama_16k keeps ~99 %)."""
+    import bench
+    w = synth.WORKLOADS["llama_16k"]
+    Q, K, V = synth.generate_workload(w)
+    tau = 3e-3
+    p = O.Params(tau=tau)
+    q, k, v = dev(Q), dev(K), dev(V)
+    cfg = s2o.make_config(w.B, w.Hq, w.Hkv, w.N, tau=tau)
+    bufs = s2o.plan(cfg, q, k)
+    Os = s2o.attention(cfg, q, k, v, bufs["perm"], bufs["nblocks"], out_dtype=s2o.OUT_F32)
+    perm, nb, _, _ = host_plan(cfg, bufs)
+    cfg0 = s2o.make_config(w.B, w.Hq, w.Hkv, w.N, tau=0.0)
+    b0 = s2o.plan(cfg0, q, k)
+    Od = s2o.attention(cfg0, q, k, v, b0["perm"], b0["nblocks"], out_dtype=s2o.OUT_F32)
+    assert s2o.last_device_error() == 0
+    G = w.Hq // w.Hkv
+    S = O.num_segments(w.N, p)
+    off = O.candidate_offsets(w.N, p)
+    kvh = 3
+    sse_o = n_o = sq_o = 0.0
+    rows = []
+    for s in (5, S // 2, S - 1):
+        keep = O.keep_set(w.N, s, perm[0, kvh, off[s]:off[s + 1]], int(nb[0, kvh, s]), p)
+        e, m = O.mse_segment(Q, K, V, 0, kvh, s, G, keep, p)
+        sse_o += e
+        n_o += m
+        sq_o += float(np.sum(O.dense_segment(Q, K, V, 0, kvh, s, G, p) ** 2))
+        rows.append(O.segment_rows(w.N, s, p))
+    sl = lambda t: torch.cat([t[0, kvh * G:(kvh + 1) * G, r0:r1] for r0, r1 in rows], dim=1).unsqueeze(0)
+    mse_gpu, _ = bench.mse_on_device(torch, sl(Os), sl(Od))
+    mse_ora = sse_o / n_o
+    assert mse_ora > 1e-6  # the sampled segments drop real mass
+    bound = 2 * parity.REL_RMS * np.sqrt(sq_o / n_o)
+    assert abs(np.sqrt(mse_gpu) - np.sqrt(mse_ora)) <= bound, (mse_gpu, mse_ora, bound)
+
+
 # ---------------------------------------------------------------------------
 # s2o_plan_filtered: only the prefix of each order the stop rule can reach
 # ---------------------------------------------------------------------------
