@@ -82,6 +82,100 @@ def kept_pairs_qperm(nblocks2: np.ndarray, rowsub: np.ndarray, N: int, G: int) -
     return total
 
 
+# DRAM bytes (read + write) per k_sparse_attn2 launch from an ncu capture,
+# by workload; entries scaled from a smaller capture say so in the design
+# notes.  None where no capture of the current kernel exists.
+ATTN_TRAFFIC = {"llama_128k": None}
+
+# fp64 multiply-add rate of this machine's B200s (DFMA and mma.sync m8n8k4 alike),
+# measured by a register-resident microbenchmark: 37 TFLOP/s = 18.5 T FMA/s
+FP64_FMA_PER_S = 18.5e12
+
+
+def prefix_lengths(torch, cfg, bufs, filtered: bool, w):
+    """Entries of each segment's order the plan sorts: all candidates for the
+    full plan; for the filtered plan whole blocks up to the number of
+    candidates with s >= M + ln(tau Z / Bk) - 1e-3 (the bound the planner
+    uses).  Returns the total over every (b, kvh, s)."""
+    B, Hkv = w.B, w.Hkv
+    S = (w.N + 127) // 128
+    T = (64 * (S - 2) ** 2) if S >= 2 else 0
+    if not filtered or w.tau <= 0.0:
+        return B * Hkv * T
+    cnt = torch.tensor([max(0, 128 * s - 192) for s in range(S)], dtype=torch.int64, device=bufs["scores"].device)
+    seg = torch.repeat_interleave(torch.arange(S, device=cnt.device), cnt)
+    stats = bufs["seg_stats"].view(B * Hkv, S, 2).double()
+    total = 0
+    for u in range(B * Hkv):
+        thr = stats[u, :, 0] + torch.log(w.tau * stats[u, :, 1] / 64.0) - 1e-3
+        sc = bufs["scores"][u * T:(u + 1) * T].double()
+        nhi = torch.zeros(S, dtype=torch.int64, device=cnt.device).index_add_(0, seg, (sc >= thr[seg]).long())
+        total += int(torch.minimum(cnt, 64 * ((nhi + 63) // 64)).sum())
+    return total
+
+
+def plan_kernel_roofline(s2o, torch, cfg, Q, K, bufs, filtered, w, peaks, peak_src, reps=3):
+    """Median device time of each plan kernel over `reps` plans (events on the
+    caller's stream between the kernels), and its compulsory HBM bytes:
+      k_pool       read Q, write the fp64 pooled queries
+      k_score      read K and the pooled queries, write the candidate scores
+                   and the causal half of the (max, sumexp) partials; also its
+                   fp64 multiply-adds (128 per admissible key per segment)
+      k_seg_stats  read the partials, write (M, Z)
+      k_bucket_plan read every candidate score, write the staged (key, index)
+                   pairs of the sorted prefix
+      k_bucket_sort read the staged pairs, write perm and the sorted scores
+      k_mass_stop  read the sorted scores of the prefix, write C(s)
+    (the prefix is every candidate for the full plan)."""
+    B, Hq, Hkv, N, d = w.B, w.Hq, w.Hkv, w.N, w.d
+    S = (N + 127) // 128
+    T = B * Hkv * ((64 * (S - 2) ** 2) if S >= 2 else 0)
+    L = prefix_lengths(torch, cfg, bufs, filtered, w)
+    parts = B * Hkv * S * (S + 1) / 2 * 8
+    bytes_of = {
+        "k_pool": B * Hq * N * d * 2 + B * Hkv * S * d * 8,
+        "k_score": B * Hkv * N * d * 2 + B * Hkv * S * d * 8 + T * 4 + parts,
+        "k_seg_stats": parts + B * Hkv * S * 16,
+        "k_bucket_plan": T * 4 + L * 8,
+        "k_bucket_sort": L * 8 + L * 8,
+        "k_mass_stop": L * 4 + B * Hkv * S * 4,
+    }
+    # admissible keys of every segment: e(s) = min(N, 128 (s + 1))
+    dfma = B * Hkv * d * sum(min(N, 128 * (s + 1)) for s in range(S))
+    s2o.stage_timing(True)
+    try:
+        runs = []
+        for _ in range(reps):
+            s2o.plan(cfg, Q, K, bufs, filtered=filtered)
+            runs.append(s2o.last_stage_times())
+    finally:
+        s2o.stage_timing(False)
+    hbm = float(peaks["hbm_gbs"])
+    out = {"plan": "filtered" if filtered else "full", "sorted_prefix_entries": L, "candidates": T,
+           "peak_hbm_gbs": hbm, "peak_source": f"{peak_src} HBM copy", "kernels": {}}
+    names = [n for n, _ in runs[0]]
+    total_ms, total_bytes = 0.0, 0.0
+    for i, name in enumerate(names):
+        ms = float(np.median([r[i][1] for r in runs]))
+        total_ms += ms
+        ent = {"ms": ms}
+        if name in bytes_of:
+            b = float(bytes_of[name])
+            total_bytes += b
+            ent.update(bytes=b, gbs=b / (ms * 1e-3) / 1e9, frac_hbm=b / (ms * 1e-3) / 1e9 / hbm)
+        if name == "k_score":
+            ent.update(fp64_fma=float(dfma), fp64_fma_per_s=dfma / (ms * 1e-3),
+                       frac_fp64=dfma / (ms * 1e-3) / FP64_FMA_PER_S,
+                       note="exact fp64 dot products (half-ulp fp32 scores): bound by the fp64 pipe, whose "
+                            "floor is above the HBM floor of its bytes")
+        out["kernels"][name] = ent
+    out["total_ms"] = total_ms
+    out["total_bytes"] = total_bytes
+    out["total_gbs"] = total_bytes / (total_ms * 1e-3) / 1e9
+    out["total_frac_hbm"] = out["total_gbs"] / hbm
+    return out
+
+
 def reduce_max_ms(ms: float, dist=None, device="cpu") -> float:
     """Max over ranks of a per-rank time (the slowest rank bounds the job)."""
     if dist is None or not dist.is_initialized() or dist.get_world_size() == 1:
@@ -189,6 +283,82 @@ def cpu_oracle_sample(Q, K, V, tau, seconds=15.0):
     return flops / dt / 1e12, sample, dt
 
 
+_FORK = {}  # arrays the all-cores oracle workers inherit (fork, before any CUDA call)
+
+
+def _oracle_item(item):
+    """One (KV head, segment) of the oracle: plan + attention of every query
+    head of the group; returns its dense-equivalent FLOPs."""
+    from oracle import s2o_oracle as O
+    kvh, s = item
+    Q, K, V, p = _FORK["Q"], _FORK["K"], _FORK["V"], _FORK["p"]
+    N, d = Q.shape[2], Q.shape[3]
+    G = Q.shape[1] // K.shape[1]
+    sp = O.plan_segment(Q, K, 0, kvh, s, G, p)
+    O.attention_segment(Q, K, V, 0, kvh, s, G, sp.keep, p)
+    r0, r1 = O.segment_rows(N, s, p)
+    return G * 4.0 * d * float(np.sum(np.arange(r0, r1, dtype=np.float64) + 1))
+
+
+def _one_blas_thread():
+    from threadpoolctl import threadpool_limits
+    _FORK["limit"] = threadpool_limits(1)
+
+
+def host_cores():
+    """(logical CPUs of the host, CPUs this process may run on)."""
+    try:
+        aff = len(os.sched_getaffinity(0))
+    except AttributeError:
+        aff = os.cpu_count() or 1
+    return os.cpu_count() or 1, aff
+
+
+def cpu_oracle_all_cores(Q, K, V, tau, seconds=15.0, max_procs=64):
+    """The same oracle items as cpu_oracle_sample, spread over one process per
+    available core (at most max_procs, to bound host memory: each item widens
+    up to 3 x 134 MB of K/V rows to fp64), one BLAS thread each.  Uses a fork
+    pool, so it must run before the process touches CUDA.  Returns
+    (dense-equivalent TFLOP/s, processes, sample text)."""
+    import multiprocessing as mp
+    from oracle import s2o_oracle as O
+
+    p = O.Params(tau=tau)
+    N = Q.shape[2]
+    S = O.num_segments(N, p)
+    order = sorted({S - 1, S // 2, S // 4, 3 * S // 4, 3, 2, 1, 0} | set(range(S - 2, 3, -97)))
+    items = [(kvh, s) for s in order for kvh in range(K.shape[1])]
+    procs = max(1, min(max_procs, host_cores()[1]))
+    _FORK.update(Q=Q, K=K, V=V, p=p)
+    flops, done = 0.0, 0
+    ctx = mp.get_context("fork")
+    pool = ctx.Pool(procs, initializer=_one_blas_thread)
+    try:
+        t0 = time.perf_counter()
+        for f in pool.imap_unordered(_oracle_item, items * 64, chunksize=1):
+            flops += f
+            done += 1
+            if time.perf_counter() - t0 > seconds:
+                break
+        dt = time.perf_counter() - t0
+    finally:
+        pool.terminate()
+        pool.join()
+        _FORK.clear()
+    sample = (f"{done} (KV head, segment) items of the same segment list over all KV heads, {procs} processes "
+              f"x 1 BLAS thread, {dt:.1f} s wall; items still running at the cut are not counted")
+    return flops / dt / 1e12, procs, sample
+
+
+def cpu_baseline_entry(Qn, Kn, Vn, tau):
+    v1, sample, _ = cpu_oracle_sample(Qn, Kn, Vn, tau, seconds=15.0)
+    vall, procs, sample_all = cpu_oracle_all_cores(Qn, Kn, Vn, tau, seconds=15.0)
+    ncpu, naff = host_cores()
+    return {"value": v1, "unit": "TFLOP/s", "cores": 1, "threads": 1, "kind": "oracle", "sample": sample,
+            "host_cores": ncpu, "affinity_cores": naff,
+            "value_all_cores": vall, "all_cores_processes": procs, "all_cores_sample": sample_all}
+
+
 def bench_config(w, world: int, plan: str) -> dict:
     """The workload description both arms print."""
     return {"workload": w.name, "B": w.B, "Hq": w.Hq, "Hkv": w.Hkv, "N": w.N, "d": w.d, "tau": w.tau,
@@ -217,10 +387,135 @@ def reference_arm(args, w, world, rank):
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1000.0 * total / max(1, args.steps),
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
         "config": bench_config(w, world, args.plan),
-        "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": 1, "kind": "oracle", "sample": sample},
+        "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": 1, "threads": 1, "kind": "oracle",
+                         "sample": sample, "host_cores": host_cores()[0], "affinity_cores": host_cores()[1]},
         "e2e": {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }
     print(json.dumps(line), flush=True)
+
+
+def _median_ms(torch, fn, reps=3, warm=2):
+    for _ in range(warm):
+        fn()
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(reps)]
+    for e0, e1 in ev:
+        e0.record()
+        fn()
+        e1.record()
+    torch.cuda.synchronize()
+    return float(np.median([e0.elapsed_time(e1) for e0, e1 in ev]))
+
+
+def mse_on_device(torch, Os, Od):
+    """Mean over every output element of (Os - Od)^2, in fp64, head by head;
+    also the mean of Od^2 (to give the relative figure)."""
+    sse = sq = 0.0
+    for b in range(Os.shape[0]):
+        for h in range(Os.shape[1]):
+            dd = Od[b, h].double()
+            diff = Os[b, h].double() - dd
+            sse += float((diff * diff).sum())
+            sq += float((dd * dd).sum())
+    n = Os.numel()
+    return sse / n, sq / n
+
+
+def c_histogram(nb: np.ndarray, N: int):
+    """Per-segment kept fraction C(s) / n_blk(s) over the segments that have
+    candidates, binned; and where, per KV head, the first segment that does
+    not keep every block lies."""
+    S = nb.shape[-1]
+    nblk = np.array([max(0, 128 * s - 192) // 64 for s in range(S)])
+    segs = np.nonzero(nblk > 0)[0]
+    frac = nb[..., segs] / nblk[segs]
+    edges = [0.0, 1e-9, 0.1, 0.2, 0.3, 0.4, 0.5, 0.6, 0.7, 0.8, 0.9, 1.0 - 1e-9, 1.0 + 1e-9]
+    labels = ["0", "(0,0.1]", "(0.1,0.2]", "(0.2,0.3]", "(0.3,0.4]", "(0.4,0.5]", "(0.5,0.6]", "(0.6,0.7]",
+              "(0.7,0.8]", "(0.8,0.9]", "(0.9,1)", "1"]
+    counts, _ = np.histogram(frac.ravel(), bins=edges)
+    first_cut = []
+    for row in frac.reshape(-1, len(segs)):
+        cut = np.nonzero(row < 1.0)[0]
+        first_cut.append(int(segs[cut[0]]) if cut.size else S)
+    ranges = []
+    step = max(1, S // 16)
+    for a in range(0, S, step):
+        sel = (segs >= a) & (segs < a + step)
+        if sel.any():
+            ranges.append({"segments": [a, min(S, a + step) - 1], "mean_kept_fraction": float(frac[..., sel].mean()),
+                           "key_positions": [128 * a, 128 * min(S, a + step)]})
+    return {"bins": dict(zip(labels, [int(c) for c in counts])), "segments_with_candidates": int(frac.size),
+            "first_segment_not_keeping_all_blocks": {"median": float(np.median(first_cut)),
+                                                     "min": int(min(first_cut)), "max": int(max(first_cut))},
+            "by_position": ranges}
+
+
+def report_main(args):
+    """Accuracy and per-configuration report (not the headline benchmark):
+    one JSON line per configuration with sparsity, MSE against dense causal
+    attention, plan and attention time; the tau sweep with the contiguous
+    block comparator at the same per-segment block count; the C(s) histogram
+    of the flat workload.  MSE is measured on the library's fp32 outputs: the
+    plan's sparse output against its tau = 0 output (which keeps every
+    admissible key, i.e. dense causal attention)."""
+    import torch
+    import score_keys_pooled_b200 as s2o
+    from score_keys_pooled_b200 import synth
+
+    dev = torch.device("cuda", 0)
+    torch.cuda.set_device(dev)
+    what = args.report
+    names = {"configs": ["tiny_1k", "llama_16k", "llama_128k", "sweep_64k", "flat_128k"],
+             "sweep": ["sweep_64k"]}[what]
+    for name in names:
+        w = synth.WORKLOADS[name]
+        Qn, Kn, Vn = synth.generate_workload(w, seed=0)
+        to_dev = lambda a: torch.from_numpy(a.view(np.int16)).to(dev)
+        Q, K, V = to_dev(Qn), to_dev(Kn), to_dev(Vn)
+        del Qn, Kn, Vn
+        G = w.Hq // w.Hkv
+        dense = dense_flops(w.B, w.Hq, w.N, w.d)
+        pairs_dense = w.B * w.Hq * w.N * (w.N + 1) / 2.0
+        taus = synth.TAU_SWEEP if what == "sweep" else (w.tau,)
+        # dense causal attention: tau = 0 keeps every block
+        cfg0 = s2o.make_config(w.B, w.Hq, w.Hkv, w.N, tau=0.0)
+        bufs = s2o.alloc_plan(cfg0, dev)
+        s2o.plan(cfg0, Q, K, bufs)
+        Od = s2o.attention(cfg0, Q, K, V, bufs["perm"], bufs["nblocks"], out_dtype=s2o.OUT_F32)
+        dense_ms = _median_ms(torch, lambda: s2o.attention(cfg0, Q, K, V, bufs["perm"], bufs["nblocks"], out_dtype=s2o.OUT_F32))
+        Os = torch.empty_like(Od)
+        for tau in taus:
+            cfg = s2o.make_config(w.B, w.Hq, w.Hkv, w.N, tau=tau)
+            plan_ms = _median_ms(torch, lambda: s2o.plan(cfg, Q, K, bufs, filtered=True))
+            full_ms = _median_ms(torch, lambda: s2o.plan(cfg, Q, K, bufs, filtered=False), reps=2, warm=1)
+            s2o.plan(cfg, Q, K, bufs, filtered=False)
+            attn_ms = _median_ms(torch, lambda: s2o.attention(cfg, Q, K, V, bufs["perm"], bufs["nblocks"], Os, out_dtype=s2o.OUT_F32))
+            if s2o.last_device_error() != 0:
+                raise RuntimeError(f"device error in the report ({name}, tau={tau})")
+            nb = bufs["nblocks"].cpu().numpy().reshape(w.B, w.Hkv, -1)
+            density = kept_pairs(nb, w.N, G) / pairs_dense
+            mse, msq = mse_on_device(torch, Os, Od)
+            line = {"report": what, "workload": name, "tau": tau, "B": w.B, "Hq": w.Hq, "Hkv": w.Hkv, "N": w.N,
+                    "kept_pair_fraction": density, "sparsity": 1.0 - density,
+                    "mse_vs_dense": mse, "relative_mse": mse / msq if msq else None,
+                    "plan_filtered_ms": plan_ms, "plan_full_ms": full_ms, "attention_ms": attn_ms,
+                    "dense_attention_ms": dense_ms, "step_tflops_dense_equiv": dense / ((plan_ms + attn_ms) * 1e-3) / 1e12,
+                    "attention_speedup_vs_dense_kernel": dense_ms / attn_ms}
+            if what == "sweep" or name == "sweep_64k":
+                # contiguous top-k: original-order blocks by pooled mass, the same C(s) per segment
+                pc = torch.empty_like(bufs["perm"])
+                s2o.plan_contiguous(cfg, bufs["scores"], bufs["seg_stats"], bufs["nblocks"], pc)
+                Oc = s2o.attention(cfg, Q, K, V, pc, bufs["nblocks"], out_dtype=s2o.OUT_F32)
+                if s2o.last_device_error() != 0:
+                    raise RuntimeError("device error in the contiguous comparator")
+                msec, _ = mse_on_device(torch, Oc, Od)
+                line.update(contiguous_mse_vs_dense=msec,
+                            contiguous_over_s2o_mse=(msec / mse) if mse > 0 else None)
+                del Oc, pc
+            if name == "flat_128k" or what == "configs":
+                line["C_histogram"] = c_histogram(nb, w.N)
+            print(json.dumps(line), flush=True)
+        del bufs, Od, Os, Q, K, V
+        torch.cuda.empty_cache()
 
 
 def main():
@@ -238,7 +533,13 @@ def main():
     ap.add_argument("--plan", default="filtered", choices=["full", "filtered"],
                     help="s2o_plan (every segment fully ordered) or s2o_plan_filtered (only the prefix the "
                          "stop rule can reach; same kept sets and output)")
+    ap.add_argument("--report", default=None, choices=["configs", "sweep"],
+                    help="instead of the benchmark line, print one accuracy/timing line per configuration "
+                         "(configs) or per tau of the sweep workload with the contiguous comparator (sweep)")
     args = ap.parse_args()
+    if args.report:
+        report_main(args)
+        return
     if args.warmup < 3 and args.impl == "s2o":
         ap.error("--warmup must be >= 3")
 
@@ -252,6 +553,14 @@ def main():
         reference_arm(args, w, world, rank)
         return
 
+    # each rank solves an independent problem (its own seed): weak scaling
+    Qn, Kn, Vn = synth.generate_workload(w, seed=rank)
+
+    # the CPU baseline forks its worker pool, so it runs before any CUDA call
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        cpu = cpu_baseline_entry(Qn, Kn, Vn, w.tau)
+
     import torch
     import score_keys_pooled_b200 as s2o
 
@@ -263,8 +572,6 @@ def main():
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300))
     dev = torch.device("cuda", local)
 
-    # each rank solves an independent problem (its own seed): weak scaling
-    Qn, Kn, Vn = synth.generate_workload(w, seed=rank)
     to_dev = lambda a: torch.from_numpy(a.view(np.int16)).to(dev)
     Q, K, V = to_dev(Qn), to_dev(Kn), to_dev(Vn)
     cfg = s2o.make_config(w.B, w.Hq, w.Hkv, w.N, tau=w.tau)
@@ -336,14 +643,32 @@ def main():
     peaks, peak_src = load_peaks()
     attn_mean = float(np.mean(attn_ms))
     achieved = 4.0 * w.d * pairs / (attn_mean * 1e-3) / 1e12
-    peak = float(peaks.get("bf16_tflops_sustained", peaks["bf16_tflops"]))
-    # DRAM bytes per launch of k_sparse_attn2 from an ncu capture of the 32K
-    # workload (764.7 MB), scaled by the rows processed to the 128K launch;
-    # None for other workloads
-    traffic = 3.06e9 if w.name == "llama_128k" else None
+    # the burst peak: each attention launch runs for tens of milliseconds,
+    # not the seconds-long loop the sustained figure was taken over
+    peak = float(peaks["bf16_tflops"])
+    peak_sus = float(peaks.get("bf16_tflops_sustained", peak))
     roofline = {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
-                "frac": achieved / peak, "traffic": traffic, "kernel": "k_sparse_attn2",
-                "peak_source": f"{peak_src} bf16 sustained"}
+                "frac": achieved / peak, "traffic": ATTN_TRAFFIC.get(w.name), "kernel": "k_sparse_attn2",
+                "peak_source": f"{peak_src} bf16 burst (cuBLAS)",
+                "peak_sustained": peak_sus, "frac_of_sustained": achieved / peak_sus}
+
+    # per-kernel time of the plan (CUDA events between its kernels) against
+    # each kernel's compulsory HBM bytes
+    plan_roofline = plan_kernel_roofline(s2o, torch, cfg, Q, K, bufs, filtered, w, peaks, peak_src)
+
+    # accuracy: MSE of the sparse output against dense causal attention (the
+    # tau = 0 plan keeps every admissible key), both from fp32 outputs
+    Os = s2o.attention(cfg, Q, K, V, bufs["perm"], bufs["nblocks"], out_dtype=s2o.OUT_F32)
+    cfg0 = s2o.make_config(w.B, w.Hq, w.Hkv, w.N, tau=0.0)
+    s2o.plan(cfg0, Q, K, bufs)
+    Od = s2o.attention(cfg0, Q, K, V, bufs["perm"], bufs["nblocks"], out_dtype=s2o.OUT_F32)
+    mse, msq = mse_on_device(torch, Os, Od)
+    accuracy = {"mse_vs_dense": mse, "relative_mse": mse / msq if msq else None,
+                "definition": "mean over all output elements of (O_sparse - O_dense)^2, fp32 outputs of the "
+                              "library; dense = the tau = 0 plan"}
+    del Os, Od
+    torch.cuda.empty_cache()
+    s2o.plan(cfg, Q, K, bufs, filtered=filtered)
 
     # the pages' run-time stop: the full order, then the attention kernel
     # deciding the stop itself; timed after the headline, reported beside it
@@ -450,11 +775,6 @@ def main():
                "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h)}
         del arena
 
-    cpu = None
-    if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        v, sample, _ = cpu_oracle_sample(Qn, Kn, Vn, w.tau, seconds=15.0)
-        cpu = {"value": v, "unit": "TFLOP/s", "cores": 1, "kind": "oracle", "sample": sample}
-
     if rank == 0:
         line = {
             "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps,
@@ -467,8 +787,9 @@ def main():
             "ranking": ranking,
             "qperm": qperm,
             "attention_only_tflops": whole_job_tflops(world, dense, attn_mean),
-            "kept_pair_fraction": density,
-            "roofline": roofline, "cpu_baseline": cpu, "e2e": e2e, "gpu_launches": launches,
+            "kept_pair_fraction": density, "accuracy": accuracy,
+            "roofline": roofline, "plan_roofline": plan_roofline,
+            "cpu_baseline": cpu, "e2e": e2e, "gpu_launches": launches,
             "clocks": clk.summary(),
         }
         print(json.dumps(line), flush=True)
