@@ -82,10 +82,12 @@ def kept_pairs_qperm(nblocks2: np.ndarray, rowsub: np.ndarray, N: int, G: int) -
     return total
 
 
-# DRAM bytes (read + write) per k_sparse_attn2 launch from an ncu capture,
-# by workload; entries scaled from a smaller capture say so in the design
-# notes.  None where no capture of the current kernel exists.
-ATTN_TRAFFIC = {"llama_128k": None}
+# DRAM bytes (read + write) per k_sparse_attn2 launch from an ncu capture of
+# the current kernel, by workload.  llama_128k: the capture of llama_32k at
+# the same kept fraction (tau = 4e-3, 26.7 % of pairs; 669.8 MB) scaled by the
+# rows processed (x 4: Q, O, K and V all grow with N).  None where no capture
+# exists.
+ATTN_TRAFFIC = {"llama_128k": 2.679e9, "llama_32k@0.004": 6.698e8}
 
 # fp64 multiply-add rate of this machine's B200s (DFMA and mma.sync m8n8k4 alike),
 # measured by a register-resident microbenchmark: 37 TFLOP/s = 18.5 T FMA/s
@@ -533,6 +535,8 @@ def main():
     ap.add_argument("--plan", default="filtered", choices=["full", "filtered"],
                     help="s2o_plan (every segment fully ordered) or s2o_plan_filtered (only the prefix the "
                          "stop rule can reach; same kept sets and output)")
+    ap.add_argument("--tau", type=float, default=None,
+                    help="override the workload's tau (e.g. to profile a small workload at the headline's density)")
     ap.add_argument("--report", default=None, choices=["configs", "sweep"],
                     help="instead of the benchmark line, print one accuracy/timing line per configuration "
                          "(configs) or per tau of the sweep workload with the contiguous comparator (sweep)")
@@ -545,6 +549,9 @@ def main():
 
     from score_keys_pooled_b200 import synth
     w = synth.WORKLOADS[args.workload]
+    if args.tau is not None:
+        import dataclasses
+        w = dataclasses.replace(w, tau=args.tau)
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
     local = int(os.environ.get("LOCAL_RANK", "0"))
@@ -648,7 +655,8 @@ def main():
     peak = float(peaks["bf16_tflops"])
     peak_sus = float(peaks.get("bf16_tflops_sustained", peak))
     roofline = {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
-                "frac": achieved / peak, "traffic": ATTN_TRAFFIC.get(w.name), "kernel": "k_sparse_attn2",
+                "frac": achieved / peak, "traffic": ATTN_TRAFFIC.get(w.name if args.tau is None else f"{w.name}@{w.tau:g}"),
+                "kernel": "k_sparse_attn2",
                 "peak_source": f"{peak_src} bf16 burst (cuBLAS)",
                 "peak_sustained": peak_sus, "frac_of_sustained": achieved / peak_sus}
 
