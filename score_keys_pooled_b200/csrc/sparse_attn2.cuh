@@ -238,6 +238,159 @@ struct Attn2Args {
   uint32_t spin;
 };
 
+// The loader warps of the attention kernels (warp kLoadWarp0 = K ring and
+// Q, warp kLoadWarp0 + 1 = V ring): for tile t of the key walk, gather its
+// 128 K (or V) rows by index into ring stage t % stages once the stage is
+// free, and arrive on the stage's full barrier after the copies landed.
+template <bool ONLINE, bool QPERM>
+__device__ __forceinline__ void attn_load_ring(const Attn2Args& a, const CUtensorMap* tmQ, uint32_t sbase,
+                                               uint8_t* sgen, int warp, int lane, int b, int bk, int s, int h0,
+                                               int row0, const Walk2& wk, int ntiles, int C0,
+                                               volatile int* stop_word) {
+  auto bar = [&](int k) { return sbase + kOff2Bar + 8u * (uint32_t)k; };
+  const bool is_k = warp == kLoadWarp0;
+  const int nst = is_k ? kStagesK : kStagesV;
+  const int bar_full = is_k ? kBarKFull : kBarVFull;
+  const int bar_empty = is_k ? kBarKEmpty : kBarVEmpty;
+  const uint32_t ring = sbase + (is_k ? kOff2K : kOff2V);
+  const uint16_t* kv = (is_k ? a.K : a.V) + (size_t)bk * a.N * kD;
+  if (is_k && lane == 0) {
+    mbar_expect_tx(bar(kBarQFull), 2 * kTile2Bytes);
+#pragma unroll
+    for (int qi = 0; qi < 2; ++qi)
+#pragma unroll
+      for (int half = 0; half < 2; ++half)
+        tma_load_2d(sbase + kOff2Q + qi * kTile2Bytes + half * (128 * 128), tmQ, 64 * half,
+                    (b * a.Hq + h0 + qi) * a.N + row0, bar(kBarQFull));
+  }
+  const int32_t* pseg = a.perm + (size_t)bk * a.T + cand_offset(s);
+  const int cand_hi = kLq * s - kWin;
+  // raw key indices of tile rows 4 lane .. 4 lane + 3 (loaded, not yet used)
+  auto fetch_keys = [&](int t, int* y) {
+    int j0;
+    const int kind = walk2_block(wk, s, 2 * t + (lane >> 4), j0);
+    const int rr = (4 * lane) & 63;
+    if (kind == 2) {
+      const int32_t* ps = pseg;
+      if (QPERM && j0 >= C0) {
+        ps = a.perm1 + (size_t)bk * a.T + cand_offset(s);
+        j0 -= C0;
+      }
+      const int4 v = *reinterpret_cast<const int4*>(ps + kBk * j0 + rr);
+      y[0] = v.x; y[1] = v.y; y[2] = v.z; y[3] = v.w;
+    } else {
+#pragma unroll
+      for (int k = 0; k < 4; ++k) y[k] = kind == 3 ? -1 : j0 + rr + k;
+    }
+  };
+  // checked keys (-1: a zero row: an empty half or a key past N) into the
+  // warp's table: row r = 2 jj + p at keys[p][jj]; true if any is -1
+  int32_t* keys = reinterpret_cast<int32_t*>(sgen + kOff2Keys + (is_k ? 0 : 512));
+  const uint32_t keys_s = sbase + kOff2Keys + (is_k ? 0u : 512u);
+  auto stage_keys = [&](int t, const int* y) {
+    int j0;
+    const int kind = walk2_block(wk, s, 2 * t + (lane >> 4), j0);
+    int k4[4];
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+      int j = y[k];
+      if (kind == 2) {
+        if (j < kSink || j >= cand_hi) {  // caller-supplied plan out of Cand(s)
+          set_error(kErrBadPlan);
+          j = kSink;
+        }
+      } else if (j >= a.N) {
+        j = -1;
+      }
+      k4[k] = j;
+    }
+    // rows 4 lane + k: parity k & 1, slot 2 lane + (k >> 1)
+    *reinterpret_cast<int2*>(keys + 2 * lane) = make_int2(k4[0], k4[2]);
+    *reinterpret_cast<int2*>(keys + 64 + 2 * lane) = make_int2(k4[1], k4[3]);
+    __syncwarp();
+    return __any_sync(0xffffffffu, k4[0] < 0 || k4[1] < 0 || k4[2] < 0 || k4[3] < 0);
+  };
+  // this lane copies 16-byte chunk q of rows 2 jj + sel (swizzle atom q / 8,
+  // chunk q % 8 xor row % 8); its destination offsets repeat with jj % 4
+  const int q = lane & 15, sel = lane >> 4;
+  uint32_t dsw[4];
+#pragma unroll
+  for (int m = 0; m < 4; ++m)
+    dsw[m] = (uint32_t)(q >> 3) * (128 * 128) + (uint32_t)sel * 128 +
+             ((uint32_t)((q & 7) ^ ((2 * m + sel) & 7)) << 4);
+  const char* src0 = reinterpret_cast<const char*>(kv) + 16 * q;
+  const uint32_t ktab = keys_s + 256u * (uint32_t)sel;
+  int y[4];
+  if (ntiles > 0) fetch_keys(0, y);
+  // with the run-time stop a tile past the stop point is not needed: the
+  // last products issued after a stop at chunk c read K of chunk c + 1
+  auto not_needed = [&](int t) {
+    const int sc = *stop_word;
+    return sc != kNoStop && t > sc / 2 + 1;
+  };
+  for (int t = 0; t < ntiles; ++t) {
+    const int st = t % nst;
+    const int round = t / nst;
+    if (ONLINE && not_needed(t)) break;
+    const bool ragged = stage_keys(t, y);
+    if (t + 1 < ntiles) fetch_keys(t + 1, y);  // in flight while this stage fills
+    bool okw;
+    if (!ONLINE) {
+      okw = warp_wait(bar(bar_empty + st), (uint32_t)((round & 1) ^ 1), a.spin);
+    } else {
+      // lane 0 waits for the stage or for a stop that makes it unneeded;
+      // after a free stage every lane acquires the barrier itself
+      int r = 0;
+      if (lane == 0) {
+        for (uint32_t it = 0; it < a.spin && r == 0; ++it) {
+          if (mbar_try_wait(bar(bar_empty + st), (uint32_t)((round & 1) ^ 1))) r = 1;
+          else if (not_needed(t)) r = 2;
+        }
+      }
+      r = __shfl_sync(0xffffffffu, r, 0);
+      if (r == 2) break;
+      okw = r == 1 && warp_wait(bar(bar_empty + st), (uint32_t)((round & 1) ^ 1), a.spin);
+    }
+    if (!okw) {
+      if (lane == 0) set_error(kErrTimeout);
+      break;
+    }
+    const uint32_t dst0 = ring + st * kTile2Bytes;
+    // 64 copies per lane; the key table is read four keys at a time.  A tile
+    // with a zero row (rare: an empty half or keys past N) takes the loop
+    // with per-row source sizes; the branch stays outside the unrolled loop
+    // so that each copy issues once.
+    if (!ragged) {
+#pragma unroll
+      for (int j4 = 0; j4 < 16; ++j4) {
+        int4 kk;
+        asm volatile("ld.shared.v4.s32 {%0, %1, %2, %3}, [%4];\n"
+                     : "=r"(kk.x), "=r"(kk.y), "=r"(kk.z), "=r"(kk.w)
+                     : "r"(ktab + 16u * (uint32_t)j4)
+                     : "memory");
+        const int key4[4] = {kk.x, kk.y, kk.z, kk.w};
+#pragma unroll
+        for (int m = 0; m < 4; ++m)
+          cp_async16(dst0 + dsw[m] + 256u * (uint32_t)(4 * j4 + m), src0 + (size_t)key4[m] * (kD * 2), 16u);
+      }
+    } else {
+#pragma unroll 4
+      for (int jj = 0; jj < 64; ++jj) {
+        const int key = keys[64 * sel + jj];
+        cp_async16(dst0 + dsw[jj & 3] + 256u * (uint32_t)jj, src0 + (size_t)(key < 0 ? 0 : key) * (kD * 2),
+                   key < 0 ? 0u : 16u);
+      }
+    }
+    cp_async_wait_all();
+    fence_proxy_async_smem();  // generic-proxy writes -> tensor-core reads
+    __syncwarp();
+    if (lane == 0) mbar_arrive(bar(bar_full + st));
+  }
+  // Q's TMA tiles may still be landing if the issuers gave up waiting for
+  // them: shared memory must not change after the CTA ends
+  if (is_k && lane == 0 && !mbar_wait_bounded(bar(kBarQFull), 0)) set_error(kErrTimeout);
+}
+
 // ONLINE selects the run-time stop, QPERM the two query sub-segments; the
 // planned-stop kernel is compiled without any of their code
 template <bool ONLINE, bool QPERM = false>
@@ -315,147 +468,8 @@ __global__ void __launch_bounds__(kAttn2Threads, 1)
     // layout the tensor core reads (one TMA gather4 per four rows issues far
     // slower than the load/store unit takes these copies).
     regs_decrease<kRegsOther>();
-    const bool is_k = warp == kLoadWarp0;
-    const int nst = is_k ? kStagesK : kStagesV;
-    const int bar_full = is_k ? kBarKFull : kBarVFull;
-    const int bar_empty = is_k ? kBarKEmpty : kBarVEmpty;
-    const uint32_t ring = sbase + (is_k ? kOff2K : kOff2V);
-    const uint16_t* kv = (is_k ? a.K : a.V) + (size_t)bk * a.N * kD;
-    if (is_k && lane == 0) {
-      mbar_expect_tx(bar(kBarQFull), 2 * kTile2Bytes);
-#pragma unroll
-      for (int qi = 0; qi < 2; ++qi)
-#pragma unroll
-        for (int half = 0; half < 2; ++half)
-          tma_load_2d(sbase + kOff2Q + qi * kTile2Bytes + half * (128 * 128), &tmQ, 64 * half,
-                      (b * a.Hq + h0 + qi) * a.N + row0, bar(kBarQFull));
-    }
-    const int32_t* pseg = a.perm + (size_t)bk * a.T + cand_offset(s);
-    const int cand_hi = kLq * s - kWin;
-    // raw key indices of tile rows 4 lane .. 4 lane + 3 (loaded, not yet used)
-    auto fetch_keys = [&](int t, int* y) {
-      int j0;
-      const int kind = walk2_block(wk, s, 2 * t + (lane >> 4), j0);
-      const int rr = (4 * lane) & 63;
-      if (kind == 2) {
-        const int32_t* ps = pseg;
-        if (QPERM && j0 >= C0) {
-          ps = a.perm1 + (size_t)bk * a.T + cand_offset(s);
-          j0 -= C0;
-        }
-        const int4 v = *reinterpret_cast<const int4*>(ps + kBk * j0 + rr);
-        y[0] = v.x; y[1] = v.y; y[2] = v.z; y[3] = v.w;
-      } else {
-#pragma unroll
-        for (int k = 0; k < 4; ++k) y[k] = kind == 3 ? -1 : j0 + rr + k;
-      }
-    };
-    // checked keys (-1: a zero row: an empty half or a key past N) into the
-    // warp's table: row r = 2 jj + p at keys[p][jj]; true if any is -1
-    int32_t* keys = reinterpret_cast<int32_t*>(sgen + kOff2Keys + (is_k ? 0 : 512));
-    const uint32_t keys_s = sbase + kOff2Keys + (is_k ? 0u : 512u);
-    auto stage_keys = [&](int t, const int* y) {
-      int j0;
-      const int kind = walk2_block(wk, s, 2 * t + (lane >> 4), j0);
-      int k4[4];
-#pragma unroll
-      for (int k = 0; k < 4; ++k) {
-        int j = y[k];
-        if (kind == 2) {
-          if (j < kSink || j >= cand_hi) {  // caller-supplied plan out of Cand(s)
-            set_error(kErrBadPlan);
-            j = kSink;
-          }
-        } else if (j >= a.N) {
-          j = -1;
-        }
-        k4[k] = j;
-      }
-      // rows 4 lane + k: parity k & 1, slot 2 lane + (k >> 1)
-      *reinterpret_cast<int2*>(keys + 2 * lane) = make_int2(k4[0], k4[2]);
-      *reinterpret_cast<int2*>(keys + 64 + 2 * lane) = make_int2(k4[1], k4[3]);
-      __syncwarp();
-      return __any_sync(0xffffffffu, k4[0] < 0 || k4[1] < 0 || k4[2] < 0 || k4[3] < 0);
-    };
-    // this lane copies 16-byte chunk q of rows 2 jj + sel (swizzle atom q / 8,
-    // chunk q % 8 xor row % 8); its destination offsets repeat with jj % 4
-    const int q = lane & 15, sel = lane >> 4;
-    uint32_t dsw[4];
-#pragma unroll
-    for (int m = 0; m < 4; ++m)
-      dsw[m] = (uint32_t)(q >> 3) * (128 * 128) + (uint32_t)sel * 128 +
-               ((uint32_t)((q & 7) ^ ((2 * m + sel) & 7)) << 4);
-    const char* src0 = reinterpret_cast<const char*>(kv) + 16 * q;
-    const uint32_t ktab = keys_s + 256u * (uint32_t)sel;
-    int y[4];
-    if (ntiles > 0) fetch_keys(0, y);
-    // with the run-time stop a tile past the stop point is not needed: the
-    // last products issued after a stop at chunk c read K of chunk c + 1
-    auto not_needed = [&](int t) {
-      const int sc = *stop_word;
-      return sc != kNoStop && t > sc / 2 + 1;
-    };
-    for (int t = 0; t < ntiles; ++t) {
-      const int st = t % nst;
-      const int round = t / nst;
-      if (ONLINE && not_needed(t)) break;
-      const bool ragged = stage_keys(t, y);
-      if (t + 1 < ntiles) fetch_keys(t + 1, y);  // in flight while this stage fills
-      bool okw;
-      if (!ONLINE) {
-        okw = warp_wait(bar(bar_empty + st), (uint32_t)((round & 1) ^ 1), a.spin);
-      } else {
-        // lane 0 waits for the stage or for a stop that makes it unneeded;
-        // after a free stage every lane acquires the barrier itself
-        int r = 0;
-        if (lane == 0) {
-          for (uint32_t it = 0; it < a.spin && r == 0; ++it) {
-            if (mbar_try_wait(bar(bar_empty + st), (uint32_t)((round & 1) ^ 1))) r = 1;
-            else if (not_needed(t)) r = 2;
-          }
-        }
-        r = __shfl_sync(0xffffffffu, r, 0);
-        if (r == 2) break;
-        okw = r == 1 && warp_wait(bar(bar_empty + st), (uint32_t)((round & 1) ^ 1), a.spin);
-      }
-      if (!okw) {
-        if (lane == 0) set_error(kErrTimeout);
-        break;
-      }
-      const uint32_t dst0 = ring + st * kTile2Bytes;
-      // 64 copies per lane; the key table is read four keys at a time.  A tile
-      // with a zero row (rare: an empty half or keys past N) takes the loop
-      // with per-row source sizes; the branch stays outside the unrolled loop
-      // so that each copy issues once.
-      if (!ragged) {
-#pragma unroll
-        for (int j4 = 0; j4 < 16; ++j4) {
-          int4 kk;
-          asm volatile("ld.shared.v4.s32 {%0, %1, %2, %3}, [%4];\n"
-                       : "=r"(kk.x), "=r"(kk.y), "=r"(kk.z), "=r"(kk.w)
-                       : "r"(ktab + 16u * (uint32_t)j4)
-                       : "memory");
-          const int key4[4] = {kk.x, kk.y, kk.z, kk.w};
-#pragma unroll
-          for (int m = 0; m < 4; ++m)
-            cp_async16(dst0 + dsw[m] + 256u * (uint32_t)(4 * j4 + m), src0 + (size_t)key4[m] * (kD * 2), 16u);
-        }
-      } else {
-#pragma unroll 4
-        for (int jj = 0; jj < 64; ++jj) {
-          const int key = keys[64 * sel + jj];
-          cp_async16(dst0 + dsw[jj & 3] + 256u * (uint32_t)jj, src0 + (size_t)(key < 0 ? 0 : key) * (kD * 2),
-                     key < 0 ? 0u : 16u);
-        }
-      }
-      cp_async_wait_all();
-      fence_proxy_async_smem();  // generic-proxy writes -> tensor-core reads
-      __syncwarp();
-      if (lane == 0) mbar_arrive(bar(bar_full + st));
-    }
-    // Q's TMA tiles may still be landing if the issuers gave up waiting for
-    // them: shared memory must not change after the CTA ends
-    if (is_k && lane == 0 && !mbar_wait_bounded(bar(kBarQFull), 0)) set_error(kErrTimeout);
+    attn_load_ring<ONLINE, QPERM>(a, &tmQ, sbase, sgen, warp, lane, b, bk, s, h0, row0, wk, ntiles, C0,
+                                  stop_word);
   } else if (warp == kMmaWarp || warp == kMmaWarp1) {
     // ------------------------------------------------------------------ MMA issuers
     // head i's products, in order: its P V of tile t-1 and half h precedes its
