@@ -111,9 +111,6 @@ cudaError_t set_kernel_attributes() {
     if (e == cudaSuccess)
       e = cudaFuncSetAttribute(k_truth_cols, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kTruthSmem);
     if (e == cudaSuccess)
-      e = cudaFuncSetAttribute(k_bucket_plan, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                               (int)(kMaxBuckets * kPlanRow * sizeof(uint32_t)));
-    if (e == cudaSuccess)
       e = cudaFuncSetAttribute(k_contig_plan, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                (int)(kContigMaxBlocks * sizeof(unsigned long long)));
     g_attr_err = e;
@@ -315,8 +312,7 @@ static void launch_plan_core(const s2o_config* cfg, const double* qbar, const ui
   k_seg_stats<<<(nwarps * 32 + 255) / 256, 256, 0, s>>>(w.part, w.segM, w.segZ, seg_stats, BH, S);
   ++t_launches;
   stage_mark(s, "k_seg_stats");
-  const size_t plan_smem = (size_t)min(kMaxBuckets, bucket_slots(num_cand(S - 1))) * kPlanRow * sizeof(uint32_t);
-  k_bucket_plan<<<BH * S, kBucketThreads, plan_smem, s>>>(scores, w.sorted, perm, w.slots, w.mode, w.range, w.keyB, w.valB,
+  k_bucket_plan<<<BH * S, kBucketThreads, 0, s>>>(scores, w.sorted, perm, w.slots, w.mode, w.range, w.keyB, w.valB,
                                                    w.segM, w.segZ, w.plen, cfg->tau, filtered, BH, S, T);
   ++t_launches;
   stage_mark(s, "k_bucket_plan");

@@ -10,17 +10,19 @@
 //                  buckets = runs of consecutive bins whose starting rank falls
 //                  in the same window of kBucketHalf ranks (a bucket holds at
 //                  most kBucketHalf + one bin <= kBucketCap elements); then a
-//                  stable multisplit of the segment into its buckets: (key,
-//                  index) pairs land at the bucket's rank range, in index order;
+//                  multisplit of the segment into its buckets: (key, index)
+//                  pairs land at the bucket's rank range, in no set order
+//                  (each warp reserves room with shared atomics, no block
+//                  barrier);
 //   k_bucket_sort  one CTA per group of kSortGroup consecutive bucket slots
 //                  (the empty ones, buckets a segment did not need, are
 //                  skipped); per bucket: loads its range into shared memory and
 //                  sorts it there: a counting sort into 4096 fine bins linear
 //                  in the score, then each fine bin (a few elements) by
-//                  (key, index); a bucket with a crowded fine bin is sorted by
-//                  a stable LSD radix sort over the bucket-relative key
-//                  instead; writes perm and the sorted scores at the bucket's
-//                  global rank;
+//                  (key, index); a bucket with a crowded fine bin, or with a
+//                  single key, is sorted by a stable LSD radix sort over the
+//                  bucket-relative index and then key instead; writes perm and
+//                  the sorted scores at the bucket's global rank;
 //   k_mass_stop    block masses of the sorted scores and the stop point C(s).
 // Filtered form (the planner's `filtered` flag): a candidate of pooled mass
 // exp(s - M)/Z below tau/Bk cannot lift a block to tau, so a block made only
@@ -48,11 +50,6 @@ constexpr int kBucketThreads = 1024;          // planner CTA
 constexpr int kSorterThreads = 512;           // bucket-sorter CTA (three per SM)
 constexpr int kSorterWarps = kSorterThreads / 32;
 constexpr int kMaxBuckets = 256;              // bucket ids per segment (N <= 2^19)
-constexpr int kPlanWarps = kBucketThreads / 32;
-constexpr int kPlanRounds = 4;                // elements per planner thread and multisplit step
-constexpr int kPlanRow = kPlanRounds * kPlanWarps + 4;  // words per bucket row of the planner's counts (16-byte rows, padded)
-static_assert(kPlanRounds * kPlanWarps == 128, "a bucket's counts are scanned by one warp, 4 per lane");
-static_assert(kPlanRounds == 4, "count rows are cleared as (bucket, round) = (q / 4, q % 4)");
 
 enum SegMode : int { kModeDone = 0, kModeBuckets = 1, kModeFallback = 2 };
 
@@ -118,9 +115,6 @@ __global__ void __launch_bounds__(kBucketThreads, 2) k_bucket_plan(const float* 
   __shared__ float red[64];
   __shared__ int flag;
   __shared__ uint8_t bin2bkt[kNumBins];  // bucket id of each bin (< kMaxBuckets = 256)
-  // [bucket][round * 32 + warp] counts, then ranks: rows of kPlanRow words
-  // (dynamic shared memory, one row per bucket id in use)
-  extern __shared__ uint32_t wcnt[];
   __shared__ int cursor[kMaxBuckets];
   __shared__ int bin_cut;  // first bin left out of the order (filtered form)
   const int q = blockIdx.x;
@@ -254,8 +248,10 @@ __global__ void __launch_bounds__(kBucketThreads, 2) k_bucket_plan(const float* 
 #pragma unroll
   for (int e = 0; e < 2; ++e)
     if (end_id[e] >= 0) myslot[end_id[e]].count = end_rank[e] - myslot[end_id[e]].base;
-  // stable multisplit into the buckets, 4096 elements per step in index order
-  // (two block barriers per step)
+  // multisplit into the buckets: each warp reserves room for its elements
+  // with one shared atomic per bucket id it holds, with no block barrier;
+  // the order inside a bucket is whatever the atomics give (the bucket
+  // sorter orders every bucket by (key, index))
   bin2bkt[2 * tid] = (uint8_t)(st0 / kBucketHalf);
   bin2bkt[2 * tid + 1] = (uint8_t)(st1 / kBucketHalf);
   __syncthreads();
@@ -270,61 +266,28 @@ __global__ void __launch_bounds__(kBucketThreads, 2) k_bucket_plan(const float* 
   const uint32_t lt_mask = (1u << lane) - 1u;
   uint32_t* skey = stage_key + base;
   uint32_t* sval = stage_val + base;
-  // bucket ids in use: those of the bins below bin_cut
-  const int nbk = bcut > 0 ? (int)bin2bkt[bcut - 1] + 1 : 0;
-  if (nbk == 0) {
+  if (bcut == 0) {
     if (tid == 0) mode[(size_t)bk * S + s] = kModeBuckets;
     return;
   }
-  // a step takes 4 rounds of 1024 elements: element i = t0 + 1024 k + tid, so
-  // index order is (round, warp, lane) and each bucket's row of 128 (round,
-  // warp) counts is scanned in that order
-  for (int t0 = 0; t0 < n; t0 += kPlanRounds * kBucketThreads) {
-    float x[kPlanRounds];
-    uint32_t d[kPlanRounds], rank[kPlanRounds];
-    bool valid[kPlanRounds];
-    __syncwarp();
-    for (int q = lane; q < kPlanRounds * nbk; q += 32) wcnt[(q >> 2) * kPlanRow + (q & 3) * kPlanWarps + warp] = 0;
-    __syncwarp();
-#pragma unroll
-    for (int k = 0; k < kPlanRounds; ++k) {
-      const int i = t0 + k * kBucketThreads + tid;
-      x[k] = i < n ? sc[i] : 0.f;
-      const int bin = score_bin(x[k], hi, scale);
-      valid[k] = i < n && bin < bcut;
-      d[k] = valid[k] ? bin2bkt[bin] : 0u;
-      // lanes holding the same bucket id (the lanes left out share one value:
-      // a match costs more the more distinct values a warp holds)
-      const uint32_t peers = __match_any_sync(0xffffffffu, valid[k] ? d[k] : 0xFFFFFFFFu);
-      rank[k] = __popc(peers & lt_mask);
-      if (valid[k] && (__ffs(peers) - 1) == lane) wcnt[d[k] * kPlanRow + k * kPlanWarps + warp] = __popc(peers);
-    }
-    __syncthreads();
-    // per bucket, one warp scans its 128 counts (4 per lane): they become
-    // absolute ranks and the bucket's cursor advances
-    for (int db = warp; db < nbk; db += kPlanWarps) {
-      uint4 v = *reinterpret_cast<const uint4*>(wcnt + db * kPlanRow + 4 * lane);
-      const uint32_t tot = v.x + v.y + v.z + v.w;
-      uint32_t incl = tot;
-#pragma unroll
-      for (int o = 1; o < 32; o <<= 1) {
-        const uint32_t y = __shfl_up_sync(0xffffffffu, incl, o);
-        if (lane >= o) incl += y;
-      }
-      const uint32_t cur = (uint32_t)cursor[db];
-      const uint32_t b0 = cur + incl - tot;
-      *reinterpret_cast<uint4*>(wcnt + db * kPlanRow + 4 * lane) =
-          make_uint4(b0, b0 + v.x, b0 + v.x + v.y, b0 + v.x + v.y + v.z);
-      if (lane == 31) cursor[db] = (int)(cur + incl);
-    }
-    __syncthreads();
-#pragma unroll
-    for (int k = 0; k < kPlanRounds; ++k) {
-      if (valid[k]) {
-        const uint32_t pos = wcnt[d[k] * kPlanRow + k * kPlanWarps + warp] + rank[k];
-        skey[pos] = desc_key(x[k]);
-        sval[pos] = (uint32_t)(t0 + k * kBucketThreads + tid);
-      }
+  for (int t0 = 0; t0 < n; t0 += kBucketThreads) {
+    const int i = t0 + tid;
+    const float x = i < n ? sc[i] : 0.f;
+    const int bin = score_bin(x, hi, scale);
+    const bool valid = i < n && bin < bcut;
+    if (!__any_sync(0xffffffffu, valid)) continue;
+    // lanes holding the same bucket id (the lanes left out share one value:
+    // a match costs more the more distinct values a warp holds)
+    const uint32_t dg = valid ? (uint32_t)bin2bkt[bin] : 0xFFFFFFFFu;
+    const uint32_t peers = __match_any_sync(0xffffffffu, dg);
+    const int leader = __ffs(peers) - 1;
+    uint32_t at = 0;
+    if (valid && lane == leader) at = (uint32_t)atomicAdd(&cursor[dg], __popc(peers));
+    at = __shfl_sync(0xffffffffu, at, leader);
+    if (valid) {
+      const uint32_t pos = at + __popc(peers & lt_mask);
+      skey[pos] = desc_key(x);
+      sval[pos] = (uint32_t)i;
     }
   }
   if (tid == 0) mode[(size_t)bk * S + s] = kModeBuckets;
@@ -353,7 +316,7 @@ struct BucketSmem {
   uint32_t cnt[kSorterWarps][256];  // radix digit counts, or the kFine fine-bin counters
   uint32_t dbase[256];
   int wtot[33];
-  uint32_t kmin, kmax;
+  uint32_t kmin, kmax, vmin, vmax;
   int big;
 };
 constexpr size_t kBucketSmem = sizeof(BucketSmem);
@@ -366,9 +329,9 @@ __device__ __forceinline__ void sort_bucket(const BucketSlot& slot, BucketSmem& 
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const size_t base = (size_t)slot.bk * T + cand_offset(slot.s) + slot.base;
   const int m = slot.count;
-  if (tid == 0) { sm.kmin = 0xFFFFFFFFu; sm.kmax = 0u; }
+  if (tid == 0) { sm.kmin = 0xFFFFFFFFu; sm.kmax = 0u; sm.vmin = 0xFFFFFFFFu; sm.vmax = 0u; }
 
-  // the bucket's pairs, already in index order at its rank range
+  // the bucket's pairs at its rank range, in no particular order
   uint32_t rk[kSortPer], rv[kSortPer];
   uint32_t kmin = 0xFFFFFFFFu, kmax = 0u;
 #pragma unroll
@@ -394,23 +357,11 @@ __device__ __forceinline__ void sort_bucket(const BucketSlot& slot, BucketSmem& 
   const uint32_t k0 = sm.kmin;
   const uint32_t span = sm.kmax - k0;
   const uint32_t lt_mask = (1u << lane) - 1u;
-  if (span == 0) {
-    // one key: the index order is the order
-#pragma unroll
-    for (int k = 0; k < kSortPer; ++k) {
-      const int i = tid + kSorterThreads * k;
-      if (i < m) {
-        sorted[base + i] = key_score(rk[k]);
-        perm[base + i] = kSink + (int32_t)rv[k];
-      }
-    }
-    return;
-  }
 
   // Fine counting sort: kFine bins linear in the score between the bucket's
   // extremes (monotone, ties share a bin), a scatter in any order, then each
   // bin sorted by (key, index) -- a total order, so the result is unique.
-  {
+  if (span > 0) {
     const float xhi = key_score(k0), xlo = key_score(sm.kmax);
     uint32_t* fcnt = &sm.cnt[0][0];  // kFine counters, then cursors
     const float fscale = (float)kFine / (xhi - xlo);
@@ -478,12 +429,44 @@ __device__ __forceinline__ void sort_bucket(const BucketSlot& slot, BucketSmem& 
     }
   }
 
-  // a crowded fine bin: stable LSD radix sort over the bucket-relative key,
-  // each pass scattering from the registers into the shared array
-  const int nbits = 32 - __clz(span);
-  const int passes = (nbits + 7) / 8;
+  // one key, or a crowded fine bin: stable LSD radix sort by (key, index):
+  // passes over the bucket-relative index first, then over the
+  // bucket-relative key, each pass scattering from the registers into the
+  // shared array
+  {
+    uint32_t vmin = 0xFFFFFFFFu, vmax = 0u;
+#pragma unroll
+    for (int k = 0; k < kSortPer; ++k) {
+      if (tid + kSorterThreads * k < m) {
+        vmin = min(vmin, rv[k]);
+        vmax = max(vmax, rv[k]);
+      }
+    }
+    vmin = __reduce_min_sync(0xffffffffu, vmin);
+    vmax = __reduce_max_sync(0xffffffffu, vmax);
+    if (lane == 0) {
+      atomicMin(&sm.vmin, vmin);
+      atomicMax(&sm.vmax, vmax);
+    }
+  }
+  __syncthreads();
+  const uint32_t v0 = sm.vmin;
+  const uint32_t vspan = sm.vmax - v0;
+  const int vpasses = (32 - __clz(vspan) + 7) / 8;
+  const int kpasses = span ? (32 - __clz(span) + 7) / 8 : 0;
+  const int passes = vpasses + kpasses;
+  if (passes == 0) {
+    // a single element
+    if (tid < m) {
+      sorted[base + tid] = key_score(rk[0]);
+      perm[base + tid] = kSink + (int32_t)rv[0];
+    }
+    return;
+  }
   for (int pass = 0; pass < passes; ++pass) {
-    const int shift = 8 * pass;
+    const bool on_val = pass < vpasses;
+    const int shift = 8 * (on_val ? pass : pass - vpasses);
+    const uint32_t org = on_val ? v0 : k0;
     if (pass) {
       // the previous pass's order, back into the registers
 #pragma unroll
@@ -500,7 +483,7 @@ __device__ __forceinline__ void sort_bucket(const BucketSlot& slot, BucketSmem& 
     __syncthreads();
 #pragma unroll
     for (int k = 0; k < kSortPer; ++k)
-      if (tid + kSorterThreads * k < m) atomicAdd(&sm.cnt[warp][((rk[k] - k0) >> shift) & 255u], 1u);
+      if (tid + kSorterThreads * k < m) atomicAdd(&sm.cnt[warp][(((on_val ? rv[k] : rk[k]) - org) >> shift) & 255u], 1u);
     __syncthreads();
     if (tid < 256) {
       uint32_t t = 0;
@@ -528,7 +511,7 @@ __device__ __forceinline__ void sort_bucket(const BucketSlot& slot, BucketSmem& 
 #pragma unroll
     for (int k = 0; k < kSortPer; ++k) {
       const bool valid = tid + kSorterThreads * k < m;
-      const uint32_t dg = ((rk[k] - k0) >> shift) & 255u;
+      const uint32_t dg = (((on_val ? rv[k] : rk[k]) - org) >> shift) & 255u;
 #pragma unroll
       for (int q = 0; q < 8; ++q) sm.cnt[warp][lane * 8 + q] = 0;
       __syncwarp();
