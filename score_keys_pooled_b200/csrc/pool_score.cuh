@@ -69,13 +69,15 @@ __global__ void __launch_bounds__(256) k_pool(const uint16_t* __restrict__ Q, do
 // the importance order is checked against.)
 // The products run on the fp64 tensor path (mma.sync m8n8k4): each warp owns
 // 16 segments x 64 keys (2 x 8 accumulator tiles), and its operand fragments
-// are reused across 256 multiply-adds per instruction, where scalar fp64 FMAs
-// were bound by shared-memory reads.  The d = 128 reduction runs in two
-// halves of 64 so that the key tile and the pooled queries (fp64, rows padded
-// to 68 doubles: the fragment pattern is then conflict-free) fit twice per
-// SM.  The sums are then staged in shared memory for the epilogue, where
-// thread (tk, ts) takes keys 2 tk + 32 a + {0, 1} (a < 4) x segments
-// ts + 16 b (b < 4).
+// are reused across 256 multiply-adds per instruction.  The key tile (bf16,
+// rows padded to 272 bytes) and the chunk's pooled queries (fp64, rows
+// padded to 132 doubles) arrive by cp.async; both fragment patterns are then
+// free of bank conflicts, and a key is widened to fp64 (exactly) as its
+// fragment is loaded.  The epilogue works on the accumulators in registers:
+// lane (fr, fc) of a warp holds segments m0 + 8 mt + fr and keys
+// n0 + 8 nt + 2 fc + {0, 1}; scores go out as pairs, and the per-(segment,
+// tile) (max, sum exp) is reduced over the lanes and the two warps that
+// share a segment.
 // Outputs:
 //   scores[bk][off(s) + j - 64] for candidate keys j of segment s
 //   part[bk][s][t] = (max over the tile's admissible keys,
@@ -83,17 +85,23 @@ __global__ void __launch_bounds__(256) k_pool(const uint16_t* __restrict__ Q, do
 // ---------------------------------------------------------------------------
 constexpr int kScoreKeys = 128;
 constexpr int kScoreSegs = 64;
-constexpr int kScoreHalf = 64;       // d per pass
-constexpr int kScoreStride = 68;     // padded rows of the fp64 operand tiles
-constexpr int kStageStride = kScoreKeys + 2;  // epilogue staging [64 segs][128 keys], padded
-constexpr size_t kScoreSmem = sizeof(double) * (kScoreKeys * kScoreStride + kScoreSegs * kScoreStride);
-static_assert(kScoreSegs * kStageStride <= kScoreKeys * kScoreStride + kScoreSegs * kScoreStride,
-              "staging must fit in the operand tiles");
+constexpr int kScoreKRow = 272;            // bytes per key row of the tile (256 + 16 padding)
+constexpr int kScoreQRow = 132;            // doubles per pooled-query row (128 + 4 padding)
+constexpr size_t kScoreKBytes = (size_t)kScoreKeys * kScoreKRow;
+constexpr size_t kScoreSmem = kScoreKBytes + sizeof(double) * kScoreSegs * kScoreQRow;
 
 __device__ __forceinline__ void dmma_8x8x4(double& c0, double& c1, double a, double b) {
   asm volatile("mma.sync.aligned.m8n8k4.row.col.f64.f64.f64.f64 {%0, %1}, {%2}, {%3}, {%0, %1};\n"
                : "+d"(c0), "+d"(c1)
                : "d"(a), "d"(b));
+}
+
+// (max, sum exp(v - max)) of two partial pairs
+__device__ __forceinline__ void merge_max_sum(float& m, float& z, float m2, float z2) {
+  const float mm = fmaxf(m, m2);
+  if (mm == -INFINITY) return;
+  z = (m == -INFINITY ? 0.f : z * exp_shifted(m, mm)) + (m2 == -INFINITY ? 0.f : z2 * exp_shifted(m2, mm));
+  m = mm;
 }
 
 __global__ void __launch_bounds__(256, 2) k_score(const uint16_t* __restrict__ K, const double* __restrict__ qbar,
@@ -114,113 +122,107 @@ __global__ void __launch_bounds__(256, 2) k_score(const uint16_t* __restrict__ K
   const int s_hi = min(S, s_lo + kScoreSegs);
   if (s_hi - 1 < t) return;
 
-  extern __shared__ double smd[];
-  double* Ks = smd;                                // [128 keys][64 d], rows of kScoreStride
-  double* Qs = smd + kScoreKeys * kScoreStride;    // [64 segs][64 d], rows of kScoreStride
+  extern __shared__ __align__(16) uint8_t sms[];
+  uint8_t* Ks = sms;                                            // [128 keys][272 B]
+  double* Qs = reinterpret_cast<double*>(sms + kScoreKBytes);   // [64 segs][132]
+  __shared__ float2 xw[2][kScoreSegs];                          // per-warp-half partials
   const int tid = threadIdx.x;
   const int lane = tid & 31, warp = tid >> 5;
   const uint16_t* Kb = K + (size_t)bk * N * kD;
   const double* qb = qbar + (size_t)bk * S * kD;
+
+  // the tile's keys (rows past N are zero: never admissible) and the chunk's
+  // pooled queries (segments past S are zero: never stored)
+  const uint32_t ks = smem_u32(Ks), qs = smem_u32(Qs);
+#pragma unroll
+  for (int q = 0; q < (kScoreKeys * 16) / 256; ++q) {
+    const int c = tid + 256 * q;               // 16-byte chunk c & 15 of key row c >> 4
+    const int key = c >> 4, j = t * kScoreKeys + key;
+    cp_async16(ks + key * kScoreKRow + (c & 15) * 16, Kb + (size_t)(j < N ? j : 0) * kD + (c & 15) * 8,
+               j < N ? 16u : 0u);
+  }
+#pragma unroll
+  for (int q = 0; q < (kScoreSegs * 64) / 256; ++q) {
+    const int c = tid + 256 * q;               // 16-byte chunk c & 63 of segment row c >> 6
+    const int seg = c >> 6, sg = s_lo + seg;
+    cp_async16(qs + seg * (kScoreQRow * 8) + (c & 63) * 16, qb + (size_t)(sg < S ? sg : 0) * kD + (c & 63) * 2,
+               sg < S ? 16u : 0u);
+  }
+  cp_async_wait_all();
+  __syncthreads();
+
   // this warp's block: segments m0 .. m0+15, keys n0 .. n0+63
   const int m0 = 16 * (warp & 3), n0 = 64 * (warp >> 2);
   const int fr = lane >> 2, fc = lane & 3;  // fragment row / column of this lane
-
   double c[2][8][2];
 #pragma unroll
   for (int mt = 0; mt < 2; ++mt)
 #pragma unroll
     for (int nt = 0; nt < 8; ++nt) c[mt][nt][0] = c[mt][nt][1] = 0.0;
-
-  for (int half = 0; half < 2; ++half) {
-    if (half) __syncthreads();
-    // key tile half -> fp64, row-major; keys >= N are zero (never admissible)
-    for (int q = tid; q < kScoreKeys * 8; q += 256) {
-      const int key = q >> 3, cch = q & 7;  // cch: 16-byte chunk 0..7 of this half
-      const int j = t * kScoreKeys + key;
-      uint4 w = make_uint4(0, 0, 0, 0);
-      if (j < N) w = *reinterpret_cast<const uint4*>(Kb + (size_t)j * kD + half * kScoreHalf + 8 * cch);
-      if (bf16x2_nonfinite(w.x) | bf16x2_nonfinite(w.y) | bf16x2_nonfinite(w.z) | bf16x2_nonfinite(w.w))
-        set_error(kErrNonFinite);
-      double* row = Ks + key * kScoreStride + 8 * cch;
-      row[0] = bf16_lo(w.x); row[1] = bf16_hi(w.x);
-      row[2] = bf16_lo(w.y); row[3] = bf16_hi(w.y);
-      row[4] = bf16_lo(w.z); row[5] = bf16_hi(w.z);
-      row[6] = bf16_lo(w.w); row[7] = bf16_hi(w.w);
-    }
-    for (int q = tid; q < kScoreSegs * kScoreHalf; q += 256) {
-      const int seg = q / kScoreHalf, dd = q % kScoreHalf;
-      const int s = s_lo + seg;
-      Qs[seg * kScoreStride + dd] = (s < S) ? qb[(size_t)s * kD + half * kScoreHalf + dd] : 0.0;
-    }
-    __syncthreads();
+  const double* qa = Qs + (m0 + fr) * kScoreQRow + fc;
+  const uint16_t* kbf = reinterpret_cast<const uint16_t*>(Ks + (n0 + fr) * kScoreKRow) + fc;
 #pragma unroll 2
-    for (int k0 = 0; k0 < kScoreHalf; k0 += 4) {
-      double a[2], bb[8];
+  for (int k0 = 0; k0 < kD; k0 += 4) {
+    double a[2], bb[8];
 #pragma unroll
-      for (int mt = 0; mt < 2; ++mt) a[mt] = Qs[(m0 + 8 * mt + fr) * kScoreStride + k0 + fc];
+    for (int mt = 0; mt < 2; ++mt) a[mt] = qa[8 * mt * kScoreQRow + k0];
 #pragma unroll
-      for (int nt = 0; nt < 8; ++nt) bb[nt] = Ks[(n0 + 8 * nt + fr) * kScoreStride + k0 + fc];
+    for (int nt = 0; nt < 8; ++nt)
+      bb[nt] = (double)__uint_as_float((uint32_t)kbf[8 * nt * (kScoreKRow / 2) + k0] << 16);
 #pragma unroll
-      for (int mt = 0; mt < 2; ++mt)
+    for (int mt = 0; mt < 2; ++mt)
 #pragma unroll
-        for (int nt = 0; nt < 8; ++nt) dmma_8x8x4(c[mt][nt][0], c[mt][nt][1], a[mt], bb[nt]);
-    }
+      for (int nt = 0; nt < 8; ++nt) dmma_8x8x4(c[mt][nt][0], c[mt][nt][1], a[mt], bb[nt]);
   }
-  // stage the sums: stg[seg][key] (accumulator element i of tile (mt, nt) is
-  // segment m0 + 8 mt + fr, key n0 + 8 nt + 2 fc + i)
-  __syncthreads();
-  double* stg = smd;
-#pragma unroll
-  for (int mt = 0; mt < 2; ++mt)
-#pragma unroll
-    for (int nt = 0; nt < 8; ++nt) {
-      double* dst = stg + (m0 + 8 * mt + fr) * kStageStride + n0 + 8 * nt + 2 * fc;
-      dst[0] = c[mt][nt][0];
-      dst[1] = c[mt][nt][1];
-    }
-  __syncthreads();
-  const int tk = tid & 15;
-  const int ts = tid >> 4;
-  double acc[8][4];
-#pragma unroll
-  for (int aa = 0; aa < 8; ++aa)
-#pragma unroll
-    for (int q = 0; q < 4; ++q) acc[aa][q] = stg[(ts + 16 * q) * kStageStride + 2 * tk + 32 * (aa >> 1) + (aa & 1)];
 
+  // epilogue from the accumulators
   float* sc_bk = scores + (size_t)bk * T;
   float2* part_bk = part + (size_t)bk * S * S;
   const double inv_sqrt_d = 0.08838834764831845;  // 1/sqrt(128), rounded to fp64
 #pragma unroll
-  for (int q = 0; q < 4; ++q) {
-    const int s = s_lo + ts + 16 * q;
+  for (int mt = 0; mt < 2; ++mt) {
+    const int seg = m0 + 8 * mt + fr;
+    const int s = s_lo + seg;
     const bool seg_ok = (s < s_hi) && (s >= t);
     const int cand_hi = s * kLq - kWin;  // candidates are [64, cand_hi)
-    float v[8];
+    float v[16];
     float mloc = -INFINITY;
 #pragma unroll
-    for (int a = 0; a < 8; ++a) {
-      const int j = t * kScoreKeys + 2 * tk + 32 * (a >> 1) + (a & 1);
-      v[a] = (float)(acc[a][q] * inv_sqrt_d);
-      const bool adm = seg_ok && (j < N);
-      if (adm) {
-        if (!isfinite(v[a])) set_error(kErrNonFinite);
-        mloc = fmaxf(mloc, v[a]);
-        if (j >= kSink && j < cand_hi) sc_bk[cand_offset(s) + (j - kSink)] = v[a];
-      } else {
-        v[a] = -INFINITY;
+    for (int nt = 0; nt < 8; ++nt) {
+      const int j = t * kScoreKeys + n0 + 8 * nt + 2 * fc;  // even; j + 1 shares j's class
+      const float v0 = (float)(c[mt][nt][0] * inv_sqrt_d), v1 = (float)(c[mt][nt][1] * inv_sqrt_d);
+      const bool adm0 = seg_ok && j < N, adm1 = seg_ok && j + 1 < N;
+      v[2 * nt] = adm0 ? v0 : -INFINITY;
+      v[2 * nt + 1] = adm1 ? v1 : -INFINITY;
+      if ((adm0 && !isfinite(v0)) || (adm1 && !isfinite(v1))) set_error(kErrNonFinite);
+      mloc = fmax3(mloc, v[2 * nt], v[2 * nt + 1]);
+      if (seg_ok && j >= kSink && j < cand_hi) {
+        float* dst = sc_bk + cand_offset(s) + (j - kSink);
+        if (adm1) *reinterpret_cast<float2*>(dst) = make_float2(v0, v1);
+        else if (adm0) dst[0] = v0;
       }
     }
-    // half-warp (16 lanes share ts) reductions: max, then sum exp(v - max)
-#pragma unroll
-    for (int o = 8; o >= 1; o >>= 1) mloc = fmaxf(mloc, __shfl_xor_sync(0xffffffffu, mloc, o));
+    // the four lanes of this fragment row hold the rest of the warp's 64 keys
+    mloc = fmaxf(mloc, __shfl_xor_sync(0xffffffffu, mloc, 1));
+    mloc = fmaxf(mloc, __shfl_xor_sync(0xffffffffu, mloc, 2));
     float z = 0.f;
     if (mloc > -INFINITY) {
 #pragma unroll
-      for (int a = 0; a < 8; ++a) z += (v[a] > -INFINITY) ? exp_shifted(v[a], mloc) : 0.f;
+      for (int k = 0; k < 16; ++k) z += (v[k] > -INFINITY) ? exp_shifted(v[k], mloc) : 0.f;
     }
-#pragma unroll
-    for (int o = 8; o >= 1; o >>= 1) z += __shfl_xor_sync(0xffffffffu, z, o);
-    if (tk == 0 && seg_ok) part_bk[(size_t)s * S + t] = make_float2(mloc, z);
+    z += __shfl_xor_sync(0xffffffffu, z, 1);
+    z += __shfl_xor_sync(0xffffffffu, z, 2);
+    if (fc == 0) xw[warp >> 2][seg] = make_float2(mloc, z);
+  }
+  __syncthreads();
+  // the two warps of a segment (keys 0-63 and 64-127 of the tile) merge
+  if (tid < kScoreSegs) {
+    const int s = s_lo + tid;
+    if (s < s_hi && s >= t) {
+      float m = xw[0][tid].x, z = xw[0][tid].y;
+      merge_max_sum(m, z, xw[1][tid].x, xw[1][tid].y);
+      part_bk[(size_t)s * S + t] = make_float2(m, z);
+    }
   }
 }
 

@@ -39,6 +39,13 @@ __device__ __forceinline__ float exp_shifted(float f, float M) {
   return expf(x) * (1.f + e);
 }
 
+// three-input max (sm_100)
+__device__ __forceinline__ float fmax3(float a, float b, float c) {
+  float d;
+  asm("max.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
+  return d;
+}
+
 // --- segment geometry (closed forms for the compiled constants) -------------
 
 // |Cand(s)| = max(0, 128 s - 192)
