@@ -107,6 +107,9 @@ cudaError_t set_kernel_attributes() {
       e = cudaFuncSetAttribute(k_sparse_attn2<false, true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                (int)kAttn2Smem);
     if (e == cudaSuccess)
+      e = cudaFuncSetAttribute(k_sparse_attn2<false, true, true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                               (int)kAttn2Smem);
+    if (e == cudaSuccess)
       e = cudaFuncSetAttribute(k_bucket_sort, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kBucketSmem);
     if (e == cudaSuccess)
       e = cudaFuncSetAttribute(k_truth_cols, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kTruthSmem);
@@ -563,8 +566,14 @@ s2o_status s2o_attention_qperm(const s2o_config* cfg, const uint16_t* Q, const u
   a.spin = kSpinLimit;
   CUtensorMap tmQ;
   if (!encode_rows_map(&tmQ, Q, (uint64_t)cfg->B * cfg->Hq * cfg->N, 128)) return S2O_ERR_CUDA;
-  const int64_t ncta = (int64_t)cfg->B * cfg->Hkv * a.S * (G / 2);
-  k_sparse_attn2<false, true><<<(unsigned)ncta, kAttn2Threads, kAttn2Smem, s>>>(a, tmQ);
+  if (G % 4 == 0) {
+    // every CTA: one sub-segment of a segment, four query heads
+    const int64_t ncta = (int64_t)cfg->B * cfg->Hkv * a.S * (G / 4) * 2;
+    k_sparse_attn2<false, true, true><<<(unsigned)ncta, kAttn2Threads, kAttn2Smem, s>>>(a, tmQ);
+  } else {
+    const int64_t ncta = (int64_t)cfg->B * cfg->Hkv * a.S * (G / 2);
+    k_sparse_attn2<false, true><<<(unsigned)ncta, kAttn2Threads, kAttn2Smem, s>>>(a, tmQ);
+  }
   ++t_launches;
   return launch_status();
 }

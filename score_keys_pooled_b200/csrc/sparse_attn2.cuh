@@ -60,7 +60,8 @@ constexpr uint32_t kOff2K = 2 * kTile2Bytes;         // K stages
 constexpr uint32_t kOff2V = kOff2K + kStagesK * kTile2Bytes;
 constexpr uint32_t kOff2Bar = kOff2V + kStagesV * kTile2Bytes;
 constexpr uint32_t kOff2Keys = kOff2Bar + 256;         // per loader warp: keys of its tile rows, by row parity
-constexpr uint32_t kAttn2SmemData = kOff2Keys + 2 * 512;
+constexpr uint32_t kOff2Rows = kOff2Keys + 2 * 512;     // regrouped Q_perm: the segment rows of one sub-segment
+constexpr uint32_t kAttn2SmemData = kOff2Rows + 4 * (kLq / 2 + 4);
 constexpr size_t kAttn2Smem = kAttn2SmemData + 1024;  // + alignment slack
 constexpr uint32_t kTmem2Cols = 512;
 
@@ -122,43 +123,6 @@ __device__ __forceinline__ uint64_t f2_add(uint64_t a, uint64_t b) {
 }
 __device__ __forceinline__ float f2_lo(uint64_t v) { return __uint_as_float((uint32_t)v); }
 __device__ __forceinline__ float f2_hi(uint64_t v) { return __uint_as_float((uint32_t)(v >> 32)); }
-__device__ __forceinline__ uint64_t f2_sub(uint64_t a, uint64_t b) {
-  uint64_t d;
-  asm("sub.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
-  return d;
-}
-
-// 2^x for a pair of fp32 values on the FMA pipe, leaving the special-function
-// unit (ex2.approx) to the other pairs of a row.  x = n + f with n = round(x)
-// and f in [-1/2, 1/2] (exact in fp32; n comes from adding 1.5 * 2^23, which
-// leaves round(x) in the low mantissa bits); 2^f is the degree-4 polynomial
-// of least maximum relative error on [-1/2, 1/2] (Remez exchange; the
-// coefficients and the generator are in exp2_poly.py), evaluated by Horner's
-// rule with packed fused multiply-adds; n is added to the exponent field.
-// Relative error below 3e-6 (the P values are then rounded to bf16).
-// Arguments are clamped to >= -125 so that the exponent stays normal.
-constexpr float kExp2C0 = 0.9999992847442627f;
-constexpr float kExp2C1 = 0.6931217908859253f;
-constexpr float kExp2C2 = 0.240247443318367f;
-constexpr float kExp2C3 = 0.05591785907745361f;
-constexpr float kExp2C4 = 0.009570102207362652f;
-__device__ __forceinline__ uint64_t exp2_poly_x2(uint64_t v) {
-  const float a = fmaxf(f2_lo(v), -125.f), b = fmaxf(f2_hi(v), -125.f);
-  const uint64_t x = f2_pack(a, b);
-  const uint64_t magic = f2_pack(12582912.f, 12582912.f);
-  const uint64_t t = f2_add(x, magic);
-  const uint64_t f = f2_sub(x, f2_sub(t, magic));
-  uint64_t p = f2_fma(f2_pack(kExp2C4, kExp2C4), f, f2_pack(kExp2C3, kExp2C3));
-  p = f2_fma(p, f, f2_pack(kExp2C2, kExp2C2));
-  p = f2_fma(p, f, f2_pack(kExp2C1, kExp2C1));
-  p = f2_fma(p, f, f2_pack(kExp2C0, kExp2C0));
-  const uint32_t lo = (uint32_t)p + ((uint32_t)t << 23);
-  const uint32_t hi = (uint32_t)(p >> 32) + ((uint32_t)(t >> 32) << 23);
-  return ((uint64_t)hi << 32) | lo;
-}
-// of every 8 pairs of a row's 64 scores in an unmasked chunk, this many take
-// exp2_poly_x2 and the rest ex2.approx
-constexpr int kPolyOf8 = 0;
 
 __device__ __forceinline__ void mbar_arrive(uint32_t bar) {
   asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];\n" ::"r"(bar) : "memory");
@@ -236,7 +200,7 @@ struct Attn2Args {
 // Q, warp kLoadWarp0 + 1 = V ring): for tile t of the key walk, gather its
 // 128 K (or V) rows by index into ring stage t % stages once the stage is
 // free, and arrive on the stage's full barrier after the copies landed.
-template <bool ONLINE, bool QPERM>
+template <bool ONLINE, bool QPERM, bool QTMA = true>
 __device__ __forceinline__ void attn_load_ring(const Attn2Args& a, const CUtensorMap* tmQ, uint32_t sbase,
                                                uint8_t* sgen, int warp, int lane, int b, int bk, int s, int h0,
                                                int row0, const Walk2& wk, int ntiles, int C0,
@@ -248,7 +212,7 @@ __device__ __forceinline__ void attn_load_ring(const Attn2Args& a, const CUtenso
   const int bar_empty = is_k ? kBarKEmpty : kBarVEmpty;
   const uint32_t ring = sbase + (is_k ? kOff2K : kOff2V);
   const uint16_t* kv = (is_k ? a.K : a.V) + (size_t)bk * a.N * kD;
-  if (is_k && lane == 0) {
+  if (QTMA && is_k && lane == 0) {
     mbar_expect_tx(bar(kBarQFull), 2 * kTile2Bytes);
 #pragma unroll
     for (int qi = 0; qi < 2; ++qi)
@@ -385,9 +349,14 @@ __device__ __forceinline__ void attn_load_ring(const Attn2Args& a, const CUtenso
   if (is_k && lane == 0 && !mbar_wait_bounded(bar(kBarQFull), 0)) set_error(kErrTimeout);
 }
 
-// ONLINE selects the run-time stop, QPERM the two query sub-segments; the
-// planned-stop kernel is compiled without any of their code
-template <bool ONLINE, bool QPERM = false>
+// ONLINE selects the run-time stop, QPERM the two query sub-segments (walked
+// together by every row, each masked for the other's rows); QGROUP (with
+// QPERM, group sizes divisible by 4) regroups the rows instead: a CTA takes
+// one sub-segment of a segment for four query heads, its two 128-row tiles
+// holding two heads' 64 rows of that sub-segment each, so every row of the
+// CTA walks the same kept set and nothing is masked.  The planned-stop
+// kernel is compiled without any of their code.
+template <bool ONLINE, bool QPERM = false, bool QGROUP = false>
 __global__ void __launch_bounds__(kAttn2Threads, 1)
     k_sparse_attn2(Attn2Args a, const __grid_constant__ CUtensorMap tmQ) {
   extern __shared__ uint8_t smem_raw[];
@@ -403,22 +372,27 @@ __global__ void __launch_bounds__(kAttn2Threads, 1)
   // head's K/V, which stays in L2), segments longest first, the pairs of a
   // segment adjacent (they gather the same rows)
   const int w = blockIdx.x;
-  const int per_bk = a.S * pairs;
+  // units of a segment: head pairs, or (QGROUP) head quads x sub-segments
+  const int units = QGROUP ? (G / 4) * 2 : pairs;
+  const int per_bk = a.S * units;
   const int bk = w / per_bk;
   const int rest = w % per_bk;
-  const int s = a.S - 1 - rest / pairs;
-  const int pair = rest % pairs;
+  const int s = a.S - 1 - rest / units;
+  const int unit = rest % units;
+  const int qsub = QGROUP ? (unit & 1) : 0;  // the sub-segment of a QGROUP CTA
   const int b = bk / a.Hkv, kvh = bk % a.Hkv;
-  const int h0 = kvh * G + 2 * pair;
+  // first query head of the CTA: tile i holds heads h0 + i (or, QGROUP,
+  // h0 + 2 i and h0 + 2 i + 1)
+  const int h0 = QGROUP ? kvh * G + 4 * (unit >> 1) : kvh * G + 2 * unit;
 
   const int cmax = (int)(num_cand(s) / kBk);
-  int C = ONLINE ? cmax : a.nblocks[(size_t)bk * a.S + s];
+  int C = ONLINE ? cmax : ((QGROUP && qsub) ? a.nblocks1 : a.nblocks)[(size_t)bk * a.S + s];
   if (C < 0 || C > cmax) {
     if (tid == 0) set_error(kErrBadPlan);
     C = C < 0 ? 0 : cmax;
   }
   const int C0 = C;  // blocks of the first list (Q_perm: sub-segment 0)
-  if (QPERM) {
+  if (QPERM && !QGROUP) {
     int C1 = a.nblocks1[(size_t)bk * a.S + s];
     if (C1 < 0 || C1 > cmax) {
       if (tid == 0) set_error(kErrBadPlan);
@@ -445,6 +419,39 @@ __global__ void __launch_bounds__(kAttn2Threads, 1)
     *reinterpret_cast<volatile int*>(sgen + kOff2Bar + 8 * kSlotStop) = kNoStop;
     fence_mbar_init();
   }
+  // QGROUP: the segment rows of sub-segment qsub, ascending (entries 0 ..
+  // n - 1), and their number n (entry kLq / 2); read by every role after the
+  // block barrier below
+  int32_t* rows_tab = reinterpret_cast<int32_t*>(sgen + kOff2Rows);
+  if (QGROUP && warp == 0) {
+    const uint32_t sub4 =
+        *reinterpret_cast<const uint32_t*>(a.rowsub + ((size_t)bk * a.S + s) * kLq + 4 * lane);
+    int f[4], cnt = 0;
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+      f[k] = (int)((sub4 >> (8 * k)) & 0xFFu) == qsub && row0 + 4 * lane + k < a.N;
+      cnt += f[k];
+    }
+    int incl = cnt;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int y = __shfl_up_sync(0xffffffffu, incl, o);
+      if (lane >= o) incl += y;
+    }
+    int pos = incl - cnt;
+#pragma unroll
+    for (int k = 0; k < 4; ++k)
+      if (f[k]) {
+        if (pos < kLq / 2) rows_tab[pos] = row0 + 4 * lane + k;
+        ++pos;
+      }
+    if (lane == 31) {
+      // a sub-segment holds at most half the rows (caller-supplied rowsub
+      // otherwise: flagged, extra rows dropped)
+      if (incl > kLq / 2) set_error(kErrBadPlan);
+      rows_tab[kLq / 2] = min(incl, kLq / 2);
+    }
+  }
   volatile int* stop_word = reinterpret_cast<volatile int*>(sgen + kOff2Bar + 8 * kSlotStop);
   if (warp == kMmaWarp) {
     tmem_alloc(smem_u32((const void*)tmem_slot), kTmem2Cols);
@@ -462,8 +469,35 @@ __global__ void __launch_bounds__(kAttn2Threads, 1)
     // layout the tensor core reads (one TMA gather4 per four rows issues far
     // slower than the load/store unit takes these copies).
     regs_decrease<kRegsOther>();
-    attn_load_ring<ONLINE, QPERM>(a, &tmQ, sbase, sgen, warp, lane, b, bk, s, h0, row0, wk, ntiles, C0,
-                                  stop_word);
+    if (QGROUP) {
+      if (warp == kLoadWarp0) {
+        // Q rows by index (lanes take 16-byte chunks of tile rows in turn),
+        // into the 128B-swizzled layout the 2D TMA writes otherwise; rows
+        // past the sub-segment's are zero
+        const int nq = rows_tab[kLq / 2];
+        for (int idx = lane; idx < 2 * kLq * 16; idx += 32) {
+          const int rr = idx >> 4, q16 = idx & 15;
+          const int ti = rr >> 7, r = rr & 127, k = r & 63;
+          const int head = h0 + 2 * ti + (r >> 6);
+          const int row = k < nq ? rows_tab[k] : -1;
+          const uint16_t* src = a.Q + ((size_t)(b * a.Hq + head) * a.N + (size_t)(row < 0 ? 0 : row)) * kD + 8 * q16;
+          const uint32_t dst = sbase + kOff2Q + ti * kTile2Bytes + (q16 >> 3) * (128 * 128) + r * 128 +
+                               (((q16 & 7) ^ (r & 7)) << 4);
+          cp_async16(dst, src, row < 0 ? 0u : 16u);
+        }
+        cp_async_wait_all();
+        fence_proxy_async_smem();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(bar(kBarQFull));
+      }
+      Attn2Args aq = a;
+      aq.perm = qsub ? a.perm1 : a.perm;
+      attn_load_ring<ONLINE, false, false>(aq, &tmQ, sbase, sgen, warp, lane, b, bk, s, h0, row0, wk, ntiles, C,
+                                           stop_word);
+    } else {
+      attn_load_ring<ONLINE, QPERM>(a, &tmQ, sbase, sgen, warp, lane, b, bk, s, h0, row0, wk, ntiles, C0,
+                                    stop_word);
+    }
   } else if (warp == kMmaWarp || warp == kMmaWarp1) {
     // ------------------------------------------------------------------ MMA issuers
     // head i's products, in order: its P V of tile t-1 and half h precedes its
@@ -536,10 +570,18 @@ __global__ void __launch_bounds__(kAttn2Threads, 1)
     // ------------------------------------------------------------------ softmax
     regs_increase<kRegsSoftmax>();
     const int qi = warp >> 2;               // head of the pair
-    const int r = tid & 127;                // row in the segment
-    const int row = row0 + r;
+    const int r = tid & 127;                // row of the tile
+    int row = row0 + r;                     // its row in the sequence
+    int head = h0 + qi;                     // and its query head
+    bool row_ok = row < a.N;
+    if (QGROUP) {
+      const int nq = rows_tab[kLq / 2];
+      head = h0 + 2 * qi + (r >> 6);
+      row_ok = (r & 63) < nq;
+      row = row_ok ? rows_tab[r & 63] : row0;
+    }
     const uint32_t lane_base = (uint32_t)((warp & 3) * 32) << 16;
-    const int my_sub = QPERM ? (int)a.rowsub[((size_t)bk * a.S + s) * kLq + r] : 0;
+    const int my_sub = (QPERM && !QGROUP) ? (int)a.rowsub[((size_t)bk * a.S + s) * kLq + r] : 0;
     const uint32_t tS = tmem + col_s(qi) + lane_base;
     const uint32_t tO = tmem + col_o(qi) + lane_base;
     const float sl2 = 1.4426950408889634f * 0.08838834764831845f;  // log2(e) / sqrt(d)
@@ -557,7 +599,7 @@ __global__ void __launch_bounds__(kAttn2Threads, 1)
       int j0;
       const int kind = walk2_block(wk, s, c, j0);
       int lim = kind == 3 ? -1 : (kind == 0 ? row - j0 : kBk);
-      if (QPERM && kind == 2 && (j0 >= C0 ? 1 : 0) != my_sub) lim = -1;  // the other sub-segment's block
+      if (QPERM && !QGROUP && kind == 2 && (j0 >= C0 ? 1 : 0) != my_sub) lim = -1;  // the other sub-segment's block
       if (!warp_wait(bar(kBarSFull + qi), (uint32_t)(c & 1), a.spin)) { ok = false; break; }
       tc_fence_after();
       float x[kBk];
@@ -614,15 +656,7 @@ __global__ void __launch_bounds__(kAttn2Threads, 1)
 #pragma unroll
         for (int k = 0; k < kBk; k += 2) {
           const uint64_t v = f2_fma(f2_pack(x[k], x[k + 1]), s2, nm2);
-          float p0, p1;
-          if (((k >> 1) & 7) < kPolyOf8) {
-            const uint64_t pp = exp2_poly_x2(v);
-            p0 = f2_lo(pp);
-            p1 = f2_hi(pp);
-          } else {
-            p0 = ex2_approx(f2_lo(v));
-            p1 = ex2_approx(f2_hi(v));
-          }
+          const float p0 = ex2_approx(f2_lo(v)), p1 = ex2_approx(f2_hi(v));
           rs2 = f2_add(rs2, f2_pack(p0, p1));
           x[k / 2] = __uint_as_float(pack_bf16x2(p0, p1));
         }
@@ -682,8 +716,8 @@ __global__ void __launch_bounds__(kAttn2Threads, 1)
     } else {
       tc_fence_after();
       const float inv = ell > 0.f ? 1.f / ell : 0.f;
-      const bool store = row < a.N;
-      const size_t orow = ((size_t)(b * a.Hq + h0 + qi) * a.N + (size_t)(store ? row : 0)) * kD;
+      const bool store = row_ok;
+      const size_t orow = ((size_t)(b * a.Hq + head) * a.N + (size_t)(store ? row : 0)) * kD;
 #pragma unroll
       for (int cc = 0; cc < 128; cc += 32) {
         float o[32];
