@@ -145,13 +145,17 @@ __global__ void __launch_bounds__(kBucketThreads, 2) k_bucket_plan(const float* 
   double cut = -INFINITY;
   if (filtered && tau > 0.0)
     cut = (double)segM[(size_t)bk * S + s] + log(tau * segZ[(size_t)bk * S + s] / (double)kBk) - 1e-3;
+  // candidate ranges start 256-byte aligned and hold a multiple of 64
+  // scores (n = 128 s - 192): every pass reads them as float4
+  const float4* sc4 = reinterpret_cast<const float4*>(sc);
+  const int n4 = n / 4;
   float lo = INFINITY, hi = -INFINITY;
   int nhi = 0;
-  for (int i = tid; i < n; i += kBucketThreads) {
-    const float x = sc[i];
-    lo = fminf(lo, x);
-    hi = fmaxf(hi, x);
-    nhi += (double)x >= cut;
+  for (int i = tid; i < n4; i += kBucketThreads) {
+    const float4 x = sc4[i];
+    lo = fminf(lo, fminf(fminf(x.x, x.y), fminf(x.z, x.w)));
+    hi = fmaxf(hi, fmaxf(fmaxf(x.x, x.y), fmaxf(x.z, x.w)));
+    nhi += ((double)x.x >= cut) + ((double)x.y >= cut) + ((double)x.z >= cut) + ((double)x.w >= cut);
   }
 #pragma unroll
   for (int o = 16; o >= 1; o >>= 1) {
@@ -190,7 +194,13 @@ __global__ void __launch_bounds__(kBucketThreads, 2) k_bucket_plan(const float* 
     return;
   }
   const float scale = (float)kNumBins / (hi - lo);
-  for (int i = tid; i < n; i += kBucketThreads) atomicAdd(&hist[score_bin(sc[i], hi, scale)], 1);
+  for (int i = tid; i < n4; i += kBucketThreads) {
+    const float4 x = sc4[i];
+    atomicAdd(&hist[score_bin(x.x, hi, scale)], 1);
+    atomicAdd(&hist[score_bin(x.y, hi, scale)], 1);
+    atomicAdd(&hist[score_bin(x.z, hi, scale)], 1);
+    atomicAdd(&hist[score_bin(x.w, hi, scale)], 1);
+  }
   __syncthreads();
   // exclusive scan over the bins: 2 per thread
   const int c0 = hist[2 * tid], c1 = hist[2 * tid + 1];
@@ -270,24 +280,29 @@ __global__ void __launch_bounds__(kBucketThreads, 2) k_bucket_plan(const float* 
     if (tid == 0) mode[(size_t)bk * S + s] = kModeBuckets;
     return;
   }
-  for (int t0 = 0; t0 < n; t0 += kBucketThreads) {
-    const int i = t0 + tid;
-    const float x = i < n ? sc[i] : 0.f;
-    const int bin = score_bin(x, hi, scale);
-    const bool valid = i < n && bin < bcut;
-    if (!__any_sync(0xffffffffu, valid)) continue;
-    // lanes holding the same bucket id (the lanes left out share one value:
-    // a match costs more the more distinct values a warp holds)
-    const uint32_t dg = valid ? (uint32_t)bin2bkt[bin] : 0xFFFFFFFFu;
-    const uint32_t peers = __match_any_sync(0xffffffffu, dg);
-    const int leader = __ffs(peers) - 1;
-    uint32_t at = 0;
-    if (valid && lane == leader) at = (uint32_t)atomicAdd(&cursor[dg], __popc(peers));
-    at = __shfl_sync(0xffffffffu, at, leader);
-    if (valid) {
-      const uint32_t pos = at + __popc(peers & lt_mask);
-      skey[pos] = desc_key(x);
-      sval[pos] = (uint32_t)i;
+  for (int t0 = 0; t0 < n4; t0 += kBucketThreads) {
+    const int i4 = t0 + tid;
+    const float4 x4 = i4 < n4 ? sc4[i4] : make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+      const int i = 4 * i4 + k;
+      const float x = k == 0 ? x4.x : k == 1 ? x4.y : k == 2 ? x4.z : x4.w;
+      const int bin = score_bin(x, hi, scale);
+      const bool valid = i4 < n4 && bin < bcut;
+      if (!__any_sync(0xffffffffu, valid)) continue;
+      // lanes holding the same bucket id (the lanes left out share one value:
+      // a match costs more the more distinct values a warp holds)
+      const uint32_t dg = valid ? (uint32_t)bin2bkt[bin] : 0xFFFFFFFFu;
+      const uint32_t peers = __match_any_sync(0xffffffffu, dg);
+      const int leader = __ffs(peers) - 1;
+      uint32_t at = 0;
+      if (valid && lane == leader) at = (uint32_t)atomicAdd(&cursor[dg], __popc(peers));
+      at = __shfl_sync(0xffffffffu, at, leader);
+      if (valid) {
+        const uint32_t pos = at + __popc(peers & lt_mask);
+        skey[pos] = desc_key(x);
+        sval[pos] = (uint32_t)i;
+      }
     }
   }
   if (tid == 0) mode[(size_t)bk * S + s] = kModeBuckets;
