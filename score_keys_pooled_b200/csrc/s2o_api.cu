@@ -321,7 +321,7 @@ static void launch_plan_core(const s2o_config* cfg, const double* qbar, const ui
   stage_mark(s, "k_bucket_plan");
   if (w.nslots > 0) {
     k_bucket_sort<<<(unsigned)((w.nslots + kSortGroup - 1) / kSortGroup), kSorterThreads, kBucketSmem, s>>>(
-        w.keyB, w.valB, w.slots, w.sorted, perm, w.nslots, T);
+        w.keyB, w.valB, w.slots, w.range, w.sorted, perm, w.nslots, S, T);
     ++t_launches;
     stage_mark(s, "k_bucket_sort");
   }

@@ -320,10 +320,6 @@ constexpr int kSortPer = kBucketCap / kSorterThreads;  // pairs per thread
 static_assert(kSortPer * kSorterThreads == kBucketCap, "a bucket fills the sorter's registers exactly");
 static_assert(kFine == kSorterWarps * 256, "fine counters reuse the radix count rows");
 
-__device__ __forceinline__ int fine_bin(float x, float hi, float scale) {
-  const int b = (int)((hi - x) * scale);
-  return min(max(b, 0), kFine - 1);
-}
 
 struct BucketSmem {
   uint32_t key[kBucketCap];
@@ -339,16 +335,14 @@ constexpr size_t kBucketSmem = sizeof(BucketSmem);
 // one bucket: sorted by (key, index) and written back at its global ranks
 __device__ __forceinline__ void sort_bucket(const BucketSlot& slot, BucketSmem& sm,
                                             const uint32_t* __restrict__ stage_key,
-                                            const uint32_t* __restrict__ stage_val, float* __restrict__ sorted,
-                                            int32_t* __restrict__ perm, int64_t T) {
+                                            const uint32_t* __restrict__ stage_val, const float2* __restrict__ range,
+                                            float* __restrict__ sorted, int32_t* __restrict__ perm, int S, int64_t T) {
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const size_t base = (size_t)slot.bk * T + cand_offset(slot.s) + slot.base;
   const int m = slot.count;
-  if (tid == 0) { sm.kmin = 0xFFFFFFFFu; sm.kmax = 0u; sm.vmin = 0xFFFFFFFFu; sm.vmax = 0u; }
 
   // the bucket's pairs at its rank range, in no particular order
   uint32_t rk[kSortPer], rv[kSortPer];
-  uint32_t kmin = 0xFFFFFFFFu, kmax = 0u;
 #pragma unroll
   for (int k = 0; k < kSortPer; ++k) {
     const int i = tid + kSorterThreads * k;
@@ -357,36 +351,32 @@ __device__ __forceinline__ void sort_bucket(const BucketSlot& slot, BucketSmem& 
     if (i < m) {
       rk[k] = stage_key[base + i];
       rv[k] = stage_val[base + i];
-      kmin = min(kmin, rk[k]);
-      kmax = max(kmax, rk[k]);
     }
   }
-  kmin = __reduce_min_sync(0xffffffffu, kmin);
-  kmax = __reduce_max_sync(0xffffffffu, kmax);
-  __syncthreads();
-  if (lane == 0) {
-    atomicMin(&sm.kmin, kmin);
-    atomicMax(&sm.kmax, kmax);
-  }
-  __syncthreads();
-  const uint32_t k0 = sm.kmin;
-  const uint32_t span = sm.kmax - k0;
   const uint32_t lt_mask = (1u << lane) - 1u;
 
-  // Fine counting sort: kFine bins linear in the score between the bucket's
-  // extremes (monotone, ties share a bin), a scatter in any order, then each
-  // bin sorted by (key, index) -- a total order, so the result is unique.
-  if (span > 0) {
-    const float xhi = key_score(k0), xlo = key_score(sm.kmax);
+  // Fine counting sort: kFine bins linear in the score over the bucket's
+  // share of the segment's bins (the planner's binning, so no pass over the
+  // bucket is needed to find its extremes; monotone, ties share a bin), a
+  // scatter in any order, then each bin sorted by (key, index) -- a total
+  // order, so the result is unique.
+  {
+    const float2 rg = range[(size_t)slot.bk * S + slot.s];
+    const float hi = rg.y, scale = (float)kNumBins / (rg.y - rg.x);  // the planner's bins
+    const float b0 = (float)slot.bin_lo;
+    const float ffac = (float)kFine / (float)(slot.bin_hi - slot.bin_lo);
+    auto fbin = [&](uint32_t key) {
+      const float u = ((hi - key_score(key)) * scale - b0) * ffac;
+      return min(max((int)u, 0), kFine - 1);
+    };
     uint32_t* fcnt = &sm.cnt[0][0];  // kFine counters, then cursors
-    const float fscale = (float)kFine / (xhi - xlo);
     constexpr int kPerT = kFine / kSorterThreads;  // counters per thread
     for (int k = tid; k < kFine; k += kSorterThreads) fcnt[k] = 0;
     if (tid == 0) sm.big = 0;
     __syncthreads();
 #pragma unroll
     for (int k = 0; k < kSortPer; ++k)
-      if (tid + kSorterThreads * k < m) atomicAdd(&fcnt[fine_bin(key_score(rk[k]), xhi, fscale)], 1u);
+      if (tid + kSorterThreads * k < m) atomicAdd(&fcnt[fbin(rk[k])], 1u);
     __syncthreads();
     int mine = 0, big = 0;
 #pragma unroll
@@ -410,7 +400,7 @@ __device__ __forceinline__ void sort_bucket(const BucketSlot& slot, BucketSmem& 
 #pragma unroll
       for (int k = 0; k < kSortPer; ++k) {
         if (tid + kSorterThreads * k < m) {
-          const uint32_t pos = atomicAdd(&fcnt[fine_bin(key_score(rk[k]), xhi, fscale)], 1u);
+          const uint32_t pos = atomicAdd(&fcnt[fbin(rk[k])], 1u);
           sm.key[pos] = rk[k];
           sm.val[pos] = rv[k];
         }
@@ -444,27 +434,37 @@ __device__ __forceinline__ void sort_bucket(const BucketSlot& slot, BucketSmem& 
     }
   }
 
-  // one key, or a crowded fine bin: stable LSD radix sort by (key, index):
-  // passes over the bucket-relative index first, then over the
-  // bucket-relative key, each pass scattering from the registers into the
-  // shared array
+  // a crowded fine bin (a cluster of near-equal or equal keys): stable LSD
+  // radix sort by (key, index), passes over the bucket-relative index first
+  // and then over the bucket-relative key, each pass scattering from the
+  // registers into the shared array
+  if (tid == 0) { sm.kmin = 0xFFFFFFFFu; sm.kmax = 0u; sm.vmin = 0xFFFFFFFFu; sm.vmax = 0u; }
+  __syncthreads();
   {
-    uint32_t vmin = 0xFFFFFFFFu, vmax = 0u;
+    uint32_t kmin = 0xFFFFFFFFu, kmax = 0u, vmin = 0xFFFFFFFFu, vmax = 0u;
 #pragma unroll
     for (int k = 0; k < kSortPer; ++k) {
       if (tid + kSorterThreads * k < m) {
+        kmin = min(kmin, rk[k]);
+        kmax = max(kmax, rk[k]);
         vmin = min(vmin, rv[k]);
         vmax = max(vmax, rv[k]);
       }
     }
+    kmin = __reduce_min_sync(0xffffffffu, kmin);
+    kmax = __reduce_max_sync(0xffffffffu, kmax);
     vmin = __reduce_min_sync(0xffffffffu, vmin);
     vmax = __reduce_max_sync(0xffffffffu, vmax);
     if (lane == 0) {
+      atomicMin(&sm.kmin, kmin);
+      atomicMax(&sm.kmax, kmax);
       atomicMin(&sm.vmin, vmin);
       atomicMax(&sm.vmax, vmax);
     }
   }
   __syncthreads();
+  const uint32_t k0 = sm.kmin;
+  const uint32_t span = sm.kmax - k0;
   const uint32_t v0 = sm.vmin;
   const uint32_t vspan = sm.vmax - v0;
   const int vpasses = (32 - __clz(vspan) + 7) / 8;
@@ -564,9 +564,10 @@ constexpr int kSortGroup = 8;
 __global__ void __launch_bounds__(kSorterThreads, 3) k_bucket_sort(const uint32_t* __restrict__ stage_key,
                                                                   const uint32_t* __restrict__ stage_val,
                                                                   const BucketSlot* __restrict__ slots,
+                                                                  const float2* __restrict__ range,
                                                                   float* __restrict__ sorted,
                                                                   int32_t* __restrict__ perm, int64_t nslots,
-                                                                  int64_t T) {
+                                                                  int S, int64_t T) {
   extern __shared__ uint8_t bsm_raw[];
   BucketSmem& sm = *reinterpret_cast<BucketSmem*>(bsm_raw);
   __shared__ BucketSlot group[kSortGroup];
@@ -581,7 +582,7 @@ __global__ void __launch_bounds__(kSorterThreads, 3) k_bucket_sort(const uint32_
   for (int gi = 0; gi < kSortGroup; ++gi) {
     const BucketSlot slot = group[gi];
     if (slot.count == 0) continue;
-    sort_bucket(slot, sm, stage_key, stage_val, sorted, perm, T);
+    sort_bucket(slot, sm, stage_key, stage_val, range, sorted, perm, S, T);
     __syncthreads();  // the next bucket reuses the shared arrays
   }
 }
