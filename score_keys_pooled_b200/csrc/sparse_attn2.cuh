@@ -520,7 +520,18 @@ __global__ void __launch_bounds__(kAttn2Threads, 1)
             if (!ok) break;
           }
           if (c > 0) {
-            ok = mbar_wait_bounded(bar(kBarSEmpty + i), (uint32_t)((c - 1) & 1), a.spin);
+            if (ONLINE) {
+              // S of chunk c - 1 read, or the tile stopped before it
+              int r = 0;
+              for (uint32_t it = 0; it < a.spin && r == 0; ++it) {
+                if (mbar_try_wait(bar(kBarSEmpty + i), (uint32_t)((c - 1) & 1))) r = 1;
+                else if (*stop_word != kNoStop && c - 1 > *stop_word) r = 2;
+              }
+              if (r == 2) break;
+              ok = r == 1;
+            } else {
+              ok = mbar_wait_bounded(bar(kBarSEmpty + i), (uint32_t)((c - 1) & 1), a.spin);
+            }
             if (!ok) break;
             tc_fence_after();
           }
@@ -541,7 +552,18 @@ __global__ void __launch_bounds__(kAttn2Threads, 1)
             ok = mbar_wait_bounded(bar(kBarVFull + tp % kStagesV), (uint32_t)((tp / kStagesV) & 1), a.spin);
             if (!ok) break;
           }
-          ok = mbar_wait_bounded(bar(kBarPFull + 2 * i + hp), (uint32_t)((cp >> 1) & 1), a.spin);
+          if (ONLINE) {
+            // P of chunk cp written, or the tile stopped before it
+            int r = 0;
+            for (uint32_t it = 0; it < a.spin && r == 0; ++it) {
+              if (mbar_try_wait(bar(kBarPFull + 2 * i + hp), (uint32_t)((cp >> 1) & 1))) r = 1;
+              else if (*stop_word != kNoStop && cp > *stop_word) r = 2;
+            }
+            if (r == 2) break;
+            ok = r == 1;
+          } else {
+            ok = mbar_wait_bounded(bar(kBarPFull + 2 * i + hp), (uint32_t)((cp >> 1) & 1), a.spin);
+          }
           if (!ok) break;
           tc_fence_after();
           const uint32_t sV = sbase + kOff2V + (tp % kStagesV) * kTile2Bytes;
@@ -552,12 +574,9 @@ __global__ void __launch_bounds__(kAttn2Threads, 1)
           }
           tc_commit(bar(kBarODone + 2 * i + hp));
           if (hp == 1) tc_commit(bar(kBarVEmpty + tp % kStagesV));
-          if (ONLINE && cp == *stop_word) {
-            // the tile stopped after chunk cp; Q K^T of chunk c (if any) is
-            // the last product in flight: wait for it before the CTA ends
-            if (c < nch) ok = mbar_wait_bounded(bar(kBarSFull + i), (uint32_t)(c & 1), a.spin);
-            break;
-          }
+          // the tile stopped after chunk cp: nothing more to multiply (products
+          // still in flight are drained below)
+          if (ONLINE && cp == *stop_word) break;
         }
       }
       if (!ok) set_error(kErrTimeout);
@@ -592,7 +611,6 @@ __global__ void __launch_bounds__(kAttn2Threads, 1)
     const float nrows_valid = 2.f * (float)min(kLq, a.N - row0);
     volatile float* gacc = reinterpret_cast<volatile float*>(sgen + kOff2Bar + 8 * kSlotGain);
     int c_online = cmax;
-    bool stop_now = false;
     int nch_done = nch;
     for (int c = 0; ok && c < nch; ++c) {
       // key k of the chunk is visible iff k <= lim
@@ -671,26 +689,36 @@ __global__ void __launch_bounds__(kAttn2Threads, 1)
           x[k / 2] = __uint_as_float(pack_bf16x2(p0, p1));
         }
       }
+      if (ONLINE && kind == 2 && j0 > 0) {
+        // the tile's decision on the previous candidate block, whose gains
+        // every warp posted one chunk ago (deciding here, not right after
+        // posting, keeps the warps from waiting on each other every chunk):
+        // below tau, the tile stopped after that block and this chunk does
+        // not count
+        const int qp = j0 - 1;
+        if (!warp_wait(bar(kBarGain), (uint32_t)(qp & 1), a.spin)) { ok = false; break; }
+        const float tot = gacc[qp % 3];
+        // the slot used for qp - 1: every warp read it before posting qp
+        if (warp == 0 && lane == 0) gacc[(qp + 2) % 3] = 0.f;
+        if (tot < a.tau * nrows_valid) {
+          c_online = qp + 1;
+          if ((warp & 3) == 0 && lane == 0) *stop_word = c - 1;  // the last chunk that counts
+          nch_done = c;
+          break;
+        }
+      }
       ell += rs;
       if (ONLINE && kind == 2) {
         // the block's gain for this row, relative to everything the row has
-        // processed (the block included; both sums share the reference m_run)
+        // processed (the block included; both sums share the reference
+        // m_run), summed over the tile's rows; decided at the next
+        // candidate block
         float gsum = row < a.N ? rs / ell : 0.f;
 #pragma unroll
         for (int o = 16; o >= 1; o >>= 1) gsum += __shfl_xor_sync(0xffffffffu, gsum, o);
-        const int q = j0;  // candidate block index
         if (lane == 0) {
-          atomicAdd(const_cast<float*>(gacc + q % 3), gsum);
+          atomicAdd(const_cast<float*>(gacc + j0 % 3), gsum);
           mbar_arrive(bar(kBarGain));
-        }
-        if (!warp_wait(bar(kBarGain), (uint32_t)(q & 1), a.spin)) { ok = false; break; }
-        const float tot = gacc[q % 3];
-        // the slot used at q - 1: every warp read it before arriving at q
-        if (warp == 0 && lane == 0) gacc[(q + 2) % 3] = 0.f;
-        stop_now = tot < a.tau * nrows_valid;
-        if (stop_now) {
-          c_online = q + 1;
-          if ((warp & 3) == 0 && lane == 0) *stop_word = c;  // read by the issuers after this chunk's P
         }
       }
       // P buffer c & 1 was last read by chunk c - 2's P V, which this head's
@@ -701,10 +729,6 @@ __global__ void __launch_bounds__(kAttn2Threads, 1)
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(bar(kBarPFull + 2 * qi + (c & 1)));
-      if (stop_now) {
-        nch_done = c + 1;
-        break;
-      }
     }
     if (ONLINE && tid == 0) {
       for (int k = 0; k < 2; ++k) a.cout[((size_t)b * a.Hq + h0 + k) * a.S + s] = c_online;
