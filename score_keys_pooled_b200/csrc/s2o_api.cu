@@ -625,63 +625,79 @@ s2o_status s2o_prefill_host(const s2o_config* cfg, const uint16_t* Q_host, const
 
   // One unit = one (b, kvh): its query heads, K and V rows are contiguous in
   // every buffer and its plan and attention depend on nothing else.  Units
-  // are copied in on one stream, planned and attended on the caller's stream
-  // and copied out on a third, so the copies of one unit overlap the kernels
-  // of the others.  The kernels see exactly the inputs of a whole-problem
-  // call, so the results are the same.
+  // are copied in on one stream (K and Q first: the plan needs only those),
+  // planned and attended on the caller's stream and copied out on a third,
+  // so the copies of one unit overlap the kernels of the others.  With an
+  // even group size a unit's attention runs one query-head pair at a time
+  // (a CTA computes one pair anyway), so the output of one pair goes out
+  // while the next is computed.  The kernels see exactly the inputs of a
+  // whole-problem call, so the results are the same.
   cudaStream_t s_in = nullptr, s_out = nullptr;
   if (!copy_streams(s_in, s_out)) return S2O_ERR_CUDA;
   const int G = cfg->Hq / cfg->Hkv;
   const int U = cfg->B * cfg->Hkv;
+  const int P = G % 2 == 0 ? G / 2 : 1;  // attention launches per unit
   s2o_config sub = *cfg;
   sub.B = 1;
   sub.Hq = G;
   sub.Hkv = 1;
-  const size_t qu = (size_t)G * cfg->N * kD, kvu = (size_t)cfg->N * kD;
+  s2o_config part = sub;
+  part.Hq = G / P;
+  const size_t qu = (size_t)G * cfg->N * kD, kvu = (size_t)cfg->N * kD, qp = qu / P;
   const size_t Tu = (size_t)ncand_total(cfg), Su = (size_t)nseg(cfg);
   const size_t oelt = out_dtype == S2O_OUT_F32 ? 4 : 2;
   size_t wsu = 0;
   s2o_plan_workspace_size(&sub, &wsu);
   cudaEvent_t ev0 = nullptr;
-  cudaEvent_t* ev = new cudaEvent_t[2 * (size_t)U]();
+  const size_t nev = 2 * (size_t)U + (size_t)U * P;  // K+Q in, V in, per-pair out
+  cudaEvent_t* ev = new cudaEvent_t[nev]();
   bool cuda_ok = cudaEventCreateWithFlags(&ev0, cudaEventDisableTiming) == cudaSuccess;
-  for (int u = 0; cuda_ok && u < 2 * U; ++u)
-    cuda_ok = cudaEventCreateWithFlags(&ev[u], cudaEventDisableTiming) == cudaSuccess;
+  for (size_t e = 0; cuda_ok && e < nev; ++e)
+    cuda_ok = cudaEventCreateWithFlags(&ev[e], cudaEventDisableTiming) == cudaSuccess;
+  cudaEvent_t* ev_kq = ev;
+  cudaEvent_t* ev_v = ev + U;
+  cudaEvent_t* ev_o = ev + 2 * U;
   // the copies start after the caller's earlier work on its stream (the
   // arena may still be in use there)
   cuda_ok = cuda_ok && cudaEventRecord(ev0, s) == cudaSuccess && cudaStreamWaitEvent(s_in, ev0, 0) == cudaSuccess &&
             cudaStreamWaitEvent(s_out, ev0, 0) == cudaSuccess;
   for (int u = 0; cuda_ok && u < U; ++u) {
-    cuda_ok = cudaMemcpyAsync(dQ + u * qu, Q_host + u * qu, qu * 2, cudaMemcpyHostToDevice, s_in) == cudaSuccess &&
-              cudaMemcpyAsync(dK + u * kvu, K_host + u * kvu, kvu * 2, cudaMemcpyHostToDevice, s_in) == cudaSuccess &&
+    cuda_ok = cudaMemcpyAsync(dK + u * kvu, K_host + u * kvu, kvu * 2, cudaMemcpyHostToDevice, s_in) == cudaSuccess &&
+              cudaMemcpyAsync(dQ + u * qu, Q_host + u * qu, qu * 2, cudaMemcpyHostToDevice, s_in) == cudaSuccess &&
+              cudaEventRecord(ev_kq[u], s_in) == cudaSuccess &&
               cudaMemcpyAsync(dV + u * kvu, V_host + u * kvu, kvu * 2, cudaMemcpyHostToDevice, s_in) == cudaSuccess &&
-              cudaEventRecord(ev[u], s_in) == cudaSuccess;
+              cudaEventRecord(ev_v[u], s_in) == cudaSuccess;
   }
   int32_t launches = 0;
   for (int u = 0; cuda_ok && st == S2O_OK && u < U; ++u) {
-    cuda_ok = cudaStreamWaitEvent(s, ev[u], 0) == cudaSuccess;
+    cuda_ok = cudaStreamWaitEvent(s, ev_kq[u], 0) == cudaSuccess;
     if (!cuda_ok) break;
     st = run_plan(&sub, dQ + u * qu, dK + u * kvu, dscores + u * Tu, dperm + u * Tu, dnb + u * Sp, nullptr, ws, wsu,
                   stream, 1);
     if (st != S2O_OK) break;
     launches += t_launches;
-    void* dOu = static_cast<uint8_t*>(dO) + u * qu * oelt;
-    st = s2o_attention(&sub, dQ + u * qu, dK + u * kvu, dV + u * kvu, dperm + u * Tu, dnb + u * Sp, dOu, out_dtype,
-                       stream);
-    if (st != S2O_OK) break;
-    launches += t_launches;
-    cuda_ok = cudaEventRecord(ev[U + u], s) == cudaSuccess && cudaStreamWaitEvent(s_out, ev[U + u], 0) == cudaSuccess &&
-              cudaMemcpyAsync(static_cast<uint8_t*>(O_host) + u * qu * oelt, dOu, qu * oelt, cudaMemcpyDeviceToHost,
-                              s_out) == cudaSuccess &&
-              (!nblocks_host || cudaMemcpyAsync(nblocks_host + u * Su, dnb + u * Sp, Su * 4, cudaMemcpyDeviceToHost,
-                                                s_out) == cudaSuccess);
+    cuda_ok = cudaStreamWaitEvent(s, ev_v[u], 0) == cudaSuccess;
+    for (int p = 0; cuda_ok && st == S2O_OK && p < P; ++p) {
+      uint8_t* dOp = static_cast<uint8_t*>(dO) + (u * qu + p * qp) * oelt;
+      st = s2o_attention(&part, dQ + u * qu + p * qp, dK + u * kvu, dV + u * kvu, dperm + u * Tu, dnb + u * Sp, dOp,
+                         out_dtype, stream);
+      if (st != S2O_OK) break;
+      launches += t_launches;
+      cudaEvent_t e = ev_o[(size_t)u * P + p];
+      cuda_ok = cudaEventRecord(e, s) == cudaSuccess && cudaStreamWaitEvent(s_out, e, 0) == cudaSuccess &&
+                cudaMemcpyAsync(static_cast<uint8_t*>(O_host) + (u * qu + p * qp) * oelt, dOp, qp * oelt,
+                                cudaMemcpyDeviceToHost, s_out) == cudaSuccess;
+    }
+    if (st != S2O_OK || !cuda_ok) break;
+    cuda_ok = !nblocks_host || cudaMemcpyAsync(nblocks_host + u * Su, dnb + u * Sp, Su * 4, cudaMemcpyDeviceToHost,
+                                               s_out) == cudaSuccess;
   }
   // every stream drains before the events go and the call returns
   const bool sync_ok = cudaStreamSynchronize(s_in) == cudaSuccess && cudaStreamSynchronize(s_out) == cudaSuccess &&
                        cudaStreamSynchronize(s) == cudaSuccess;
   if (ev0) cudaEventDestroy(ev0);
-  for (int u = 0; u < 2 * U; ++u)
-    if (ev[u]) cudaEventDestroy(ev[u]);
+  for (size_t e = 0; e < nev; ++e)
+    if (ev[e]) cudaEventDestroy(ev[e]);
   delete[] ev;
   t_launches = launches;
   if (st != S2O_OK) return st;

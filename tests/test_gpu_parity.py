@@ -654,6 +654,20 @@ def test_qperm_small_cases(B, Hq, Hkv, N, tau, planted, band):
     check_qperm(Q, K, V, cfg, qp, out, what=f"qperm small N={N}")
 
 
+@pytest.mark.parametrize("B,Hq,Hkv,N,tau", [(1, 16, 2, 1280, 3e-3), (2, 8, 1, 1000, 1e-2)])
+def test_qperm_two_head_quads_per_segment(B, Hq, Hkv, N, tau):
+    # group size 8: each segment's rows go to two CTAs per sub-segment (heads
+    # 0-3 and 4-7); the second case also has a ragged last segment whose
+    # second sub-segment is short
+    Q, K, V = synth.generate(B, Hq, Hkv, N, 128, planted=True, band=True, n_stripe=8, seed=N + 13)
+    cfg = s2o.make_config(B, Hq, Hkv, N, tau=tau)
+    q, k, v = dev(Q), dev(K), dev(V)
+    qp = s2o.plan_qperm(cfg, q, k)
+    out = s2o.attention_qperm(cfg, q, k, v, qp)
+    assert s2o.last_device_error() == 0
+    check_qperm(Q, K, V, cfg, qp, out, what=f"qperm G={Hq // Hkv} N={N}")
+
+
 def test_qperm_identical_rows_equal_the_plain_path():
     # every row of a segment equal in every head: both sub-segments pool to
     # the segment's query, so plans and output equal the plain method's
