@@ -326,9 +326,12 @@ s2o_status s2o_block_truth(const s2o_config* cfg, const uint16_t* Q, const uint1
  * the device arena, plans (s2o_plan_filtered: it returns no perm, and O and
  * C(s) equal those of s2o_plan), runs the attention and copies O back to
  * host O.  The work is split by (b, kvh), whose rows are contiguous in every
- * buffer: the copies in run on one library stream, plan and attention on
- * `stream`, the copies out on another library stream, so one group's copies
- * overlap the kernels of the others (results equal a single whole call).
+ * buffer: the copies in run on one library stream (K and Q of a group before
+ * its V, so its plan can start first), plan and attention on `stream`, the
+ * copies out on another library stream, so one group's copies overlap the
+ * kernels of the others; with an even group size the attention of a group
+ * runs one query-head pair at a time and each pair's O goes out while the
+ * next is computed (results equal a single whole call).
  * Host buffers should be page-locked for full copy speed.  The arena is
  * caller-allocated device memory of s2o_prefill_arena_size() bytes, 256-byte
  * aligned.  Synchronises the stream before returning and reports device

@@ -311,8 +311,9 @@ __global__ void __launch_bounds__(kBucketThreads, 2) k_bucket_plan(const float* 
 // ---------------------------------------------------------------------------
 // bucket sorter: one 512-thread CTA per group of slots, three CTAs per SM.
 // A bucket's pairs live in registers while they are counted and scattered
-// (pair k of thread tid is element tid + 512 k, so index order is (k, warp,
-// lane)); shared memory holds one key/value array, the scatter target.
+// (pair k of thread tid is element tid + 512 k of the bucket's range, the
+// order the radix passes keep stable); shared memory holds one key/value
+// array, the scatter target.
 // ---------------------------------------------------------------------------
 constexpr int kFine = 4096;     // fine bins of a bucket (= kSorterWarps * 256 counters)
 constexpr int kFineMax = 64;    // larger fine bins send the bucket to the radix path
@@ -522,7 +523,7 @@ __device__ __forceinline__ void sort_bucket(const BucketSlot& slot, BucketSmem& 
       for (int k = 0; k < 8; ++k) sm.dbase[lane * 8 + k] = excl + v[k];
     }
     __syncthreads();
-    // stable scatter, 512 pairs (one per thread) per step, in index order
+    // stable scatter, 512 pairs (one per thread) per step, in register order
 #pragma unroll
     for (int k = 0; k < kSortPer; ++k) {
       const bool valid = tid + kSorterThreads * k < m;
