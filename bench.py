@@ -188,6 +188,27 @@ def reduce_max_ms(ms: float, dist=None, device="cpu") -> float:
     return float(t.item())
 
 
+def kv_head_slice(Hkv: int, world: int, rank: int) -> tuple[int, int]:
+    """KV heads [k0, k1) of one rank when a single problem is sharded by KV
+    head: each rank plans and attends its KV heads and their groups' query
+    heads alone (a KV group's plan and attention depend on nothing else, so
+    no data crosses ranks).  Contiguous shares; the first Hkv % world ranks
+    take one head more."""
+    if not 1 <= world <= Hkv or not 0 <= rank < world:
+        raise ValueError("KV-head sharding needs 1 <= world <= Hkv")
+    base, extra = divmod(Hkv, world)
+    k0 = rank * base + min(rank, extra)
+    return k0, k0 + base + (1 if rank < extra else 0)
+
+
+def shard_inputs(Q, K, V, world: int, rank: int):
+    """This rank's Q, K, V (numpy bf16 bits) under kv_head_slice."""
+    G = Q.shape[1] // K.shape[1]
+    k0, k1 = kv_head_slice(K.shape[1], world, rank)
+    c = np.ascontiguousarray
+    return c(Q[:, k0 * G:k1 * G]), c(K[:, k0:k1]), c(V[:, k0:k1])
+
+
 def whole_job_tflops(world: int, flops_per_rank: float, ms: float) -> float:
     """Every rank solves its own problem: the job's throughput is all ranks'
     work over the slowest rank's time."""
@@ -361,10 +382,12 @@ def cpu_baseline_entry(Qn, Kn, Vn, tau):
             "value_all_cores": vall, "all_cores_processes": procs, "all_cores_sample": sample_all}
 
 
-def bench_config(w, world: int, plan: str) -> dict:
-    """The workload description both arms print."""
+def bench_config(w, world: int, plan: str, shard: bool = False) -> dict:
+    """The workload description both arms print (Hq, Hkv: one rank's share
+    when the problem is sharded by KV head)."""
     return {"workload": w.name, "B": w.B, "Hq": w.Hq, "Hkv": w.Hkv, "N": w.N, "d": w.d, "tau": w.tau,
-            "global_batch": w.B * world, "seq_len": w.N, "parallelism": f"independent x{world}",
+            "global_batch": w.B if shard else w.B * world, "seq_len": w.N,
+            "parallelism": f"kv-head shards x{world}" if shard else f"independent x{world}",
             "l2": "inputs larger than L2 (Q alone is 1 GiB)" if w.N >= 131072 else "inputs per step exceed L2",
             "plan": plan}
 
@@ -535,6 +558,10 @@ def main():
     ap.add_argument("--plan", default="filtered", choices=["full", "filtered"],
                     help="s2o_plan (every segment fully ordered) or s2o_plan_filtered (only the prefix the "
                          "stop rule can reach; same kept sets and output)")
+    ap.add_argument("--shard", default="none", choices=["none", "heads"],
+                    help="none: every rank solves its own problem (weak scaling); heads: the ranks share one "
+                         "problem, each taking a contiguous share of its KV heads (strong scaling, no data "
+                         "exchange)")
     ap.add_argument("--tau", type=float, default=None,
                     help="override the workload's tau (e.g. to profile a small workload at the headline's density)")
     ap.add_argument("--report", default=None, choices=["configs", "sweep"],
@@ -560,8 +587,15 @@ def main():
         reference_arm(args, w, world, rank)
         return
 
-    # each rank solves an independent problem (its own seed): weak scaling
-    Qn, Kn, Vn = synth.generate_workload(w, seed=rank)
+    # each rank solves an independent problem (its own seed): weak scaling;
+    # or (--shard heads) its share of the KV heads of one problem: strong
+    shard = args.shard == "heads" and world > 1
+    dense_full = dense_flops(w.B, w.Hq, w.N, w.d)
+    Qn, Kn, Vn = synth.generate_workload(w, seed=0 if shard else rank)
+    if shard:
+        import dataclasses
+        Qn, Kn, Vn = shard_inputs(Qn, Kn, Vn, world, rank)
+        w = dataclasses.replace(w, Hq=Qn.shape[1], Hkv=Kn.shape[1])
 
     # the CPU baseline forks its worker pool, so it runs before any CUDA call
     cpu = None
@@ -643,7 +677,9 @@ def main():
     dense = dense_flops(w.B, w.Hq, w.N, w.d)
     density = pairs / (w.B * w.Hq * w.N * (w.N + 1) / 2.0)
     ms_step = total_ms / args.steps
-    value = whole_job_tflops(world, dense, ms_step)
+    job_flops = dense_full if shard else world * dense
+    job_tflops = lambda ms: job_flops / (ms * 1e-3) / 1e12
+    value = job_tflops(ms_step)
 
     # roofline of the dominant kernel (sparse attention): algorithmic flops
     # = 4 d x kept (row, key) pairs, per launch, over its CUDA-event time
@@ -699,7 +735,7 @@ def main():
         op = float(np.mean([e[0].elapsed_time(e[1]) for e in evo]))
         oa = float(np.mean([e[1].elapsed_time(e[2]) for e in evo]))
         co = cout.cpu().numpy().reshape(w.B, w.Hq, -1)
-        online = {"plan_ms": op, "attention_ms": oa, "value": whole_job_tflops(world, dense, op + oa),
+        online = {"plan_ms": op, "attention_ms": oa, "value": job_tflops(op + oa),
                   "kept_pair_fraction": kept_pairs(co, w.N, 1) / (w.B * w.Hq * w.N * (w.N + 1) / 2.0),
                   "rule": "stop after the first candidate block whose mean relative gain over the tile is < tau"}
         s2o.plan(cfg, Q, K, bufs, filtered=filtered)
@@ -724,7 +760,7 @@ def main():
         qat = float(np.mean([e[1].elapsed_time(e[2]) for e in evq]))
         nb2 = qp["nblocks"].cpu().numpy().reshape(2, w.B, w.Hkv, -1)
         rsub = qp["rowsub"].cpu().numpy().reshape(w.B, w.Hkv, -1, 128)
-        qperm = {"plan_ms": qpl, "attention_ms": qat, "value": whole_job_tflops(world, dense, qpl + qat),
+        qperm = {"plan_ms": qpl, "attention_ms": qat, "value": job_tflops(qpl + qat),
                  "kept_pair_fraction": kept_pairs_qperm(nb2, rsub, w.N, w.Hq // w.Hkv) /
                  (w.B * w.Hq * w.N * (w.N + 1) / 2.0)}
         del qp
@@ -779,22 +815,23 @@ def main():
         e2e_ms = reduce_max_ms(e2e_ms, dist, dev)
         h2d = (Qn.nbytes + Kn.nbytes + Vn.nbytes)
         d2h = Qn.nbytes + nb.size * 4
-        e2e = {"value": whole_job_tflops(world, dense, e2e_ms), "unit": "TFLOP/s", "ms_per_step": e2e_ms,
+        e2e = {"value": job_tflops(e2e_ms), "unit": "TFLOP/s", "ms_per_step": e2e_ms,
                "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h)}
         del arena
 
     if rank == 0:
         line = {
             "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps,
-            "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak",
+            "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True,
+            "scaling": "strong" if shard else "weak",
             "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
-            "config": bench_config(w, world, args.plan),
+            "config": bench_config(w, world, args.plan, shard),
             "plan_ms": float(np.mean(plan_ms)), "attention_ms": attn_mean,
             "plan_other": {"kind": "full" if filtered else "filtered", "ms": other_ms},
             "online_stop": online,
             "ranking": ranking,
             "qperm": qperm,
-            "attention_only_tflops": whole_job_tflops(world, dense, attn_mean),
+            "attention_only_tflops": job_tflops(attn_mean),
             "kept_pair_fraction": density, "accuracy": accuracy,
             "roofline": roofline, "plan_roofline": plan_roofline,
             "cpu_baseline": cpu, "e2e": e2e, "gpu_launches": launches,

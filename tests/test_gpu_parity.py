@@ -150,6 +150,26 @@ def test_all_ties_bit_exact(tau):
         assert stats[0, 0, s, 0] == 0.0 and stats[0, 0, s, 1] == float(e)
 
 
+@pytest.mark.parametrize("world", [2, 3, 8])
+def test_kv_head_shards_reassemble_the_whole_problem(world):
+    """One problem sharded by KV head (bench.py --shard heads): every rank's
+    library call on its share, run here one after another on one GPU, gives
+    exactly the whole call's C(s) and output rows."""
+    import bench
+    B, Hq, Hkv, N, tau = 1, 32, 8, 2048, 3e-3
+    Q, K, V = synth.generate(B, Hq, Hkv, N, 128, planted=True, band=True, n_stripe=16, seed=23)
+    cfg, bufs, out = run_path(Q, K, V, tau)
+    G = Hq // Hkv
+    S = s2o.num_segments(cfg)
+    nb_all = bufs["nblocks"].view(B, Hkv, S)
+    for rank in range(world):
+        k0, k1 = bench.kv_head_slice(Hkv, world, rank)
+        q, k, v = bench.shard_inputs(Q, K, V, world, rank)
+        c_loc, b_loc, o_loc = run_path(q, k, v, tau)
+        assert torch.equal(b_loc["nblocks"].view(B, k1 - k0, S), nb_all[:, k0:k1])
+        assert torch.equal(o_loc, out[:, k0 * G:k1 * G])
+
+
 def test_nonfinite_input_is_reported():
     Q, K, V = synth.generate(1, 4, 1, 512, 128, planted=True, band=False, n_stripe=4, seed=9)
     K = K.copy()
