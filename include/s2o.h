@@ -284,9 +284,15 @@ s2o_status s2o_attention_online(const s2o_config* cfg, const uint16_t* Q, const 
  *   workspace  device scratch of s2o_plan_qperm_workspace_size() bytes,
  *            256-byte aligned
  * s2o_attention_qperm -- the sparse output with each row over its own
- * sub-segment's kept set; perm, nblocks, rowsub as produced above; other
- * arguments as s2o_attention.  Requires an even group size Hq/Hkv
- * (S2O_ERR_UNSUPPORTED_SHAPE otherwise).
+ * sub-segment's kept set; perm, nblocks, rowsub (16-byte aligned) as
+ * produced above; other arguments as s2o_attention.  Requires an even group
+ * size Hq/Hkv (S2O_ERR_UNSUPPORTED_SHAPE otherwise).  With Hq/Hkv divisible
+ * by 4 each CTA takes one sub-segment of a segment for four query heads, so
+ * a row walks only its own sub-segment's kept blocks; otherwise every row
+ * walks both sub-segments' kept blocks, masked for the other's rows.  A
+ * rowsub that puts more than 64 of a segment's rows in one sub-segment (not
+ * one s2o_plan_qperm writes) sets S2O_ERR_BAD_PLAN; the extra rows are then
+ * not computed.
  */
 s2o_status s2o_plan_qperm_workspace_size(const s2o_config* cfg, size_t* bytes);
 s2o_status s2o_plan_qperm(const s2o_config* cfg, const uint16_t* Q, const uint16_t* K, float* scores,

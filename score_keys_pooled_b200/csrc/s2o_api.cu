@@ -547,7 +547,8 @@ s2o_status s2o_attention_qperm(const s2o_config* cfg, const uint16_t* Q, const u
   if (st != S2O_OK) return st;
   if (!Q || !K || !V || !perm || !nblocks || !rowsub || !O) return S2O_ERR_INVALID_ARG;
   if (out_dtype != S2O_OUT_BF16 && out_dtype != S2O_OUT_F32) return S2O_ERR_INVALID_ARG;
-  if (!aligned16(Q) || !aligned16(K) || !aligned16(V) || !aligned16(O) || !aligned16(perm)) return S2O_ERR_INVALID_ARG;
+  if (!aligned16(Q) || !aligned16(K) || !aligned16(V) || !aligned16(O) || !aligned16(perm) || !aligned16(rowsub))
+    return S2O_ERR_INVALID_ARG;
   const int G = cfg->Hq / cfg->Hkv;
   if (G % 2 != 0 || (int64_t)cfg->B * cfg->Hq * cfg->N >= (int64_t)INT32_MAX) return S2O_ERR_UNSUPPORTED_SHAPE;
   if (set_kernel_attributes() != cudaSuccess) return S2O_ERR_CUDA;
