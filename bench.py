@@ -89,9 +89,12 @@ def kept_pairs_qperm(nblocks2: np.ndarray, rowsub: np.ndarray, N: int, G: int) -
 # exists.
 ATTN_TRAFFIC = {"llama_128k": 2.679e9, "llama_32k@0.004": 6.698e8}
 
-# fp64 multiply-add rate of this machine's B200s (DFMA and mma.sync m8n8k4 alike),
-# measured by a register-resident microbenchmark: 37 TFLOP/s = 18.5 T FMA/s
-FP64_FMA_PER_S = 18.5e12
+# int8 tensor-core rate relative to the measured bf16 rate: the nominal dense
+# ratio of B200 (4.5 POPS int8 / 2.25 PFLOP/s bf16)
+I8_OVER_BF16 = 2.0
+# digit products per (segment, admissible key) pair of the integer scorer:
+# 11 products of 128 int8 multiply-adds
+I8_MACS_PER_PAIR = 11 * 128
 
 
 def prefix_lengths(torch, cfg, bufs, filtered: bool, w):
@@ -120,9 +123,12 @@ def plan_kernel_roofline(s2o, torch, cfg, Q, K, bufs, filtered, w, peaks, peak_s
     """Median device time of each plan kernel over `reps` plans (events on the
     caller's stream between the kernels), and its compulsory HBM bytes:
       k_pool       read Q, write the fp64 pooled queries
-      k_score      read K and the pooled queries, write the candidate scores
-                   and the causal half of the (max, sumexp) partials; also its
-                   fp64 multiply-adds (128 per admissible key per segment)
+      k_kdig       read K, write its three 8-bit digit planes and row exponents
+      k_qdig       read the pooled queries, write their four digit planes
+      k_score8     read the key and query digits once, write the candidate
+                   scores and the causal half of the (max, sumexp) partials;
+                   also its int8 multiply-adds (11 x 128 per admissible key
+                   per segment) against the int8 tensor peak
       k_seg_stats  read the partials, write (M, Z)
       k_bucket_plan read every candidate score, write the staged (key, index)
                    pairs of the sorted prefix
@@ -134,16 +140,22 @@ def plan_kernel_roofline(s2o, torch, cfg, Q, K, bufs, filtered, w, peaks, peak_s
     T = B * Hkv * ((64 * (S - 2) ** 2) if S >= 2 else 0)
     L = prefix_lengths(torch, cfg, bufs, filtered, w)
     parts = B * Hkv * S * (S + 1) / 2 * 8
+    ntiles = (N + 31) // 32
+    kdig = B * Hkv * ntiles * (3 * 32 * 128 + 32 * 4)
+    qdig = B * Hkv * S * (4 * 128 + 4)
     bytes_of = {
         "k_pool": B * Hq * N * d * 2 + B * Hkv * S * d * 8,
-        "k_score": B * Hkv * N * d * 2 + B * Hkv * S * d * 8 + T * 4 + parts,
+        "k_kdig": B * Hkv * N * d * 2 + kdig,
+        "k_qdig": B * Hkv * S * d * 8 + qdig,
+        "k_score8": kdig + qdig + T * 4 + parts,
         "k_seg_stats": parts + B * Hkv * S * 16,
         "k_bucket_plan": T * 4 + L * 8,
         "k_bucket_sort": L * 8 + L * 8,
         "k_mass_stop": L * 4 + B * Hkv * S * 4,
     }
     # admissible keys of every segment: e(s) = min(N, 128 (s + 1))
-    dfma = B * Hkv * d * sum(min(N, 128 * (s + 1)) for s in range(S))
+    i8_macs = B * Hkv * I8_MACS_PER_PAIR * sum(min(N, 128 * (s + 1)) for s in range(S))
+    i8_peak = float(peaks["bf16_tflops"]) * 1e12 * I8_OVER_BF16 / 2  # multiply-adds per second
     s2o.stage_timing(True)
     try:
         runs = []
@@ -165,11 +177,10 @@ def plan_kernel_roofline(s2o, torch, cfg, Q, K, bufs, filtered, w, peaks, peak_s
             b = float(bytes_of[name])
             total_bytes += b
             ent.update(bytes=b, gbs=b / (ms * 1e-3) / 1e9, frac_hbm=b / (ms * 1e-3) / 1e9 / hbm)
-        if name == "k_score":
-            ent.update(fp64_fma=float(dfma), fp64_fma_per_s=dfma / (ms * 1e-3),
-                       frac_fp64=dfma / (ms * 1e-3) / FP64_FMA_PER_S,
-                       note="exact fp64 dot products (half-ulp fp32 scores): bound by the fp64 pipe, whose "
-                            "floor is above the HBM floor of its bytes")
+        if name == "k_score8":
+            ent.update(i8_macs=float(i8_macs), i8_tops=2 * i8_macs / (ms * 1e-3) / 1e12,
+                       frac_i8=i8_macs / (ms * 1e-3) / i8_peak,
+                       note="int8 peak = measured bf16 burst x 2 (nominal dense ratio)")
         out["kernels"][name] = ent
     out["total_ms"] = total_ms
     out["total_bytes"] = total_bytes

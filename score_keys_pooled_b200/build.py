@@ -15,7 +15,7 @@ ROOT = os.path.dirname(PKG)
 CSRC = os.path.join(PKG, "csrc")
 LIB = os.path.join(PKG, "libs2o.so")
 SOURCES = ["s2o_api.cu"]
-HEADERS = ["s2o_common.cuh", "pool_score.cuh", "seg_sort.cuh", "seg_sort2.cuh", "sparse_attn.cuh", "sparse_attn2.cuh", "block_truth.cuh", "qperm.cuh"]
+HEADERS = ["s2o_common.cuh", "pool_score.cuh", "score_i8.cuh", "seg_sort.cuh", "seg_sort2.cuh", "sparse_attn.cuh", "sparse_attn2.cuh", "block_truth.cuh", "qperm.cuh"]
 
 
 def nvcc() -> str:

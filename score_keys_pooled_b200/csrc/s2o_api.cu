@@ -8,6 +8,7 @@
 #include "s2o.h"
 #include "s2o_common.cuh"
 #include "pool_score.cuh"
+#include "score_i8.cuh"
 #include "seg_sort.cuh"
 #include "seg_sort2.cuh"
 #include "sparse_attn.cuh"
@@ -58,6 +59,10 @@ struct PlanWs {
   int* mode;
   int* plen;
   float2* range;
+  uint8_t* kd;      // key digits, per 32-key tile
+  int32_t* kexp;    // row exponent per key (tiles padded to 32 keys)
+  uint8_t* qd;      // pooled-query digits, per segment
+  int32_t* qexp;    // row exponent per segment
   int64_t nslots;
   size_t bytes;
 };
@@ -87,6 +92,11 @@ PlanWs plan_layout(const s2o_config* c, void* base) {
   w.mode = static_cast<int*>(take(BH * S * sizeof(int)));
   w.plen = static_cast<int*>(take(BH * S * sizeof(int)));
   w.range = static_cast<float2*>(take(BH * S * sizeof(float2)));
+  const size_t ntiles = ((size_t)c->N + kI8TileKeys - 1) / kI8TileKeys;
+  w.kd = static_cast<uint8_t*>(take(BH * ntiles * kI8TileBytes));
+  w.kexp = static_cast<int32_t*>(take(BH * ntiles * kI8TileKeys * sizeof(int32_t)));
+  w.qd = static_cast<uint8_t*>(take(BH * S * kI8QRowBytes));
+  w.qexp = static_cast<int32_t*>(take(BH * S * sizeof(int32_t)));
   w.bytes = off;
   return w;
 }
@@ -96,7 +106,7 @@ cudaError_t g_attr_err = cudaSuccess;
 
 cudaError_t set_kernel_attributes() {
   std::call_once(g_attr_once, [] {
-    cudaError_t e = cudaFuncSetAttribute(k_score, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kScoreSmem);
+    cudaError_t e = cudaFuncSetAttribute(k_score8, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kI8Smem);
     if (e == cudaSuccess)
       e = cudaFuncSetAttribute(k_sparse_attn, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kAttnSmem);
     if (e == cudaSuccess)
@@ -267,7 +277,7 @@ s2o_status s2o_plan_workspace_size(const s2o_config* cfg, size_t* bytes) {
 
 static void launch_plan_core(const s2o_config* cfg, const double* qbar, const uint16_t* K, float* scores,
                              int32_t* perm, int32_t* nblocks, float* seg_stats, const PlanWs& w, cudaStream_t s,
-                             int filtered);
+                             int filtered, bool key_digits);
 
 // the plan's launches; `filtered` sorts only the prefix of each segment's
 // order that the stop rule can reach
@@ -292,7 +302,7 @@ static s2o_status run_plan(const s2o_config* cfg, const uint16_t* Q, const uint1
   k_pool<<<dim3(S, BH), 256, 0, s>>>(Q, w.qbar, cfg->Hq, cfg->Hkv, cfg->N, S);
   ++t_launches;
   stage_mark(s, "k_pool");
-  launch_plan_core(cfg, w.qbar, K, scores, perm, nblocks, seg_stats, w, s, filtered);
+  launch_plan_core(cfg, w.qbar, K, scores, perm, nblocks, seg_stats, w, s, filtered, true);
   return launch_status();
 }
 
@@ -300,17 +310,40 @@ static s2o_status run_plan(const s2o_config* cfg, const uint16_t* Q, const uint1
 // partials, (M, Z), the order (bucketed sort, global fallback), the stop
 static void launch_plan_core(const s2o_config* cfg, const double* qbar, const uint16_t* K, float* scores,
                              int32_t* perm, int32_t* nblocks, float* seg_stats, const PlanWs& w, cudaStream_t s,
-                             int filtered) {
+                             int filtered, bool key_digits) {
   const int S = nseg(cfg);
   const int BH = cfg->B * cfg->Hkv;
   const int64_t T = ncand_total(cfg);
-  // (chunk, tile) pairs on or below the causal diagonal: chunk c reaches tiles t < min(S, 64 (c + 1))
-  const int nchunks = (S + kScoreSegs - 1) / kScoreSegs;
-  int pairs = 0;
-  for (int c = 0; c < nchunks; ++c) pairs += min(S, kScoreSegs * (c + 1));
-  k_score<<<dim3(pairs, BH), 256, kScoreSmem, s>>>(K, qbar, scores, w.part, cfg->Hkv, cfg->N, S, T);
+  I8Geom g;
+  g.S = S;
+  g.N = cfg->N;
+  g.nsb = (S + 127) / 128;
+  g.ntiles = (cfg->N + kI8TileKeys - 1) / kI8TileKeys;
+  if (key_digits) {
+    k_kdig<<<dim3(g.ntiles, BH), 256, 0, s>>>(K, w.kd, w.kexp, cfg->N);
+    ++t_launches;
+    stage_mark(s, "k_kdig");
+  }
+  k_qdig<<<(BH * S * 32 + 255) / 256, 256, 0, s>>>(qbar, w.qd, w.qexp, BH * S);
   ++t_launches;
-  stage_mark(s, "k_score");
+  stage_mark(s, "k_qdig");
+  // work units: (b*Hkv, 128-segment block, run of wu 128-key windows); wu is
+  // the largest power of two up to 32 that still gives two units per SM
+  int dev = 0, nsm = 148;
+  if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&nsm, cudaDevAttrMultiProcessorCount, dev);
+  auto units_for = [&](int wu) {
+    int n = 0;
+    for (int sb = 0; sb < g.nsb; ++sb) n += (i8_windows(g, sb) + wu - 1) / wu;
+    return n;
+  };
+  g.wu = 32;
+  while (g.wu > 1 && (int64_t)BH * units_for(g.wu) < 2 * nsm) g.wu >>= 1;
+  g.units_per_bk = units_for(g.wu);
+  const int total_units = BH * g.units_per_bk;
+  k_score8<<<min(total_units, nsm), kI8Threads, kI8Smem, s>>>(w.kd, w.kexp, w.qd, w.qexp, scores, w.part, g, T,
+                                                              total_units);
+  ++t_launches;
+  stage_mark(s, "k_score8");
   const int nwarps = BH * S;
   k_seg_stats<<<(nwarps * 32 + 255) / 256, 256, 0, s>>>(w.part, w.segM, w.segZ, seg_stats, BH, S);
   ++t_launches;
@@ -379,9 +412,9 @@ s2o_status s2o_plan_qperm(const s2o_config* cfg, const uint16_t* Q, const uint16
   ++t_launches;
   k_qperm<<<dim3(S, BH), kLq, 0, s>>>(Q, w.qbar, qsub0, qsub1, rowsub, cfg->Hq, cfg->Hkv, cfg->N, S);
   ++t_launches;
-  launch_plan_core(cfg, qsub0, K, scores, perm, nblocks, nullptr, w, s, 1);
+  launch_plan_core(cfg, qsub0, K, scores, perm, nblocks, nullptr, w, s, 1, true);
   launch_plan_core(cfg, qsub1, K, scores + (size_t)BH * T, perm + (size_t)BH * T, nblocks + (size_t)BH * S, nullptr,
-                   w, s, 1);
+                   w, s, 1, false);  // same keys: their digits are already in the workspace
   return launch_status();
 }
 

@@ -27,6 +27,32 @@ from oracle import s2o_oracle as O
 MAX_ABS = 1.5e-2
 REL_RMS = 4e-3
 
+
+def score_error_bound(qbar: np.ndarray, Kf: np.ndarray) -> np.ndarray:
+    """Bound on |GPU score - exact score| beyond fp32 rounding, per key row.
+
+    The GPU scores in fixed point (the integer tensor-core scorer): qbar is
+    rounded to a multiple of 2^(f-28), f = floor(log2 max|qbar|); each key
+    element to a multiple of 2^(E-148), E = max(1, biased bf16 exponent of
+    the row's largest magnitude), which changes only elements below
+    2^(E-141); one digit product of weight 2^(f+E-176) is left out.  The
+    three terms are
+        [2^(f-29) ||k||_1 + 2^(E-149) sum_{d: |k_d| < 2^(E-141)} |qbar_d|
+         + 2^(f+E-156)] / sqrt(d).
+    Kf: [n, d] fp64 key rows (bf16 values).  The 1e-6 x max|s| near-tie band
+    of the order is three orders above this for bf16 data of any scale.
+    """
+    Kf = np.asarray(Kf, dtype=np.float64)
+    mq = float(np.max(np.abs(qbar))) if qbar.size else 0.0
+    f = (np.frexp(mq)[1] - 1) if mq > 0 else 0
+    mk = np.max(np.abs(Kf), axis=1)
+    E = np.where(mk >= 2.0 ** -126, np.frexp(np.maximum(mk, 2.0 ** -126))[1] + 126, 1)
+    d = Kf.shape[1]
+    small = np.abs(Kf) < np.ldexp(1.0, E - 141)[:, None]
+    b = (np.ldexp(1.0, f - 29) * np.abs(Kf).sum(axis=1) + np.ldexp(1.0, E - 149) * (small @ np.abs(qbar))
+         + np.ldexp(1.0, f + E - 156))
+    return b / np.sqrt(d)
+
 # allowances used in this process: segments compared, positions holding a
 # different (near-tied) key, and blocks between differing stop points
 TOTALS = {"segments": 0, "swapped_positions": 0, "C_flips": 0, "online_C_flips": 0, "cases": 0}

@@ -59,13 +59,19 @@ def check_plan(Q, K, cfg, bufs, p, segments=None, kvheads=None, what="", prefix_
             sp = O.plan_segment(Q, K, b, kvh, s, G, p)
             plans[(b, kvh, s)] = sp
             lo, hi = O.candidate_range(cfg.N, s, p)
-            # scores are the fp64 values rounded once to fp32 (half an ulp)
+            # scores: the exact values rounded to fp32 (half an ulp), plus the
+            # fixed-point representation's bound
+            e = len(sp.scores)
+            bound = parity.score_error_bound(sp.qbar, O.widen_bf16(K[b, kvh, :e]) if K.dtype == np.uint16
+                                             else K[b, kvh, :e])
             gs = scores[b, kvh, off[s]:off[s + 1]].astype(np.float64)
             ref = sp.scores[lo:hi]
             half_ulp = 0.5 * np.spacing(np.abs(ref).astype(np.float32)).astype(np.float64)
-            assert np.all(np.abs(gs - ref) <= half_ulp + 1e-13 * np.abs(ref) + 1e-300)
-            assert abs(stats[b, kvh, s, 0] - sp.M) <= 0.5 * float(np.spacing(np.float32(abs(sp.M)))) + 1e-13 * abs(sp.M)
-            assert abs(stats[b, kvh, s, 1] / sp.Z - 1.0) <= 1e-5
+            assert np.all(np.abs(gs - ref) <= half_ulp + bound[lo:hi] + 1e-300)
+            # (in fp64: numpy keeps float32 - float in float32)
+            assert abs(float(stats[b, kvh, s, 0]) - sp.M) <= (0.5 * float(np.spacing(np.float32(abs(sp.M))))
+                                                              + float(bound.max(initial=0.0)))
+            assert abs(float(stats[b, kvh, s, 1]) / sp.Z - 1.0) <= 1e-5
             sw, fl = parity.compare_segment_plan(perm[b, kvh, off[s]:off[s + 1]], int(nb[b, kvh, s]), sp, p,
                                                  prefix_only=prefix_only)
             swaps += sw
