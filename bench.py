@@ -139,10 +139,11 @@ def plan_kernel_roofline(s2o, torch, cfg, Q, K, bufs, filtered, w, peaks, peak_s
     S = (N + 127) // 128
     T = B * Hkv * ((64 * (S - 2) ** 2) if S >= 2 else 0)
     L = prefix_lengths(torch, cfg, bufs, filtered, w)
-    parts = B * Hkv * S * (S + 1) / 2 * 8
-    ntiles = (N + 31) // 32
-    kdig = B * Hkv * ntiles * (3 * 32 * 128 + 32 * 4)
-    qdig = B * Hkv * S * (4 * 128 + 4)
+    # (max, sum exp) partials: one per (segment, 96-key tile holding admissible keys)
+    parts = B * Hkv * sum((min(N, 128 * (s + 1)) + 95) // 96 for s in range(S)) * 8
+    ntiles = (N + 95) // 96
+    kdig = B * Hkv * ntiles * (3 * 96 * 128 + 100 * 4)
+    qdig = B * Hkv * (((S + 127) // 128) * 128 * 4 * 128 + S * 4)
     bytes_of = {
         "k_pool": B * Hq * N * d * 2 + B * Hkv * S * d * 8,
         "k_kdig": B * Hkv * N * d * 2 + kdig,

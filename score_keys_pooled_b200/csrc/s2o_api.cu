@@ -77,7 +77,9 @@ PlanWs plan_layout(const s2o_config* c, void* base) {
     return static_cast<void*>(p);
   };
   w.qbar = static_cast<double*>(take(BH * S * kD * sizeof(double)));
-  w.part = static_cast<float2*>(take(BH * S * S * sizeof(float2)));
+  const size_t ntiles = ((size_t)c->N + kI8TileKeys - 1) / kI8TileKeys;
+  const size_t nsb = (S + 127) / 128;
+  w.part = static_cast<float2*>(take(BH * S * ntiles * sizeof(float2)));
   w.segM = static_cast<float*>(take(BH * S * sizeof(float)));
   w.segZ = static_cast<double*>(take(BH * S * sizeof(double)));
   w.keyA = static_cast<uint32_t*>(take(BH * T * 4 + 16));
@@ -92,10 +94,9 @@ PlanWs plan_layout(const s2o_config* c, void* base) {
   w.mode = static_cast<int*>(take(BH * S * sizeof(int)));
   w.plen = static_cast<int*>(take(BH * S * sizeof(int)));
   w.range = static_cast<float2*>(take(BH * S * sizeof(float2)));
-  const size_t ntiles = ((size_t)c->N + kI8TileKeys - 1) / kI8TileKeys;
   w.kd = static_cast<uint8_t*>(take(BH * ntiles * kI8TileBytes));
-  w.kexp = static_cast<int32_t*>(take(BH * ntiles * kI8TileKeys * sizeof(int32_t)));
-  w.qd = static_cast<uint8_t*>(take(BH * S * kI8QRowBytes));
+  w.kexp = static_cast<int32_t*>(take(BH * ntiles * kI8ExpRec * sizeof(int32_t)));
+  w.qd = static_cast<uint8_t*>(take(BH * nsb * kI8QBytes));
   w.qexp = static_cast<int32_t*>(take(BH * S * sizeof(int32_t)));
   w.bytes = off;
   return w;
@@ -324,16 +325,16 @@ static void launch_plan_core(const s2o_config* cfg, const double* qbar, const ui
     ++t_launches;
     stage_mark(s, "k_kdig");
   }
-  k_qdig<<<(BH * S * 32 + 255) / 256, 256, 0, s>>>(qbar, w.qd, w.qexp, BH * S);
+  k_qdig<<<(BH * g.nsb * 128 * 32 + 255) / 256, 256, 0, s>>>(qbar, w.qd, w.qexp, BH, S, g.nsb);
   ++t_launches;
   stage_mark(s, "k_qdig");
-  // work units: (b*Hkv, 128-segment block, run of wu 128-key windows); wu is
+  // work units: (b*Hkv, 128-segment block, run of wu 96-key tiles); wu is
   // the largest power of two up to 32 that still gives two units per SM
   int dev = 0, nsm = 148;
   if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&nsm, cudaDevAttrMultiProcessorCount, dev);
   auto units_for = [&](int wu) {
     int n = 0;
-    for (int sb = 0; sb < g.nsb; ++sb) n += (i8_windows(g, sb) + wu - 1) / wu;
+    for (int sb = 0; sb < g.nsb; ++sb) n += (i8_tiles(g, sb) + wu - 1) / wu;
     return n;
   };
   g.wu = 32;
@@ -345,7 +346,8 @@ static void launch_plan_core(const s2o_config* cfg, const double* qbar, const ui
   ++t_launches;
   stage_mark(s, "k_score8");
   const int nwarps = BH * S;
-  k_seg_stats<<<(nwarps * 32 + 255) / 256, 256, 0, s>>>(w.part, w.segM, w.segZ, seg_stats, BH, S);
+  k_seg_stats<kI8TileKeys><<<(nwarps * 32 + 255) / 256, 256, 0, s>>>(w.part, w.segM, w.segZ, seg_stats, BH, S,
+                                                                      cfg->N, g.ntiles);
   ++t_launches;
   stage_mark(s, "k_seg_stats");
   k_bucket_plan<<<BH * S, kBucketThreads, 0, s>>>(scores, w.sorted, perm, w.slots, w.mode, w.range, w.keyB, w.valB,

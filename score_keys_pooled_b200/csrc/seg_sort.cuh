@@ -31,21 +31,25 @@ __device__ __forceinline__ float key_score(uint32_t k) {
 }
 
 // ---------------------------------------------------------------------------
-// (M, Z) per segment from the per-tile partials; one warp per segment.
+// (M, Z) per segment from the per-tile partials (max, sum exp) of the scorer:
+// tiles of kTile keys, row stride `ntiles`, the first ceil(e(s) / kTile)
+// entries of a row filled; one warp per segment.
 // ---------------------------------------------------------------------------
+template <int kTile>
 __global__ void k_seg_stats(const float2* __restrict__ part, float* __restrict__ segM, double* __restrict__ segZ,
-                            float* __restrict__ seg_stats, int BHkv, int S) {
+                            float* __restrict__ seg_stats, int BHkv, int S, int N, int ntiles) {
   const int warp = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
   const int lane = threadIdx.x & 31;
   if (warp >= BHkv * S) return;
   const int bk = warp / S, s = warp % S;
-  const float2* p = part + ((size_t)bk * S + s) * S;
+  const float2* p = part + ((size_t)bk * S + s) * ntiles;
+  const int nt = (min(N, kLq * (s + 1)) + kTile - 1) / kTile;
   float m = -INFINITY;
-  for (int t = lane; t <= s; t += 32) m = fmaxf(m, p[t].x);
+  for (int t = lane; t < nt; t += 32) m = fmaxf(m, p[t].x);
 #pragma unroll
   for (int o = 16; o >= 1; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
   double z = 0.0;
-  for (int t = lane; t <= s; t += 32) z += (double)p[t].y * exp((double)p[t].x - (double)m);
+  for (int t = lane; t < nt; t += 32) z += (double)p[t].y * exp((double)p[t].x - (double)m);
 #pragma unroll
   for (int o = 16; o >= 1; o >>= 1) z += __shfl_xor_sync(0xffffffffu, z, o);
   if (lane == 0) {

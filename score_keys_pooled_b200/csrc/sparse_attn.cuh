@@ -109,12 +109,6 @@ __device__ __forceinline__ void load_kv_tile(uint32_t dst, const uint16_t* src_h
   }
 }
 
-__device__ __forceinline__ float ex2_approx(float x) {
-  float y;
-  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
-  return y;
-}
-
 __global__ void __launch_bounds__(kAttnThreads, 2) k_sparse_attn(AttnArgs a) {
   extern __shared__ uint8_t smem_raw[];
   const uint32_t sbase = (smem_u32(smem_raw) + 1023u) & ~1023u;
