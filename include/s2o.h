@@ -167,7 +167,7 @@ s2o_status s2o_plan_filtered(const s2o_config* cfg, const uint16_t* Q, const uin
  *   Scratch: a 32 MiB array in the library's device memory (a file-scope
  *   __device__ buffer that every GPU loading the library holds until the
  *   process exits).  Configs whose plan workspace (s2o_plan_workspace_size)
- *   exceeds 32 MiB -- e.g. B=1, 8 KV heads, N above ~7K -- are rejected with
+ *   exceeds 32 MiB -- e.g. B=1, 8 KV heads, N above ~5K -- are rejected with
  *   S2O_ERR_WORKSPACE_TOO_SMALL before anything is launched.
  *   The 32 MiB are committed by the driver when the library's device code is
  *   loaded into a context: with lazy loading (the default since CUDA 12.2)
