@@ -567,6 +567,8 @@ def main():
     ap.add_argument("--online-steps", type=int, default=3,
                     help="steps of the run-time stop variant (full plan + s2o_attention_online), reported beside "
                          "the headline; 0 skips it")
+    ap.add_argument("--graph", action=argparse.BooleanOptionalAction, default=False,
+                    help="replay the timed step's plan and attention as CUDA graphs instead of launching them")
     ap.add_argument("--plan", default="filtered", choices=["full", "filtered"],
                     help="s2o_plan (every segment fully ordered) or s2o_plan_filtered (only the prefix the "
                          "stop rule can reach; same kept sets and output)")
@@ -644,6 +646,28 @@ def main():
     if st != 0:
         raise RuntimeError(f"device error after warm-up: {s2o.status_string(st)}")
 
+    # the step's launches, captured once as two CUDA graphs (plan, attention)
+    # and replayed: the same kernels on the same buffers, without the host's
+    # per-launch gaps between them
+    plan_run = lambda: s2o.plan(cfg, Q, K, bufs, filtered=filtered)
+    attn_run = lambda: s2o.attention(cfg, Q, K, V, bufs["perm"], bufs["nblocks"], O)
+    n_plan, n_attn = 0, 0
+    if args.graph:
+        g_plan, g_attn = torch.cuda.CUDAGraph(), torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g_plan):
+            plan_run()
+            n_plan = s2o.last_launch_count()
+        with torch.cuda.graph(g_attn):
+            attn_run()
+            n_attn = s2o.last_launch_count()
+        plan_run, attn_run = g_plan.replay, g_attn.replay
+        for _ in range(2):
+            plan_run()
+            attn_run()
+        st = s2o.last_device_error()
+        if st != 0:
+            raise RuntimeError(f"device error in the graph warm-up: {s2o.status_string(st)}")
+
     ev = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(args.steps)]
     launches = 0
     if dist:
@@ -655,11 +679,11 @@ def main():
         t_start.record(stream)
         for k in range(args.steps):
             ev[k][0].record(stream)
-            s2o.plan(cfg, Q, K, bufs, filtered=filtered)
-            launches += s2o.last_launch_count()
+            plan_run()
+            launches += n_plan if args.graph else s2o.last_launch_count()
             ev[k][1].record(stream)
-            s2o.attention(cfg, Q, K, V, bufs["perm"], bufs["nblocks"], O)
-            launches += s2o.last_launch_count()
+            attn_run()
+            launches += n_attn if args.graph else s2o.last_launch_count()
             ev[k][2].record(stream)
         t_end.record(stream)
         torch.cuda.synchronize()
@@ -846,7 +870,7 @@ def main():
             "attention_only_tflops": job_tflops(attn_mean),
             "kept_pair_fraction": density, "accuracy": accuracy,
             "roofline": roofline, "plan_roofline": plan_roofline,
-            "cpu_baseline": cpu, "e2e": e2e, "gpu_launches": launches,
+            "cpu_baseline": cpu, "e2e": e2e, "gpu_launches": launches, "launch_mode": "cuda graph replay" if args.graph else "eager",
             "clocks": clk.summary(),
         }
         print(json.dumps(line), flush=True)

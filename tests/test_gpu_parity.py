@@ -156,6 +156,39 @@ def test_all_ties_bit_exact(tau):
         assert stats[0, 0, s, 0] == 0.0 and stats[0, 0, s, 1] == float(e)
 
 
+@pytest.mark.parametrize("seed", [41, 42])
+def test_scores_across_wide_exponent_ranges(seed):
+    """Inputs that strain the scorer's fixed point: key rows whose elements
+    span up to 80 binades (most of a row's small elements are rounded), rows
+    with a single nonzero element, rows of bf16 subnormals and zeros, and
+    pooled queries from 2^-100 to 2^40 in scale.  Scores must stay within half
+    an ulp plus the representation bound of the exact values, and the order,
+    M, Z and C(s) must match the oracle as everywhere else."""
+    B, Hq, Hkv, N, tau = 1, 4, 2, 1280, 1e-3
+    Q, K, V = synth.generate(B, Hq, Hkv, N, 128, planted=True, band=True, n_stripe=8, seed=seed)
+    rng = np.random.default_rng(seed)
+    Kf = O.widen_bf16(K).astype(np.float32)
+    # per-element scales 2^e, e uniform in [-40, 40], on a third of the rows
+    rows = rng.random(N) < 1 / 3
+    Kf[:, :, rows] *= np.exp2(rng.integers(-40, 41, size=(B, Hkv, int(rows.sum()), 128))).astype(np.float32)
+    # single-element rows and subnormal rows
+    for j in rng.choice(np.arange(64, N), size=24, replace=False):
+        Kf[:, :, j] = 0.0
+        Kf[:, :, j, rng.integers(0, 128)] = rng.choice([-1.0, 1.0]) * np.float32(2.0 ** rng.integers(-30, 30))
+    for j in rng.choice(np.arange(64, N), size=8, replace=False):
+        Kf[:, :, j] = rng.standard_normal(128).astype(np.float32) * np.float32(2.0 ** -130)
+    K = synth.to_bf16_bits(Kf)
+    # pooled queries of very different scales, one segment each
+    Qf = O.widen_bf16(Q).astype(np.float32)
+    for s, e in ((2, -100), (3, -20), (5, 20), (7, 40)):
+        Qf[:, :, 128 * s:128 * s + 128] *= np.float32(2.0 ** e)
+    Q = synth.to_bf16_bits(Qf)
+    cfg = s2o.make_config(B, Hq, Hkv, N, tau=tau)
+    bufs = s2o.plan(cfg, dev(Q), dev(K))
+    assert s2o.last_device_error() == 0
+    check_plan(Q, K, cfg, bufs, O.Params(tau=tau), what=f"wide exponents seed={seed}")
+
+
 @pytest.mark.parametrize("world", [2, 3, 8])
 def test_kv_head_shards_reassemble_the_whole_problem(world):
     """One problem sharded by KV head (bench.py --shard heads): every rank's
