@@ -131,6 +131,15 @@ s2o_status s2o_plan_workspace_size(const s2o_config* cfg, size_t* bytes);
  *   seg_stats  out, device fp32 [B,Hkv,S,2] or NULL
  *   workspace  device scratch of at least s2o_plan_workspace_size() bytes,
  *              256-byte aligned; its contents need no initialisation
+ * Accuracy: a score is the exact qbar . k_j / sqrt(d) (qbar the exact mean of
+ * the bf16 rows) to within half an fp32 ulp plus
+ *   [2^(f-29) |k_j|_1 + 2^(E-149) sum_{d: |k_jd| < 2^(E-141)} |qbar_d|
+ *    + 2^(f+E-156)] / sqrt(d),
+ * f = floor(log2 max|qbar|), E = the biased bf16 exponent of max|k_j| (at
+ * least 1): qbar and k_j are taken in fixed point against their own largest
+ * exponents (29 and 22 bits) and multiplied exactly on the integer tensor
+ * core; about 1e-9 of |qbar| |k_j|.  The order sorts these fp32 values,
+ * ties to the lower key index; M and Z (seg_stats) are formed from them.
  */
 s2o_status s2o_plan(const s2o_config* cfg, const uint16_t* Q, const uint16_t* K,
                     float* scores, int32_t* perm, int32_t* nblocks, float* seg_stats,
