@@ -29,7 +29,7 @@
 // Kernels:
 //   k_kdig   K -> key digits, per 96-key tile already in the tensor core's
 //            128B-swizzled K-major layout (3 digit planes x 96 rows x 128 B),
-//            and E_j per key;
+//            and E_j per key followed by the tile's largest E_j;
 //   k_qdig   qbar -> query digits, per block of 128 segments in the same
 //            layout (4 planes x 128 rows x 128 B), and f per segment;
 //   k_score8 one persistent CTA per SM.  A work unit is (b*Hkv, block of 128
