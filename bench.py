@@ -84,10 +84,10 @@ def kept_pairs_qperm(nblocks2: np.ndarray, rowsub: np.ndarray, N: int, G: int) -
 
 # DRAM bytes (read + write) per k_sparse_attn2 launch from an ncu capture of
 # the current kernel, by workload.  llama_128k: the capture of llama_32k at
-# the same kept fraction (tau = 4e-3, 26.7 % of pairs; 669.8 MB) scaled by the
-# rows processed (x 4: Q, O, K and V all grow with N).  None where no capture
-# exists.
-ATTN_TRAFFIC = {"llama_128k": 2.679e9, "llama_32k@0.004": 6.698e8}
+# the same kept fraction (tau = 4e-3, 26.7 % of pairs; 436.8 + 232.7 MB)
+# scaled by the rows processed (x 4: Q, O, K and V all grow with N).  None
+# where no capture exists.
+ATTN_TRAFFIC = {"llama_128k": 2.678e9, "llama_32k@0.004": 6.695e8}
 
 # int8 tensor-core rate relative to the measured bf16 rate: the nominal dense
 # ratio of B200 (4.5 POPS int8 / 2.25 PFLOP/s bf16)
