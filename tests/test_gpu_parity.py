@@ -110,6 +110,7 @@ SMALL = [
     (1, 4, 1, 1000, 1e-2, True, True),
     (1, 4, 1, 1111, 5e-3, False, False),
     (1, 4, 4, 640, 1e-3, True, True),
+    (1, 6, 2, 900, 3e-3, True, True),  # G = 3: the odd-group kernel
 ]
 
 
@@ -236,7 +237,7 @@ def test_out_of_range_plan_is_clamped_and_reported():
 
 
 @pytest.mark.parametrize("B,Hq,Hkv,N,out_dtype", [(1, 8, 2, 1536, s2o.OUT_BF16), (2, 4, 2, 1000, s2o.OUT_F32),
-                                                  (2, 4, 4, 640, s2o.OUT_BF16)])
+                                                  (2, 4, 4, 640, s2o.OUT_BF16), (1, 6, 2, 900, s2o.OUT_BF16)])
 def test_host_buffer_entry_matches_device_path(B, Hq, Hkv, N, out_dtype):
     # the host entry pipelines its work by (b, kvh) over three streams; the
     # result must equal the device path bit for bit
