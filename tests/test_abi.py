@@ -82,3 +82,18 @@ def test_workspace_size_grows_with_candidates(L):
     cfg = s2o.make_config(1, 32, 8, 131072)
     # 4 sort buffers of 4 bytes per candidate dominate
     assert s2o.plan_workspace_size(cfg) >= 16 * 8 * s2o.num_candidates(cfg)
+
+
+def test_noalloc_rejects_configs_over_its_scratch(L):
+    """s2o_plan_noalloc refuses, before any CUDA call, every config whose plan
+    workspace exceeds its 32 MiB scratch; the header's example (B = 1, 8 KV
+    heads: N above about 5K) holds for the current workspace layout (the key
+    digits take 384 bytes per key and KV head)."""
+    limit = 32 << 20
+    P = ctypes.c_void_p
+    good = P(1 << 20)
+    assert s2o.plan_workspace_size(s2o.make_config(1, 32, 8, 5120)) <= limit
+    for N in (5504, 8192, 131072):
+        cfg = s2o.make_config(1, 32, 8, N)
+        assert s2o.plan_workspace_size(cfg) > limit
+        assert L.s2o_plan_noalloc(ctypes.byref(cfg), good, good, good, good, good, None, None) == 3
