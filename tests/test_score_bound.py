@@ -54,8 +54,11 @@ def _model_scores(qbar, kbits):
     G = np.rint(qbar * 2.0 ** (28 - f)).astype(np.int64)
     qd = _signed_digits(G, 4)
     kd = _signed_digits(F, 3)
+    assert np.abs(kd[0]).max() <= 64 and np.abs(qd[0]).max() <= 33
+    assert all(np.abs(x).max() <= 128 for x in kd[1:] + qd[1:])
     S = [sum(kd[b] @ qd[t - b] for b in range(3) if 0 <= t - b <= 3) for t in range(5)]
     Y = (S[0] * 256 + S[1]) * 2 ** 24 + (S[2] * 256 + S[3]) * 256 + S[4]
+    assert np.abs(Y).max() < 2 ** 51
     s64 = Y.astype(np.float64) * np.ldexp(math.sqrt(2.0), (f + E - 172).astype(np.int64))
     return s64.astype(np.float32).astype(np.float64)
 
@@ -109,3 +112,35 @@ def test_the_bound_is_needed():
     got = _model_scores(qbar, kbits)
     half_ulp = 0.5 * np.spacing(np.abs(exact).astype(np.float32)).astype(np.float64)
     assert np.any(np.abs(got - exact) > half_ulp + 1e-13 * np.abs(exact))
+
+
+def test_digit_ranges_keep_accumulators_exact():
+    """The scheme's integer ranges: key digits |d0| <= 64, |d1|, |d2| <= 128;
+    query digits |c0| <= 33, |c1..c3| <= 128; so every S_t (a sum of at most
+    three 128-term digit products) fits int32, hi = 256 S0 + S1 and
+    mid = 256 S2 + S3 fit int32, and |Y| < 2^51 (Y converts to fp64
+    exactly).  Checked from the ranges and on extreme inputs."""
+    dmax = [64, 128, 128]
+    cmax = [33, 128, 128, 128]
+    S = [sum(128 * cmax[t - b] * dmax[b] for b in range(3) if 0 <= t - b <= 3) for t in range(5)]
+    hi, mid = 256 * S[0] + S[1], 256 * S[2] + S[3]
+    Y = hi * 2 ** 24 + mid * 256 + S[4]
+    assert max(S) < 2 ** 31 and hi < 2 ** 31 and mid < 2 ** 31
+    assert Y < 2 ** 51
+    # extreme rows: every element at the row maximum (largest top digits) or
+    # alternating signs, with the query at the top of its range
+    rng = np.random.default_rng(5)
+    for sign in (1.0, -1.0):
+        K = np.full((8, 128), 3.0e38 * sign, dtype=np.float32)
+        K[1::2, ::2] *= -1
+        K[4:] = rng.choice([-1.0, 1.0], size=(4, 128)) * np.float32(1.9921875)  # mantissa all ones
+        kbits = synth.to_bf16_bits(K)
+        qbar = np.full(128, 1.999999) * sign
+        qbar[::3] *= -1
+        with np.errstate(over="ignore"):  # rows of 3e38 overflow fp32 (the kernel flags those)
+            got = _model_scores(qbar, kbits)  # asserts inside check the digit ranges
+            exact = O.widen_bf16(kbits) @ qbar / math.sqrt(128)
+            fin = np.isfinite(exact.astype(np.float32))
+            half_ulp = 0.5 * np.spacing(np.abs(exact).astype(np.float32)).astype(np.float64)
+        bound = parity.score_error_bound(qbar, O.widen_bf16(kbits))
+        assert np.all(np.abs(got[fin] - exact[fin]) <= half_ulp[fin] + bound[fin])
