@@ -325,7 +325,7 @@ static void launch_plan_core(const s2o_config* cfg, const double* qbar, const ui
     ++t_launches;
     stage_mark(s, "k_kdig");
   }
-  k_qdig<<<(BH * g.nsb * 128 * 32 + 255) / 256, 256, 0, s>>>(qbar, w.qd, w.qexp, BH, S, g.nsb);
+  k_qdig<<<BH * g.nsb * 16, 256, 0, s>>>(qbar, w.qd, w.qexp, BH, S, g.nsb);  // a warp per segment row
   ++t_launches;
   stage_mark(s, "k_qdig");
   // work units: (b*Hkv, 128-segment block, run of wu 96-key tiles); wu is
@@ -346,7 +346,7 @@ static void launch_plan_core(const s2o_config* cfg, const double* qbar, const ui
   ++t_launches;
   stage_mark(s, "k_score8");
   const int nwarps = BH * S;
-  k_seg_stats<kI8TileKeys><<<(nwarps * 32 + 255) / 256, 256, 0, s>>>(w.part, w.segM, w.segZ, seg_stats, BH, S,
+  k_seg_stats<kI8TileKeys><<<(nwarps + 7) / 8, 256, 0, s>>>(w.part, w.segM, w.segZ, seg_stats, BH, S,
                                                                       cfg->N, g.ntiles);
   ++t_launches;
   stage_mark(s, "k_seg_stats");

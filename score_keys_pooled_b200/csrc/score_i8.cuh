@@ -214,7 +214,7 @@ __global__ void __launch_bounds__(256) k_kdig(const uint16_t* __restrict__ K, ui
 // ---------------------------------------------------------------------------
 __global__ void __launch_bounds__(256) k_qdig(const double* __restrict__ qbar, uint8_t* __restrict__ qd,
                                              int32_t* __restrict__ qexp, int BH, int S, int nsb) {
-  const int gw = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
+  const int gw = (int)(((unsigned long long)blockIdx.x * blockDim.x + threadIdx.x) >> 5);
   const int lane = threadIdx.x & 31;
   if (gw >= BH * nsb * 128) return;
   const int bk = gw / (nsb * 128), rem = gw - bk * nsb * 128;

@@ -38,7 +38,7 @@ __device__ __forceinline__ float key_score(uint32_t k) {
 template <int kTile>
 __global__ void k_seg_stats(const float2* __restrict__ part, float* __restrict__ segM, double* __restrict__ segZ,
                             float* __restrict__ seg_stats, int BHkv, int S, int N, int ntiles) {
-  const int warp = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
+  const int warp = (int)(((unsigned long long)blockIdx.x * blockDim.x + threadIdx.x) >> 5);
   const int lane = threadIdx.x & 31;
   if (warp >= BHkv * S) return;
   const int bk = warp / S, s = warp % S;
